@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the causal sliding-window attention hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+  * the depth-24 shape (B=32, T=2048, H=12, D=128) through the "SSSL" window
+    pattern (three layers at W=512, one at W=2048): forward (O, lse) and
+    backward (dQ, dK, dV) per layer;
+  * single-token decode over the KV-cache workload (32 sequences, H=12,
+    D=128, capacity 2048, cache_len ~ U[1, 2048]) at W=2048 and W=1024.
+value = unmasked fwd+bwd FLOPs of the step / step time (decode time included).
+FLOPs count only (i, j) pairs inside the band: 4*D per pair forward, 10*D per
+pair backward (five matmuls with the recomputed scores).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs its own independent batch (weak scaling, no data-path collective) and
+the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd+bwd TFLOP/s (unmasked FLOPs) & % BF16 peak; decode HBM GB/s"
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def band_pairs(T: int, W: int) -> int:
+    """Number of (i, j) pairs with i - W < j <= i, 0 <= j <= i < T."""
+    if W >= T:
+        return T * (T + 1) // 2
+    return W * (W + 1) // 2 + (T - W) * W
+
+
+def fwd_flops(B, T, H, D, W):
+    return 4 * D * B * H * band_pairs(T, W)
+
+
+def bwd_flops(B, T, H, D, W):
+    return 10 * D * B * H * band_pairs(T, W)
+
+
+def decode_bytes(cache_len, H, D, W):
+    n = np.minimum(cache_len.astype(np.int64), W)
+    B = len(cache_len)
+    return int(n.sum()) * H * D * 2 * 2 + 2 * B * H * D * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling of one GPU while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, path: str | None):
+        self.proc = None
+        self.path = path
+        try:
+            self.out = open(path, "w") if path else subprocess.PIPE
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            text = ""
+        if self.path:
+            self.out.close()
+            text = open(self.path).read()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (text or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        load = [s for s in sm if smax and s > 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(dev) -> str:
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+def make_inputs(rank: int):
+    from causal_sliding_window_b200 import inputs
+
+    cfg = inputs.WORKLOADS["d24"]
+    att = inputs.attention_inputs(cfg["B"], cfg["T"], cfg["H"], cfg["D"], seed=cfg["seed"] + 1000 * rank)
+    dc = inputs.DECODE_WORKLOAD
+    dec = inputs.decode_inputs(dc["B"], dc["cap"], dc["H"], dc["D"], seed=dc["seed"] + 1000 * rank)
+    return cfg, att, dc, dec
+
+
+def to_bf16(bits, device, pin=False):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    if pin:
+        return t.pin_memory()
+    return t.to(device)
+
+
+def cpu_baseline_sample(cfg, att, heads=None):
+    """The oracle, as it stands, on sequence 0 (first `heads` heads) of the d24 SSSL step (fwd + bwd)."""
+    from oracle import oracle_bwd, oracle_fwd, oracle_threads
+
+    heads = cfg["H"] if heads is None else heads
+    q, k, v, do = (np.ascontiguousarray(att[n][:1, :, :heads]) for n in ("q", "k", "v", "do"))
+    B, T, H, D = 1, cfg["T"], heads, cfg["D"]
+    t0 = time.perf_counter()
+    flops = 0
+    for W in cfg["windows"]:
+        oracle_fwd(q, k, v, W)
+        oracle_bwd(q, k, v, do, W)
+        flops += fwd_flops(B, T, H, D, W) + bwd_flops(B, T, H, D, W)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"sequence 0 of the d24 batch (1 x {T} x {H} x {D}), SSSL windows {list(cfg['windows'])}, "
+                      f"fwd+bwd in fp64; {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    from causal_sliding_window_b200 import inputs
+
+    cfg = inputs.WORKLOADS["d24"]
+    att = inputs.attention_inputs(1, cfg["T"], cfg["H"], cfg["D"], seed=cfg["seed"])
+    heads = 2   # bounded sample per step: sequence 0, heads 0-1 (a few seconds of fp64 work)
+    for _ in range(args.warmup):
+        cpu_baseline_sample(cfg, att, heads)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        cb = cpu_baseline_sample(cfg, att, heads)
+        times.append(cb["seconds"])
+        flops = cb["value"] * 1e12 * cb["seconds"]
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"d24 SSSL fwd+bwd, bounded sample: sequence 0 of 32, heads 0-{heads - 1} of 12",
+                   "global_batch": 1, "seq_len": cfg["T"], "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    from causal_sliding_window_b200 import ops
+
+    cfg, att, dc, dec = make_inputs(rank)
+    B, T, H, D = cfg["B"], cfg["T"], cfg["H"], cfg["D"]
+    windows = list(cfg["windows"])
+    dwins = list(dc["windows"])
+    # Device-resident inputs and outputs.
+    q, k, v, do = (to_bf16(att[n], dev) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+    dB, cap, dH, dD = dc["B"], dc["cap"], dc["H"], dc["D"]
+    dq_in = to_bf16(dec["q"], dev)
+    kc, vc = to_bf16(dec["k_cache"], dev), to_bf16(dec["v_cache"], dev)
+    cl = torch.from_numpy(dec["cache_len"]).to(dev)
+    d_o = torch.empty((dB, dH, dD), dtype=torch.bfloat16, device=dev)
+    d_lse = torch.empty((dB, dH), dtype=torch.float32, device=dev)
+    dws = ops.decode_workspace(dB, cap, dH, dD, dev)
+
+    stream = torch.cuda.current_stream()
+    step_flops = sum(fwd_flops(B, T, H, D, W) + bwd_flops(B, T, H, D, W) for W in windows)
+    step_fwd_flops = sum(fwd_flops(B, T, H, D, W) for W in windows)
+    step_bwd_flops = sum(bwd_flops(B, T, H, D, W) for W in windows)
+    step_dec_bytes = sum(decode_bytes(dec["cache_len"], dH, dD, W) for W in dwins)
+    launches_per_step = 4 * len(windows) + len(dwins)
+
+    def run_step(ev=None):
+        for li, W in enumerate(windows):
+            if ev is not None:
+                ev["f0"][li].record(stream)
+            ops.attn_fwd(q, k, v, o, lse, W, stream=stream)
+            if ev is not None:
+                ev["f1"][li].record(stream)
+                ops.attn_bwd_set_profile_events(ev["bp"][li], ev["bm"][li])
+            ops.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, W, stream=stream)
+            if ev is not None:
+                ops.attn_bwd_set_profile_events(None, None)
+                ev["b1"][li].record(stream)
+        for di, W in enumerate(dwins):
+            if ev is not None:
+                ev["d0"][di].record(stream)
+            ops.attn_decode(dq_in, kc, vc, cl, d_o, d_lse, dws, W, stream=stream)
+            if ev is not None:
+                ev["d1"][di].record(stream)
+
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0, "device wait timed out during warm-up"
+
+    mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]  # noqa: E731
+    evs = [{"f0": mk(len(windows)), "f1": mk(len(windows)), "bp": mk(len(windows)), "bm": mk(len(windows)),
+            "b1": mk(len(windows)), "d0": mk(len(dwins)), "d1": mk(len(dwins))} for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_uuid(dev), args.clock_log if rank == 0 else None)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for s in range(args.steps):
+        run_step(evs[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    status = ops.attn_device_status(clear=True)
+    assert status == 0, "device wait timed out during the timed region"
+    t_fwd = sum(e["f0"][i].elapsed_time(e["f1"][i]) for e in evs for i in range(len(windows)))
+    t_pre = sum(e["f1"][i].elapsed_time(e["bp"][i]) for e in evs for i in range(len(windows)))
+    t_bmain = sum(e["bp"][i].elapsed_time(e["bm"][i]) for e in evs for i in range(len(windows)))
+    t_conv = sum(e["bm"][i].elapsed_time(e["b1"][i]) for e in evs for i in range(len(windows)))
+    t_dec = sum(e["d0"][i].elapsed_time(e["d1"][i]) for e in evs for i in range(len(dwins)))
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    finite = bool(torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all()
+                  and torch.isfinite(d_o.float()).all())
+
+    # ---- end to end: host buffers in, results out, every step ----
+    host = {n: to_bf16(att[n], None, pin=True) for n in ("q", "k", "v", "do")}
+    host_dec = {"q": to_bf16(dec["q"], None, pin=True), "k": to_bf16(dec["k_cache"], None, pin=True),
+                "v": to_bf16(dec["v_cache"], None, pin=True),
+                "cl": torch.from_numpy(dec["cache_len"]).pin_memory()}
+    out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
+                (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("d_o", d_o), ("d_lse", d_lse))}
+    h2d = sum(t.numel() * t.element_size() for t in list(host.values()) + list(host_dec.values()))
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+
+    def e2e_step():
+        for n, dst in (("q", q), ("k", k), ("v", v), ("do", do)):
+            dst.copy_(host[n], non_blocking=True)
+        dq_in.copy_(host_dec["q"], non_blocking=True)
+        kc.copy_(host_dec["k"], non_blocking=True)
+        vc.copy_(host_dec["v"], non_blocking=True)
+        cl.copy_(host_dec["cl"], non_blocking=True)
+        run_step()
+        for n, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("d_o", d_o),
+                       ("d_lse", d_lse)):
+            out_host[n].copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        K = args.steps
+        value = step_flops * world * K / (ms_max * 1e-3) / 1e12
+        fwd_tf = step_fwd_flops * K / (t_fwd * 1e-3) / 1e12
+        bmain_tf = step_bwd_flops * K / (t_bmain * 1e-3) / 1e12
+        bwd_tf = step_bwd_flops * K / ((t_pre + t_bmain + t_conv) * 1e-3) / 1e12
+        dec_gbs = step_dec_bytes * K / (t_dec * 1e-3) / 1e9
+        parts = {"fwd_ms": t_fwd / K, "bwd_pre_ms": t_pre / K, "bwd_main_ms": t_bmain / K,
+                 "bwd_dq_convert_ms": t_conv / K, "decode_ms": t_dec / K}
+        dominant = max(parts, key=parts.get)
+        peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        if dominant == "fwd_ms":
+            roof = {"kernel": "swa_fwd_kernel<128>", "bound": "tensor", "achieved": fwd_tf, "peak": peak_t,
+                    "unit": "TFLOP/s"}
+        elif dominant == "decode_ms":
+            roof = {"kernel": "swa_decode_kernel<128>", "bound": "hbm", "achieved": dec_gbs, "peak": peak_h,
+                    "unit": "GB/s"}
+        else:
+            roof = {"kernel": "swa_bwd_kernel<128>", "bound": "tensor", "achieved": bmain_tf, "peak": peak_t,
+                    "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = None
+        roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['unit'] == 'TFLOP/s' else 'copy'})"
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline_sample(cfg, att)
+            cb.pop("seconds")
+            cpu = cb
+        e2e_val = step_flops * world / (float(e2e_ms.item()) * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "d24 SSSL fwd+bwd (B=32,T=2048,H=12,D=128; W=512,512,512,2048) "
+                                   "+ decode (32 seqs, cap 2048, H=12, D=128; W=2048,1024)",
+                       "global_batch": B * world, "seq_len": T, "heads": H, "head_dim": D,
+                       "windows": windows, "decode_windows": dwins,
+                       "l2": "inputs larger than L2 (q,k,v,dO 201 MB each; decode caches 403 MB each)",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "parts": {
+                **{k2: round(v2, 4) for k2, v2 in parts.items()},
+                "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "bwd_main_tflops": bmain_tf, "decode_gbs": dec_gbs,
+                "fwd_frac_spec_2250": fwd_tf / SPEC_BF16_TFLOPS, "bwd_frac_spec_2250": bwd_tf / SPEC_BF16_TFLOPS,
+                "decode_frac_spec_8000": dec_gbs / SPEC_HBM_GBS,
+                "fwd_frac_measured": fwd_tf / peak_t, "bwd_frac_measured": bwd_tf / peak_t,
+                "decode_frac_measured": dec_gbs / peak_h,
+            },
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clk,
+            "outputs_finite": finite,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,471 @@
+// bwd.cuh -- backward kernels of causal sliding-window attention.
+//
+// Gradients of sum(dO * O) for the forward in fwd.cuh (training runs through
+// flash_attn_func, apidog guide "Train your own ChatGPT", section 5).  With
+// P = softmax of the banded scores, Delta_i = sum_d dO_id O_id:
+//   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - Delta),
+//   dK = scale * dS^T Q,   dQ = scale * dS K.
+//
+// Three launches:
+//   swa_bwd_pre_kernel      Delta and lse*log2(e) as fp32 rows [B*H, Tp] padded to
+//                           Tp = 128*ceil(T/128) (padding: Delta 0, lse +inf), and a
+//                           zeroed fp32 dQ accumulator
+//   swa_bwd_kernel          one CTA per 128-row key/value tile, walking the
+//                           query tiles of its band; P^T is recomputed from lse,
+//                           dK and dV stay in TMEM, dQ partials are added to the
+//                           fp32 accumulator with vector atomics
+//   swa_bwd_dq_kernel       dQ = bf16(scale * accumulator)
+//
+// swa_bwd_kernel roles:
+//   warp 8       TMA producer: K, V once; Q_i and dO_i per query tile into a ring
+//   warp 9       MMA issuer: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO (P^T from TMEM),
+//                dK += dS^T Q, dQ_i = dS K
+//   warps 0..3   thread = key row: P^T = exp2(S^T*scale*log2e - lse*log2e) with the
+//                band mask, dS^T = P^T (dP^T - Delta) to shared memory
+//   warps 4..7   thread = query row: drain dQ_i from TMEM into the accumulator
+//   warps 0..7   epilogue: dV (warps 0..3) and scale*dK (warps 4..7) to bf16
+#pragma once
+
+#include "sm100.cuh"
+
+namespace swa {
+
+template <int D>
+struct BwdCfg {
+    static constexpr int BN = 128;                 // key rows per CTA (MMA M for S^T, dP^T, dV, dK)
+    static constexpr int BM = 128;                 // query rows per step
+    static constexpr int TILE = 128 * D * 2;
+    static constexpr int BOX = 128 * 64 * 2;
+    static constexpr int NBOX = D / 64;
+    static constexpr int NSTAGE = 2;               // Q_i / dO_i ring
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = TILE;
+    static constexpr int OFF_QD = 2 * TILE;        // stage s: Q at OFF_QD + s*2*TILE, dO after it
+    static constexpr int OFF_DS = OFF_QD + NSTAGE * 2 * TILE;   // dS^T: 128 key rows x 128 query cols bf16
+    static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;      // per stage: 128 floats lse*log2e, 128 Delta
+    static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
+    static constexpr int NUM_BAR = 1 + 2 * NSTAGE + 9;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 64;
+    // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
+    // the kernel checks at run time that the aligned layout fits what it was given.
+    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;     // S^T | dP^T (then dQ) | dV | dK
+    static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BM, 0, 0);       // K-major A, K-major B
+    static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);      // K-major A, MN-major B
+    static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 1, 1);       // MN-major A, MN-major B
+    static_assert(SMEM_USED <= 232448, "shared memory");
+};
+
+struct BwdParams {
+    const float* lse2;    // [B*H, Tp] lse * log2(e), +inf past T
+    const float* delta;   // [B*H, Tp], 0 past T
+    float* dq_acc;        // [B,T,H,D]
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    int B, T, H;
+    long long W;
+    float scale;
+    float scale_log2;
+    int n_kblk;
+    int Tp;               // T rounded up to 128
+    long long wait_limit;
+};
+
+// ---------------------------------------------------------------------------
+// Delta_i = sum_d dO_id * O_id and zeroing of the dQ accumulator.
+// One thread per 8 consecutive elements (16 bytes) of a [B,T,H,D] row.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) swa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                          const __nv_bfloat16* __restrict__ dout,
+                                                          const float* __restrict__ lse,
+                                                          float* __restrict__ lse2, float* __restrict__ delta,
+                                                          float* __restrict__ dq_acc, int B, int T, int H, int Tp) {
+    constexpr int LPR = D / 8;   // lanes per row
+    const long long nrows = (long long)B * T * H;
+    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    // lse * log2(e) into the padded rows; padding columns get +inf (and Delta 0).
+    for (long long e = tid; e < (long long)B * H * Tp; e += stride) {
+        const long long bh = e / Tp, t = e % Tp;
+        if (t < T) {
+            lse2[e] = lse[bh * T + t] * 1.4426950408889634f;
+        } else {
+            lse2[e] = INFINITY;
+            delta[e] = 0.f;
+        }
+    }
+    // Trip count is uniform across each group of LPR lanes (rows are LPR-aligned).
+    for (long long e = tid; e < ((nrows * LPR + 31) / 32) * 32; e += stride) {
+        const long long row = e / LPR;
+        const int c = int(e % LPR);
+        float acc = 0.f;
+        if (row < nrows) {
+            const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + c * 8);
+            const uint4 g = *reinterpret_cast<const uint4*>(dout + row * D + c * 8);
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 fa = __bfloat1622float2(a2[i]);
+                const float2 fg = __bfloat1622float2(g2[i]);
+                acc = fmaf(fa.x, fg.x, acc);
+                acc = fmaf(fa.y, fg.y, acc);
+            }
+            float4* z = reinterpret_cast<float4*>(dq_acc + row * D + c * 8);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (row < nrows && c == 0) {
+            const long long h = row % H;
+            const long long bt = row / H;
+            const long long t = bt % T, b = bt / T;
+            delta[(b * H + h) * Tp + t] = acc;
+        }
+    }
+}
+
+// dq = bf16(scale * dq_acc), 8 elements per thread.
+__global__ void __launch_bounds__(256) swa_bwd_dq_kernel(const float* __restrict__ dq_acc,
+                                                         __nv_bfloat16* __restrict__ dq, long long n8,
+                                                         float scale) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += stride) {
+        const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * e];
+        const float4 b = reinterpret_cast<const float4*>(dq_acc)[2 * e + 1];
+        uint4 w;
+        w.x = pack_bf16x2(a.x * scale, a.y * scale);
+        w.y = pack_bf16x2(a.z * scale, a.w * scale);
+        w.z = pack_bf16x2(b.x * scale, b.y * scale);
+        w.w = pack_bf16x2(b.z * scale, b.w * scale);
+        reinterpret_cast<uint4*>(dq)[e] = w;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const BwdParams p) {
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    if (int(base - raw) + C::SMEM_USED > C::SMEM) {   // uniform across the CTA: nothing started yet
+        if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusSmemLayout);
+        return;
+    }
+
+    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQD = base + C::OFF_QD, sDS = base + C::OFF_DS;
+    const uint32_t sLSE = base + C::OFF_LSE;   // stage s: lse2 at sLSE + s*1024, Delta 512 bytes later
+    const uint32_t bar0 = base + C::OFF_BAR;
+    const uint32_t kv_full = bar0;
+    auto qd_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto qd_empty = [&](int s) { return bar0 + 8u * (1 + C::NSTAGE + s); };
+    const uint32_t b9 = bar0 + 8u * (1 + 2 * C::NSTAGE);
+    const uint32_t s_full = b9, dp_full = b9 + 8, p_full = b9 + 16, ds_full = b9 + 24, dv_done = b9 + 32,
+                   dq_full = b9 + 40, dq_free = b9 + 48, ds_free = b9 + 56, mma_done = b9 + 64;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
+
+    const int BH = p.B * p.H;
+    const int kblk = int(blockIdx.x / BH);          // low key blocks have the most query tiles: first
+    const int bh = int(blockIdx.x % BH);
+    const int b = bh / p.H, h = bh % p.H;
+    const int T = p.T;
+    const long long W = p.W;
+    const long long k0 = (long long)kblk * C::BN;
+    const int ilo = int(k0 / C::BM);
+    const int ihi = int(imin_ll(T - 1, k0 + C::BN - 1 + W - 1) / C::BM);
+    const int nsteps = ihi - ilo + 1;
+
+    const int warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(qd_full(s), 1);
+            mbar_init(qd_empty(s), 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(ds_full, 128);
+        mbar_init(dv_done, 1);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_free, 128);
+        mbar_init(ds_free, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tDP = tmem + 128u, tDV = tmem + 256u, tDK = tmem + 256u + uint32_t(D);
+
+    if (warp == 8) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+            for (int x = 0; x < C::NBOX; ++x) {
+                tma_load_4d(sK + x * C::BOX, &tm_k, kv_full, x * 64, h, int(k0), b);
+                tma_load_4d(sV + x * C::BOX, &tm_v, kv_full, x * 64, h, int(k0), b);
+            }
+            int n = 0;
+            for (; n < nsteps; ++n) {
+                const int s = n % C::NSTAGE;
+                if (!mbar_wait(qd_empty(s), ((n / C::NSTAGE) & 1) ^ 1u, abort_flag, p.wait_limit,
+                               kStatusTimeoutProducer))
+                    break;
+                const int qrow = (ilo + n) * C::BM;
+                mbar_arrive_expect_tx(qd_full(s), 2 * C::TILE + 1024);
+                const uint32_t dst = sQD + s * 2 * C::TILE;
+                for (int x = 0; x < C::NBOX; ++x) {
+                    tma_load_4d(dst + x * C::BOX, &tm_q, qd_full(s), x * 64, h, qrow, b);
+                    tma_load_4d(dst + C::TILE + x * C::BOX, &tm_do, qd_full(s), x * 64, h, qrow, b);
+                }
+                const size_t row = size_t(bh) * p.Tp + size_t(qrow);
+                bulk_load(sLSE + s * 1024, p.lse2 + row, 512, qd_full(s));
+                bulk_load(sLSE + s * 1024 + 512, p.delta + row, 512, qd_full(s));
+            }
+            for (int s = 0; s < C::NSTAGE && s < n; ++s) {
+                const int fills = (n - s + C::NSTAGE - 1) / C::NSTAGE;
+                mbar_wait(qd_full(s), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            }
+            mbar_wait(kv_full, 0, abort_flag, p.wait_limit, kStatusTimeoutProducer);
+        }
+    } else if (warp == 9) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            bool ok = mbar_wait(kv_full, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
+            for (int n = 0; n < nsteps && ok; ++n) {
+                const int s = n % C::NSTAGE;
+                const uint32_t par = uint32_t(n & 1);
+                ok = mbar_wait(qd_full(s), (n / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                if (!ok) break;
+                const uint32_t sQ = sQD + s * 2 * C::TILE, sDO = sQ + C::TILE;
+                // S^T overwrites the P^T columns read by dV of the previous step.
+                if (n > 0) {
+                    ok = mbar_wait(dv_done, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    if (!ok) break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), C::IDESC_S, kk > 0);
+                }
+                tc_commit(s_full);
+                // dP^T reuses the columns the dQ drain of the previous step reads.
+                if (n > 0) {
+                    ok = mbar_wait(dq_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), C::IDESC_S,
+                           kk > 0);
+                }
+                tc_commit(dp_full);
+                // dV += P^T dO
+                ok = mbar_wait(p_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C::BM / 16; ++kk)
+                    mma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(dv_done);
+                // dK += dS^T Q ; dQ_i = dS K
+                ok = mbar_wait(ds_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < C::BM / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tDK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, C::BOX, 1024),
+                           C::IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    mma_ss(tDP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024), sdesc_sw128(sK + kk * 2048, C::BOX, 1024),
+                           C::IDESC_DQ, kk > 0);
+                tc_commit(dq_full);
+                tc_commit(ds_free);
+                tc_commit(qd_empty(s));
+            }
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
+        }
+    } else if (warp < 4) {
+        // ------------------------------ key-row warps: P^T and dS^T ------------------------------
+        const int row = warp * 32 + lane;
+        const long long kv = k0 + row;
+        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int n = 0; n < nsteps && ok; ++n) {
+            const uint32_t par = uint32_t(n & 1);
+            const long long q0 = (long long)(ilo + n) * C::BM;
+            // S^T is committed after the MMA warp saw this stage's loads (Q, dO, lse, Delta) land.
+            const float* lse2_s = reinterpret_cast<const float*>(gbase + C::OFF_LSE + (n % C::NSTAGE) * 1024);
+            const float* delta_s = lse2_s + 128;
+            ok = __all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+            if (!ok) break;
+            tc_fence_after();
+            // Band of this key row: queries kv .. kv+W-1 (and < T).
+            const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
+            float pr[C::BM];
+#pragma unroll
+            for (int c = 0; c < C::BM / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tS + lane_off + c * 32, r);
+                tmem_ld_wait(r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int col = c * 32 + i;
+                    float v = ex2_approx(fmaf(__uint_as_float(r[i]), sl2, -lse2_s[col]));
+                    if (!full) {
+                        const long long qq = q0 + col;
+                        if (!(qq >= kv && qq - kv < W && qq < T && kv < T)) v = 0.f;
+                    }
+                    pr[col] = v;
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < C::BM / 64; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[c * 64 + 2 * i], pr[c * 64 + 2 * i + 1]);
+                tmem_st32(tS + lane_off + c * 32, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(p_full);
+            // dS^T = P^T (dP^T - Delta)
+            ok = __all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+            if (!ok) break;
+            tc_fence_after();
+            if (n > 0) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(ds_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                if (!ok) break;
+            }
+#pragma unroll
+            for (int c = 0; c < C::BM / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tDP + lane_off + c * 32, r);
+                tmem_ld_wait(r);
+                // 32 query columns = four 16-byte chunks of this key row in the 128B-swizzled tile.
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = c * 32 + g * 8 + 2 * e;
+                        const float d0 = pr[col] * (__uint_as_float(r[g * 8 + 2 * e]) - delta_s[col]);
+                        const float d1 = pr[col + 1] * (__uint_as_float(r[g * 8 + 2 * e + 1]) - delta_s[col + 1]);
+                        w[e] = pack_bf16x2(d0, d1);
+                    }
+                    const int chunk = (c * 32 + g * 8) >> 3;            // 0..15 across the 128 columns
+                    const int box = chunk >> 3, cib = chunk & 7;
+                    const uint32_t addr = sDS + box * C::BOX + row * 128 + ((cib ^ (row & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
+                                 "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+    } else {
+        // ------------------------------ query-row warps: dQ drain ------------------------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+        bool ok = true;
+        for (int n = 0; n < nsteps && ok; ++n) {
+            const long long qr = (long long)(ilo + n) * C::BM + row;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(dq_full, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
+            if (!ok) break;
+            tc_fence_after();
+            float acc[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tDP + lane_off + c * 32, r);
+                tmem_ld_wait(r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[c * 32 + i] = __uint_as_float(r[i]);
+            }
+            tc_fence_before();
+            mbar_arrive(dq_free);
+            if (qr < T) {
+                float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t(b) * T + size_t(qr)) * p.H + h) * D);
+#pragma unroll
+                for (int v4 = 0; v4 < D / 4; ++v4)
+                    atomicAdd(dst + v4, make_float4(acc[4 * v4], acc[4 * v4 + 1], acc[4 * v4 + 2], acc[4 * v4 + 3]));
+            }
+        }
+    }
+
+    // ------------------------------ epilogue: dV, dK ------------------------------
+    if (warp < 8) {
+        const bool ok = __all_sync(0xffffffffu,
+                                   mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
+        if (ok) {
+            tc_fence_after();
+            const int quarter = warp & 3;
+            const int row = quarter * 32 + lane;
+            const long long kv = k0 + row;
+            const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+            const bool is_dv = warp < 4;
+            const uint32_t src = (is_dv ? tDV : tDK) + lane_off;
+            const float mul = is_dv ? 1.f : p.scale;
+            __nv_bfloat16* dst = (is_dv ? p.dv : p.dk) + ((size_t(b) * T + size_t(kv < T ? kv : 0)) * p.H + h) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(src + c * 32, r);
+                tmem_ld_wait(r);
+                if (kv < T) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * mul, __uint_as_float(r[v4 * 8 + 1]) * mul);
+                        w.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * mul, __uint_as_float(r[v4 * 8 + 3]) * mul);
+                        w.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * mul, __uint_as_float(r[v4 * 8 + 5]) * mul);
+                        w.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * mul, __uint_as_float(r[v4 * 8 + 7]) * mul);
+                        *reinterpret_cast<uint4*>(dst + c * 32 + v4 * 8) = w;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace swa

@@ -1,0 +1,306 @@
+// swa_attn.cu -- C-ABI entry points of libswa_b200.so (declared in include/swa_attn.h).
+//
+// Host side only: argument validation, TMA tensor maps, workspace carving and
+// kernel launches on the caller's stream.  No allocation, no synchronisation
+// (except attn_device_status, which is documented to synchronise).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/swa_attn.h"
+#include "bwd.cuh"
+#include "decode.cuh"
+#include "fwd.cuh"
+
+namespace {
+
+using namespace swa;
+
+constexpr long long kDefaultWaitLimit = 1LL << 33;   // ~4 s of SM clocks
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [B, T, H, D] bf16 viewed as a 4-D tensor (D, H, T, B), boxes of 64 x 1 x 128 x 1
+// with 128-byte swizzle (one box = 128 rows of one head, 64 columns).
+bool make_bthd_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+    cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2, cuuint64_t(T) * H * D * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// cudaFuncSetAttribute for the large-shared-memory kernels, once per (device, kernel).
+bool ensure_smem(const void* func, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (done.count({dev, func})) return true;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done.insert({dev, func});
+    return true;
+}
+
+bool valid_common(int B, int T, int H, int D, int W, float scale) {
+    if (B < 1 || T < 1 || H < 1 || W < 1) return false;
+    if (!(scale > 0.f) || scale != scale || scale > 3.4e38f) return false;
+    (void)D;
+    return true;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Optional events recorded between the three launches of attn_bwd (see
+// attn_bwd_set_profile_events); per calling thread.
+thread_local cudaEvent_t g_ev_after_pre = nullptr;
+thread_local cudaEvent_t g_ev_after_main = nullptr;
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
+
+int grid_for(long long work_items, int threads) {
+    long long blocks = (work_items + threads - 1) / threads;
+    const long long cap = 148LL * 32;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return int(blocks);
+}
+
+__global__ void swa_selftest_wait_kernel(long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t a = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(a, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // Nobody arrives on this barrier: the wait must give up after limit_cycles.
+    if (threadIdx.x == 0) mbar_wait(a, 0, &abort_flag, limit_cycles, kStatusTimeoutSelftest);
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B, int T,
+             int H, int D, int W, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    const int n_qblk = (T + 255) / 256;
+    const long long grid = (long long)n_qblk * B * H;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv;
+    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, H, D) || !make_bthd_map(&mv, v, B, T, H, D))
+        return ATTN_ERR_LAUNCH;
+    FwdParams p;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.W = W;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.n_qblk = n_qblk;
+    p.wait_limit = kDefaultWaitLimit;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (D == 128) {
+        if (!ensure_smem((const void*)swa_fwd_kernel<128>, FwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_fwd_kernel<128><<<unsigned(grid), FwdCfg<128>::THREADS, FwdCfg<128>::SMEM, s>>>(mq, mk, mv, p);
+    } else {
+        if (!ensure_smem((const void*)swa_fwd_kernel<64>, FwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_fwd_kernel<64><<<unsigned(grid), FwdCfg<64>::THREADS, FwdCfg<64>::SMEM, s>>>(mq, mk, mv, p);
+    }
+    return launch_status();
+}
+
+// Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128),
+// then the fp32 dQ accumulator [B, T, H, D].
+size_t attn_bwd_workspace_bytes(int B, int T, int H, int D) {
+    if (B < 1 || T < 1 || H < 1 || D < 1) return 0;
+    const size_t Tp = (size_t(T) + 127) / 128 * 128;
+    return 2 * align256(size_t(B) * H * Tp * 4) + align256(size_t(B) * T * H * D * 4);
+}
+
+int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
+             const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace, size_t ws_bytes,
+             int B, int T, int H, int D, int W, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (ws_bytes < attn_bwd_workspace_bytes(B, T, H, D)) return ATTN_ERR_WORKSPACE;
+    const int n_kblk = (T + 127) / 128;
+    const long long grid = (long long)n_kblk * B * H;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, H, D) ||
+        !make_bthd_map(&mv, v, B, T, H, D) || !make_bthd_map(&mdo, dout, B, T, H, D))
+        return ATTN_ERR_LAUNCH;
+    const int Tp = (T + 127) / 128 * 128;
+    const size_t row_bytes = align256(size_t(B) * H * Tp * 4);
+    float* lse2 = reinterpret_cast<float*>(workspace);
+    float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + row_bytes);
+    float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * row_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long rows = (long long)B * T * H;
+    const auto* o_b = reinterpret_cast<const __nv_bfloat16*>(o);
+    const auto* do_b = reinterpret_cast<const __nv_bfloat16*>(dout);
+    if (D == 128)
+        swa_bwd_pre_kernel<128><<<grid_for(rows * 16, 256), 256, 0, s>>>(o_b, do_b, lse, lse2, delta, dq_acc, B,
+                                                                         T, H, Tp);
+    else
+        swa_bwd_pre_kernel<64><<<grid_for(rows * 8, 256), 256, 0, s>>>(o_b, do_b, lse, lse2, delta, dq_acc, B, T,
+                                                                       H, Tp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
+    if (g_ev_after_pre) cudaEventRecord(g_ev_after_pre, s);
+
+    BwdParams p;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.dq_acc = dq_acc;
+    p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+    p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.W = W;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.n_kblk = n_kblk;
+    p.Tp = Tp;
+    p.wait_limit = kDefaultWaitLimit;
+    if (D == 128) {
+        if (!ensure_smem((const void*)swa_bwd_kernel<128>, BwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_bwd_kernel<128><<<unsigned(grid), BwdCfg<128>::THREADS, BwdCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
+    } else {
+        if (!ensure_smem((const void*)swa_bwd_kernel<64>, BwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_bwd_kernel<64><<<unsigned(grid), BwdCfg<64>::THREADS, BwdCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
+    }
+    if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
+    if (g_ev_after_main) cudaEventRecord(g_ev_after_main, s);
+    const long long n8 = rows * D / 8;
+    swa_bwd_dq_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, reinterpret_cast<__nv_bfloat16*>(dq), n8, scale);
+    return launch_status();
+}
+
+size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
+    if (B < 1 || cap < 1 || H < 1 || D < 1) return 0;
+    const size_t nsm = size_t((cap + kDecodeChunk - 1) / kDecodeChunk);
+    const size_t nhg = size_t((H + kDecodeThreads / (D / 8) - 1) / (kDecodeThreads / (D / 8)));
+    return align256(size_t(B) * nhg * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
+           align256(size_t(B) * nsm * H * D * 4);
+}
+
+int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache, const int32_t* cache_len,
+                attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B, int cap, int H, int D, int W,
+                float scale, void* stream) {
+    if (!q || !k_cache || !v_cache || !cache_len || !o || !workspace) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, cap, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (ws_bytes < attn_decode_workspace_bytes(B, cap, H, D)) return ATTN_ERR_WORKSPACE;
+    const int nsm = (cap + kDecodeChunk - 1) / kDecodeChunk;
+    const int span = W < cap ? W : cap;
+    DecParams p;
+    p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    p.kc = reinterpret_cast<const __nv_bfloat16*>(k_cache);
+    p.vc = reinterpret_cast<const __nv_bfloat16*>(v_cache);
+    p.cache_len = cache_len;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    const int heads_per_cta = kDecodeThreads / (D / 8);
+    const int nhg = (H + heads_per_cta - 1) / heads_per_cta;
+    if (nhg > 65535) return ATTN_ERR_UNSUPPORTED;
+    char* ws = static_cast<char*>(workspace);
+    const size_t cnt_bytes = align256(size_t(B) * nhg * 4);
+    p.counters = reinterpret_cast<int*>(ws);
+    p.part_ml = reinterpret_cast<float*>(ws + cnt_bytes);
+    p.part_o = reinterpret_cast<float*>(ws + cnt_bytes + align256(size_t(B) * nsm * H * 2 * 4));
+    p.B = B;
+    p.cap = cap;
+    p.H = H;
+    p.W = W;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.nsplit = (span + kDecodeChunk - 1) / kDecodeChunk;
+    p.nsplit_max = nsm;
+    const int threads = ((std::min(H, heads_per_cta) * (D / 8)) + 31) / 32 * 32;
+    dim3 grid(p.nsplit, B, nhg);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (D == 128)
+        swa_decode_kernel<128><<<grid, threads, 0, s>>>(p);
+    else
+        swa_decode_kernel<64><<<grid, threads, 0, s>>>(p);
+    return launch_status();
+}
+
+int attn_bwd_set_profile_events(void* after_pre, void* after_main) {
+    g_ev_after_pre = reinterpret_cast<cudaEvent_t>(after_pre);
+    g_ev_after_main = reinterpret_cast<cudaEvent_t>(after_main);
+    return ATTN_OK;
+}
+
+int attn_device_status(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, swa::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(swa::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+    }
+    return v ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+}
+
+int attn_selftest_wait_timeout(long long limit_cycles, void* stream) {
+    if (limit_cycles < 1 || limit_cycles > (1LL << 34)) return ATTN_ERR_INVALID_ARG;
+    swa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    return launch_status();
+}
+
+const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ATTN_ERR_LAUNCH: return "kernel launch failed";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case ATTN_ERR_WORKSPACE: return "workspace too small";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -17,6 +17,8 @@ depth 24 -> 12 heads, depth 26 -> 13 heads.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -47,16 +49,31 @@ def _u64_stream(seed: int, tag: int, start: int, count: int) -> np.ndarray:
         return _mix(key + ctr * _GOLDEN)
 
 
-def normal_f64(seed: int, tag: int, n: int, chunk: int = 1 << 24) -> np.ndarray:
-    """n standard normals (float64) from the counter-based stream (seed, tag)."""
+def normal_f64(seed: int, tag: int, n: int, chunk: int = 1 << 22) -> np.ndarray:
+    """n standard normals (float64) from the counter-based stream (seed, tag).
+
+    Chunks are independent (the stream is counter-based), so they are filled
+    by a thread pool; the result does not depend on the chunking.
+    """
     out = np.empty(n, dtype=np.float64)
     inv = 1.0 / 9007199254740992.0  # 2**-53
-    for s in range(0, n, chunk):
+
+    def fill(s: int):
         c = min(chunk, n - s)
         u = _u64_stream(seed, tag, 2 * s, 2 * c)
         u1 = ((u[0::2] >> np.uint64(11)).astype(np.float64) + 0.5) * inv
         u2 = ((u[1::2] >> np.uint64(11)).astype(np.float64) + 0.5) * inv
         out[s:s + c] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+
+    starts = range(0, n, chunk)
+    if n <= chunk:
+        for s in starts:
+            fill(s)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
     return out
 
 

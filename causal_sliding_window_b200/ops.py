@@ -1,0 +1,182 @@
+"""ctypes binding of libswa_b200.so, with the C entry points' names.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI (include/swa_attn.h). PyTorch supplies device
+memory and the stream. Importing this module loads the library and raises
+if it is missing; there is no fallback path.
+
+Low-level calls (caller provides every buffer, torch tensors on one CUDA device):
+  attn_fwd(q, k, v, o, lse, W, scale=None, stream=None)
+  attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, W, scale=None, stream=None)
+  attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W, scale=None, stream=None)
+Convenience wrappers that allocate outputs: forward, backward, decode.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libswa_b200.so")
+
+ATTN_OK = 0
+STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported configuration", -3: "kernel launch failed",
+          -4: "device wait timed out", -5: "workspace too small"}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m causal_sliding_window_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_p, _i, _f, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
+_lib.attn_fwd.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_fwd.restype = _i
+_lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.attn_bwd_workspace_bytes.restype = _sz
+_lib.attn_bwd.argtypes = [_p] * 10 + [_sz, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_bwd.restype = _i
+_lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.attn_decode_workspace_bytes.restype = _sz
+_lib.attn_decode.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_decode.restype = _i
+_lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
+_lib.attn_bwd_set_profile_events.restype = _i
+_lib.attn_device_status.argtypes = [_i]
+_lib.attn_device_status.restype = _i
+_lib.attn_selftest_wait_timeout.argtypes = [_ll, _p]
+_lib.attn_selftest_wait_timeout.restype = _i
+_lib.attn_status_string.argtypes = [_i]
+_lib.attn_status_string.restype = ctypes.c_char_p
+
+EXPORTED = ["attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_decode_workspace_bytes", "attn_decode",
+            "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
+            "attn_status_string"]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bthd(*ts):
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("expected contiguous bf16 CUDA tensors of shape [B, T, H, D]")
+    shape = ts[0].shape
+    if any(t.shape != shape for t in ts):
+        raise ValueError("shape mismatch")
+    return shape
+
+
+def _scale(scale, D):
+    return 1.0 / math.sqrt(D) if scale is None else float(scale)
+
+
+def attn_fwd(q, k, v, o, lse, W: int, scale=None, stream=None):
+    B, T, H, D = _bthd(q, k, v, o)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, T] tensor")
+    _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, H, D, int(W), _scale(scale, D),
+                         _stream(stream)), "attn_fwd")
+
+
+def attn_bwd_workspace_bytes(B: int, T: int, H: int, D: int) -> int:
+    return int(_lib.attn_bwd_workspace_bytes(B, T, H, D))
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, W: int, scale=None, stream=None):
+    B, T, H, D = _bthd(q, k, v, o, dout, dq, dk, dv)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T):
+        raise ValueError("lse must be float32 [B, H, T]")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                         _ptr(workspace), ws_bytes, B, T, H, D, int(W), _scale(scale, D), _stream(stream)),
+           "attn_bwd")
+
+
+def attn_decode_workspace_bytes(B: int, cap: int, H: int, D: int) -> int:
+    return int(_lib.attn_decode_workspace_bytes(B, cap, H, D))
+
+
+def attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W: int, scale=None, stream=None):
+    B, cap, H, D = _bthd(k_cache, v_cache)
+    if tuple(q.shape) != (B, H, D) or tuple(o.shape) != (B, H, D) or q.dtype != torch.bfloat16:
+        raise ValueError("q and o must be bf16 [B, H, D]")
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or not cache_len.is_cuda:
+        raise ValueError("cache_len must be an int32 CUDA tensor of shape [B]")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), _ptr(o), _ptr(lse),
+                            _ptr(workspace), ws_bytes, B, cap, H, D, int(W), _scale(scale, D), _stream(stream)),
+           "attn_decode")
+
+
+def attn_bwd_set_profile_events(after_pre=None, after_main=None):
+    """Record torch.cuda.Event objects between attn_bwd's launches (None disables)."""
+    h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event)  # noqa: E731
+    _check(_lib.attn_bwd_set_profile_events(h(after_pre), h(after_main)), "attn_bwd_set_profile_events")
+
+
+def attn_device_status(clear: bool = True) -> int:
+    return int(_lib.attn_device_status(1 if clear else 0))
+
+
+def attn_selftest_wait_timeout(limit_cycles: int, stream=None) -> int:
+    return int(_lib.attn_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
+
+
+def attn_status_string(status: int) -> str:
+    return _lib.attn_status_string(int(status)).decode()
+
+
+# ---------------------------------------------------------------------------
+# Convenience wrappers (allocate outputs with torch; compute still in the kernels)
+# ---------------------------------------------------------------------------
+
+def forward(q, k, v, W: int, scale=None, stream=None):
+    B, T, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    attn_fwd(q, k, v, o, lse, W, scale, stream)
+    return o, lse
+
+
+def backward(q, k, v, o, lse, dout, W: int, scale=None, stream=None, workspace=None):
+    B, T, H, D = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=q.device)
+    attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, W, scale, stream)
+    return dq, dk, dv
+
+
+def decode_workspace(B: int, cap: int, H: int, D: int, device) -> torch.Tensor:
+    """Zero-filled decode workspace (the decode call keeps it zeroed between calls)."""
+    return torch.zeros(attn_decode_workspace_bytes(B, cap, H, D), dtype=torch.uint8, device=device)
+
+
+def decode(q, k_cache, v_cache, cache_len, W: int, scale=None, stream=None, workspace=None):
+    B, cap, H, D = k_cache.shape
+    o = torch.empty((B, H, D), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(B, cap, H, D, q.device)
+    attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W, scale, stream)
+    return o, lse

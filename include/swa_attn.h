@@ -1,0 +1,146 @@
+/*
+ * swa_attn.h -- C ABI of the B200 (sm_100a) causal sliding-window attention library.
+ *
+ * The operation.  nanochat's GPT computes attention once per layer through
+ * flash_attn_func(q, k, v, causal=True, window_size=window_size) (apidog guide
+ * "Train your own ChatGPT", section 5 "Flash Attention unification"), with a
+ * per-layer window that alternates short and long contexts in the "SSSL"
+ * pattern (same guide, section 1 "GPT model", architecture features), and it
+ * decodes tokens against a KV cache prefilled through flash_attn_with_kvcache
+ * (same guide, section 6 "Inference engine", KV cache).  Karpathy's nanochat
+ * GPT-2-speedrun post (first page) ranks the Flash Attention 3 kernels, whose
+ * window_size keyword makes the alternating patterns possible, among the
+ * changes that helped most.
+ *
+ * Window convention used throughout: query i attends to key j iff
+ * i - W < j <= i, so row i has min(i + 1, W) keys; W >= T is full causal.
+ * The softmax is exp(scale * <q_i, k_j>) normalised over the band; lse is its
+ * natural-log normaliser.
+ *
+ * Common rules for every entry point:
+ *  - Tensors are dense, row-major, and live in device memory (the decode
+ *    cache_len array too).  The caller owns every buffer, including
+ *    workspaces; the library never allocates device memory and never
+ *    synchronises in attn_fwd / attn_bwd / attn_decode.  Work is enqueued on
+ *    `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *  - bf16 tensors are passed as attn_bf16 (the raw 16-bit pattern).
+ *    [B, T, H, D] means element (b, t, h, d) at ((b*T + t)*H + h)*D + d.
+ *  - Every pointer must be 16-byte aligned; D must be 64 or 128; B, T, H >= 1;
+ *    W >= 1; scale > 0 and finite.  A violation returns ATTN_ERR_INVALID_ARG
+ *    (or ATTN_ERR_UNSUPPORTED for an unsupported D) before anything is
+ *    launched.  A failed launch returns ATTN_ERR_LAUNCH.
+ *  - Outputs are written with round-to-nearest-even to bf16; lse is fp32.
+ *  - Device-side waits are bounded.  If one gives up (a condition that
+ *    correct use never produces), the kernel stops early and records a flag
+ *    that attn_device_status() reports as ATTN_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef SWA_ATTN_H
+#define SWA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t attn_bf16;
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = -1,
+    ATTN_ERR_UNSUPPORTED = -2,
+    ATTN_ERR_LAUNCH = -3,
+    ATTN_ERR_DEVICE_TIMEOUT = -4,
+    ATTN_ERR_WORKSPACE = -5
+} attn_status;
+
+/*
+ * Forward (training / prefill): O and logsumexp.
+ *   q, k, v  [B, T, H, D] bf16, read only.
+ *   o        [B, T, H, D] bf16, written.
+ *   lse      [B, H, T] fp32, written; lse[b,h,i] = ln sum_{j in band(i)} exp(scale <q_i, k_j>).
+ *   W        window (>= 1; values >= T mean full causal).
+ * Defined by: flash_attn_func(q, k, v, causal=True, window_size=...) in the
+ * apidog guide, section 5; the window per layer from section 1 ("SSSL").
+ */
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
+             int B, int T, int H, int D, int W, float scale, void* stream);
+
+/* Bytes of workspace attn_bwd needs: fp32 rows of lse*log2(e) and Delta, [B*H, T rounded up
+ * to 128] each, and the fp32 dQ accumulator [B,T,H,D]. */
+size_t attn_bwd_workspace_bytes(int B, int T, int H, int D);
+
+/*
+ * Backward: gradients of sum(dO * O) with respect to q, k, v.
+ *   q, k, v, o, dout  [B, T, H, D] bf16 (o and lse are the forward's outputs).
+ *   lse               [B, H, T] fp32.
+ *   dq, dk, dv        [B, T, H, D] bf16, written.
+ *   workspace         device buffer of at least attn_bwd_workspace_bytes(B,T,H,D)
+ *                     bytes, 256-byte aligned, contents need not be initialised;
+ *                     ws_bytes smaller than required returns ATTN_ERR_WORKSPACE.
+ * Probabilities are recomputed from lse; dQ is accumulated in fp32.
+ * Defined by: training through flash_attn_func (apidog guide, section 5; the
+ * training runs of its "scripts.base_train" walkthrough).
+ */
+int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o,
+             const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+             void* workspace, size_t ws_bytes, int B, int T, int H, int D, int W, float scale,
+             void* stream);
+
+/* Bytes of workspace attn_decode needs for B sequences of capacity cap (any W). */
+size_t attn_decode_workspace_bytes(int B, int cap, int H, int D);
+
+/*
+ * Single-token decode over a KV cache (split over the cache, then combined).
+ *   q          [B, H, D] bf16: the new token's query, which sits at position cache_len[b]-1.
+ *   k_cache    [B, cap, H, D] bf16; v_cache likewise.  Slot cache_len[b]-1 already
+ *              holds the new token's key and value.  Only slots
+ *              max(0, L-W) .. L-1 (L = cache_len[b]) are read.
+ *   cache_len  [B] int32 in device memory, each in [1, cap].
+ *   o          [B, H, D] bf16, written.   lse  [B, H] fp32, written (may be NULL).
+ *   workspace  at least attn_decode_workspace_bytes(B, cap, H, D) bytes, 256-byte
+ *              aligned.  It must be zero-filled before its first use; every
+ *              call leaves it in that state again.  Concurrent calls must not
+ *              share a workspace.
+ * Defined by: the engine's KV cache and flash_attn_with_kvcache (apidog guide,
+ * section 6 "Inference engine").
+ */
+int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes,
+                int B, int cap, int H, int D, int W, float scale, void* stream);
+
+/*
+ * Profiling aid: when set (non-NULL cudaEvent_t handles), every later
+ * attn_bwd call made from this host thread records `after_pre` on its stream
+ * right after the Delta / accumulator-zeroing launch and `after_main` right
+ * after the main backward launch, so a caller that brackets attn_bwd with its
+ * own events can time the three launches separately.  Pass NULLs to stop.
+ * Nothing else changes; no work is skipped.
+ */
+int attn_bwd_set_profile_events(void* after_pre, void* after_main);
+
+/*
+ * Device status word: returns ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if any
+ * kernel of this library gave up a bounded wait (or found its shared-memory
+ * window unusable and did no work) since the last clear.
+ * Synchronises the current device.  `clear` != 0 resets the word.
+ */
+int attn_device_status(int clear);
+
+/*
+ * Diagnostic: launches one tiny kernel whose mbarrier wait can never complete,
+ * bounded by `limit_cycles` SM clocks, so that the bounded-wait path can be
+ * exercised without faulting or hanging the GPU.  Returns the launch status;
+ * attn_device_status() then reports ATTN_ERR_DEVICE_TIMEOUT.
+ */
+int attn_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/* Human-readable name of a status code. */
+const char* attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_ATTN_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments with the documented status before launching anything
+(these calls never reach the GPU, so they run on a CPU-only machine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from causal_sliding_window_b200.build import HEADER, build_library
+
+build_library()
+from causal_sliding_window_b200 import ops  # noqa: E402
+
+ERR_INVALID, ERR_UNSUPPORTED, ERR_WORKSPACE = -1, -2, -5
+A = 1 << 20          # a fake, 256-byte-aligned device address; never dereferenced on these paths
+MIS = A + 8          # misaligned
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(attn_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_entry_points_are_exported():
+    names = declared_functions()
+    assert {"attn_fwd", "attn_bwd", "attn_decode", "attn_bwd_workspace_bytes",
+            "attn_decode_workspace_bytes", "attn_device_status", "attn_status_string",
+            "attn_selftest_wait_timeout"} <= set(names)
+    lib = ctypes.CDLL(ops.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(ops.EXPORTED) | {n for n in names if hasattr(ops, n)}
+
+
+def test_library_is_sm100a_only_build():
+    from causal_sliding_window_b200 import build
+
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+
+
+def fwd(q=A, k=A, v=A, o=A, lse=A, B=1, T=16, H=1, D=128, W=4, scale=0.1):
+    return ops._lib.attn_fwd(q, k, v, o, lse, B, T, H, D, W, scale, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), ERR_INVALID), (dict(lse=None), ERR_INVALID), (dict(o=MIS), ERR_INVALID),
+    (dict(B=0), ERR_INVALID), (dict(T=0), ERR_INVALID), (dict(H=-1), ERR_INVALID), (dict(W=0), ERR_INVALID),
+    (dict(scale=0.0), ERR_INVALID), (dict(scale=float("nan")), ERR_INVALID), (dict(scale=-1.0), ERR_INVALID),
+    (dict(D=96), ERR_UNSUPPORTED), (dict(D=256), ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_bad_arguments(kw, expect):
+    assert fwd(**kw) == expect
+
+
+def bwd(ws_bytes=None, ws=A, B=1, T=16, H=1, D=128, W=4, scale=0.1, dq=A):
+    if ws_bytes is None:
+        ws_bytes = ops.attn_bwd_workspace_bytes(B, T, H, D) if B > 0 and T > 0 and H > 0 else 0
+    return ops._lib.attn_bwd(A, A, A, A, A, A, dq, A, A, ws, ws_bytes, B, T, H, D, W, scale, None)
+
+
+def test_bwd_rejects_bad_arguments():
+    assert bwd(ws=None) == ERR_INVALID
+    assert bwd(ws=A + 16) == ERR_INVALID               # workspace must be 256-byte aligned
+    assert bwd(dq=MIS) == ERR_INVALID
+    assert bwd(W=0) == ERR_INVALID
+    assert bwd(D=80) == ERR_UNSUPPORTED
+    assert bwd(ws_bytes=ops.attn_bwd_workspace_bytes(1, 16, 1, 128) - 1) == ERR_WORKSPACE
+
+
+def test_workspace_sizes():
+    # lse*log2e and Delta [B*H, Tp] fp32 + dQ accumulator [B,T,H,D] fp32, each 256-byte padded.
+    assert ops.attn_bwd_workspace_bytes(32, 2048, 12, 128) == 2 * 32 * 12 * 2048 * 4 + 32 * 2048 * 12 * 128 * 4
+    assert ops.attn_bwd_workspace_bytes(1, 130, 1, 64) == 2 * 256 * 4 + 130 * 64 * 4   # Tp = 256
+    assert ops.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
+    assert ops.attn_decode_workspace_bytes(32, 2048, 12, 128) > 32 * 32 * 12 * 128 * 4
+    assert ops.attn_decode_workspace_bytes(1, 0, 1, 64) == 0
+
+
+def dec(q=A, cl=A, ws=A, ws_bytes=None, B=2, cap=64, H=2, D=128, W=8, scale=0.1, lse=A):
+    if ws_bytes is None:
+        ws_bytes = ops.attn_decode_workspace_bytes(B, cap, H, D) if B > 0 and cap > 0 and H > 0 else 0
+    return ops._lib.attn_decode(q, A, A, cl, A, lse, ws, ws_bytes, B, cap, H, D, W, scale, None)
+
+
+def test_decode_rejects_bad_arguments():
+    assert dec(q=None) == ERR_INVALID
+    assert dec(cl=None) == ERR_INVALID
+    assert dec(cl=A + 2) == ERR_INVALID
+    assert dec(ws=A + 64) == ERR_INVALID
+    assert dec(cap=0) == ERR_INVALID
+    assert dec(W=0) == ERR_INVALID
+    assert dec(D=32) == ERR_UNSUPPORTED
+    assert dec(ws_bytes=16) == ERR_WORKSPACE
+
+
+def test_status_strings_and_selftest_argument_check():
+    assert ops.attn_status_string(0) == "ok"
+    assert ops.attn_status_string(-4) == "device wait timed out"
+    assert ops.attn_status_string(7) == "unknown status"
+    assert ops._lib.attn_selftest_wait_timeout(0, None) == ERR_INVALID
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The package never imports the oracle, and ops raises if the library is absent."""
+    pkg = os.path.dirname(ops.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(root, f)).read()
+                assert "oracle" not in src.replace("oracle_", "").lower() or f == "inputs.py", f
+    src = open(ops.__file__).read()
+    assert "raise ImportError" in src

@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+Tolerances (fixed by the target, written here):
+  O      relative L2 <= 5e-3 and max-abs <= 2e-2
+  lse    max-abs <= 1e-3
+  dQ/dK/dV relative L2 <= 1e-2
+Small shapes are compared element by element over the whole output; the
+full-size workloads (depth 12 / 24 / 26 shapes, decode batch) are compared on
+sampled rows the oracle computes one by one, plus whole-tensor properties.
+"""
+import numpy as np
+import pytest
+import torch
+
+from causal_sliding_window_b200 import inputs
+from oracle import (oracle_bwd, oracle_decode, oracle_dkv_rows, oracle_dq_rows, oracle_fwd,
+                    oracle_fwd_rows)
+
+pytestmark = pytest.mark.gpu
+
+O_REL, O_ABS, LSE_ABS, G_REL = 5e-3, 2e-2, 1e-3, 1e-2
+GUARD = 64                      # guard elements on each side of every output (a multiple of 16 bytes)
+SENTINEL_BF16 = 0x7BAD
+SENTINEL_F32 = 0x7F8BADBD     # a float32 NaN pattern; fits in int32
+
+
+@pytest.fixture(scope="module")
+def ops(cuda_device):
+    from causal_sliding_window_b200 import ops as _ops
+
+    _ops.attn_device_status(clear=True)
+    return _ops
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+class Guarded:
+    """An output tensor with sentinel-filled guard bands before and after it."""
+
+    def __init__(self, shape, dtype):
+        n = int(np.prod(shape))
+        self.buf = torch.empty(n + 2 * GUARD, dtype=dtype, device="cuda")
+        raw = self.buf.view(torch.int16 if dtype == torch.bfloat16 else torch.int32)
+        raw.fill_(SENTINEL_BF16 if dtype == torch.bfloat16 else SENTINEL_F32)
+        self.t = self.buf[GUARD:GUARD + n].view(shape)
+
+    def guards_intact(self) -> bool:
+        raw = self.buf.view(torch.int16 if self.buf.dtype == torch.bfloat16 else torch.int32)
+        want = SENTINEL_BF16 if self.buf.dtype == torch.bfloat16 else SENTINEL_F32
+        return bool((raw[:GUARD] == want).all() and (raw[-GUARD:] == want).all())
+
+
+def rel_l2(x, ref):
+    return float(np.linalg.norm((x - ref).ravel()) / max(np.linalg.norm(ref.ravel()), 1e-30))
+
+
+def run_fwd_bwd(ops, x, W, with_bwd=True):
+    B, T, H, D = x["B"], x["T"], x["H"], x["D"]
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    o, lse = Guarded((B, T, H, D), torch.bfloat16), Guarded((B, H, T), torch.float32)
+    ops.attn_fwd(q, k, v, o.t, lse.t, W)
+    out = {"o": o, "lse": lse}
+    if with_bwd:
+        do = dev_bf16(x["do"])
+        dq, dk, dv = (Guarded((B, T, H, D), torch.bfloat16) for _ in range(3))
+        ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device="cuda")
+        ops.attn_bwd(q, k, v, o.t, lse.t, do, dq.t, dk.t, dv.t, ws, W)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    for g in out.values():
+        assert g.guards_intact(), "write outside an output buffer"
+    return {n: host_f64(g.t) for n, g in out.items()}
+
+
+SMALL = [
+    # (B, T, H, D, W): the tiny workload, ragged tails, several tiles, odd heads, degenerate windows
+    (1, 128, 2, 64, 128),
+    (1, 128, 2, 64, 32),
+    (2, 333, 3, 128, 333),
+    (2, 333, 3, 128, 100),
+    (2, 333, 3, 128, 129),
+    (2, 333, 3, 128, 1),
+    (1, 300, 2, 64, 10 ** 9),
+    (3, 5, 2, 128, 3),
+    (1, 1, 1, 128, 1),
+    (1, 1, 2, 64, 7),
+    (1, 129, 1, 128, 64),
+    (1, 640, 1, 128, 256),
+    (1, 700, 13, 128, 200),
+    (1, 512, 2, 64, 511),
+]
+
+
+@pytest.mark.parametrize("B,T,H,D,W", SMALL)
+def test_small_shapes_match_oracle_elementwise(ops, B, T, H, D, W):
+    x = inputs.attention_inputs(B, T, H, D, seed=100 + T + H + (W % 1000))
+    got = run_fwd_bwd(ops, x, W)
+    o, lse = oracle_fwd(x["q"], x["k"], x["v"], W)
+    dq, dk, dv = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    assert rel_l2(got["o"], o) <= O_REL
+    assert np.max(np.abs(got["o"] - o)) <= O_ABS
+    assert np.max(np.abs(got["lse"] - lse)) <= LSE_ABS
+    for name, ref in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if np.linalg.norm(ref) == 0:
+            assert np.max(np.abs(got[name])) == 0, name
+        else:
+            assert rel_l2(got[name], ref) <= G_REL, (name, rel_l2(got[name], ref))
+
+
+FULL = [(name, W) for name in ("d12", "d24", "d26") for W in sorted(set(inputs.WORKLOADS[name]["windows"]))]
+
+
+def sample_rows(rng, B, T, H, W, n_rand):
+    fixed_i = sorted(i for i in {0, 1, W - 1, W, T - 1, T // 2, 127, 128} if 0 <= i < T)
+    rows = [(0, 0, i) for i in fixed_i] + [(B - 1, H - 1, i) for i in fixed_i]
+    rows += [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(T))) for _ in range(n_rand)]
+    return np.array(rows, dtype=np.int64)
+
+
+@pytest.mark.parametrize("name,W", FULL)
+def test_full_size_workloads_sampled(ops, name, W):
+    cfg = inputs.WORKLOADS[name]
+    B, T, H, D = cfg["B"], cfg["T"], cfg["H"], cfg["D"]
+    x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"], peaky=cfg["peaky"])
+    got = run_fwd_bwd(ops, x, W)
+    for n, a in got.items():
+        assert np.isfinite(a).all(), n
+    rng = np.random.default_rng(W + H)
+    rows = sample_rows(rng, B, T, H, W, 24)
+    ro, rl = oracle_fwd_rows(x["q"], x["k"], x["v"], W, rows)
+    go = np.stack([got["o"][b, i, h] for b, h, i in rows])
+    gl = np.array([got["lse"][b, h, i] for b, h, i in rows])
+    assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
+    assert np.max(np.abs(gl - rl)) <= LSE_ABS
+    rdq = oracle_dq_rows(x["q"], x["k"], x["v"], x["do"], W, rows)
+    gdq = np.stack([got["dq"][b, i, h] for b, h, i in rows])
+    assert rel_l2(gdq, rdq) <= G_REL
+    krows = sample_rows(rng, B, T, H, W, 4)[:10]
+    rdk, rdv = oracle_dkv_rows(x["q"], x["k"], x["v"], x["do"], W, krows)
+    gdk = np.stack([got["dk"][b, j, h] for b, h, j in krows])
+    gdv = np.stack([got["dv"][b, j, h] for b, h, j in krows])
+    assert rel_l2(gdk, rdk) <= G_REL and rel_l2(gdv, rdv) <= G_REL
+    # Whole-tensor property: key i is always in the band of query i, so lse_i >= scale <q_i, k_i>.
+    qf, kf = inputs.bf16_bits_to_f64(x["q"][0]), inputs.bf16_bits_to_f64(x["k"][0])
+    diag = x["scale"] * np.einsum("thd,thd->ht", qf, kf)
+    assert np.all(got["lse"][0] >= diag - LSE_ABS)
+
+
+def run_decode(ops, x, W, workspace=None, nan_outside=False):
+    B, cap, H, D = x["B"], x["cap"], x["H"], x["D"]
+    kc, vc = x["k_cache"].copy(), x["v_cache"].copy()
+    if nan_outside:
+        for b, L in enumerate(x["cache_len"]):
+            lo = max(0, int(L) - W)
+            kc[b, :lo] = vc[b, :lo] = 0x7FC0       # bf16 NaN in slots before the window
+            kc[b, L:] = vc[b, L:] = 0x7FC0         # and in slots past the cache length
+    cl = torch.from_numpy(x["cache_len"]).cuda()
+    o, lse = Guarded((B, H, D), torch.bfloat16), Guarded((B, H), torch.float32)
+    ws = workspace if workspace is not None else ops.decode_workspace(B, cap, H, D, "cuda")
+    ops.attn_decode(dev_bf16(x["q"]), dev_bf16(kc), dev_bf16(vc), cl, o.t, lse.t, ws, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    assert o.guards_intact() and lse.guards_intact()
+    return host_f64(o.t), host_f64(lse.t), kc, vc
+
+
+def check_decode(got_o, got_l, ref_o, ref_l):
+    assert np.isfinite(got_o).all() and np.isfinite(got_l).all()
+    assert rel_l2(got_o, ref_o) <= O_REL
+    assert np.max(np.abs(got_o - ref_o)) <= O_ABS
+    assert np.max(np.abs(got_l - ref_l)) <= LSE_ABS
+
+
+@pytest.mark.parametrize("W", [2048, 1024])
+def test_decode_workload_matches_oracle(ops, W):
+    c = inputs.DECODE_WORKLOAD
+    x = inputs.decode_inputs(c["B"], c["cap"], c["H"], c["D"], seed=c["seed"])
+    go, gl, _, _ = run_decode(ops, x, W)
+    ro, rl = oracle_decode(x["q"], x["k_cache"], x["v_cache"], x["cache_len"], W)
+    check_decode(go, gl, ro, rl)
+
+
+@pytest.mark.parametrize("H,D,W", [(12, 128, 2048), (12, 128, 100), (13, 128, 64), (3, 64, 1), (40, 128, 300),
+                                   (5, 64, 10 ** 9)])
+def test_decode_edge_lengths_never_read_outside_window(ops, H, D, W):
+    lens = np.array([1, 2, 127, 128, 129, 2048, 64, 65, 1000, 1999])
+    x = inputs.decode_inputs(len(lens), 2048, H, D, seed=H * D + W % 977, cache_len=lens)
+    go, gl, kc, vc = run_decode(ops, x, W, nan_outside=True)
+    ro, rl = oracle_decode(x["q"], kc, vc, x["cache_len"], W)
+    check_decode(go, gl, ro, rl)
+
+
+def test_decode_workspace_reuse_is_stable(ops):
+    x = inputs.decode_inputs(8, 512, 12, 128, seed=5)
+    ws = ops.decode_workspace(8, 512, 12, 128, "cuda")
+    first = run_decode(ops, x, 300, workspace=ws)
+    second = run_decode(ops, x, 300, workspace=ws)
+    assert np.array_equal(first[0], second[0]) and np.array_equal(first[1], second[1])
+    assert int(ws[:256].view(torch.int32)[:8].abs().sum()) == 0   # ticket counters back at zero
+
+
+def test_forward_is_deterministic(ops):
+    x = inputs.attention_inputs(2, 400, 3, 128, seed=9, with_do=False)
+    a = run_fwd_bwd(ops, x, 150, with_bwd=False)
+    b = run_fwd_bwd(ops, x, 150, with_bwd=False)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"])
+
+
+def test_bounded_wait_reports_timeout_without_hanging(ops):
+    assert ops.attn_device_status(clear=True) == 0
+    assert ops.attn_selftest_wait_timeout(200_000) == 0
+    assert ops.attn_device_status(clear=True) == -4       # ATTN_ERR_DEVICE_TIMEOUT
+    assert ops.attn_device_status(clear=True) == 0
+    # The context is still usable afterwards.
+    x = inputs.attention_inputs(1, 64, 1, 64, seed=3, with_do=False)
+    got = run_fwd_bwd(ops, x, 16, with_bwd=False)
+    o, _ = oracle_fwd(x["q"], x["k"], x["v"], 16)
+    assert rel_l2(got["o"], o) <= O_REL
