@@ -199,6 +199,42 @@ def run_reference(args, rank, world):
     return 0
 
 
+def run_case(args):
+    """Profiling helper: `--warmup` untimed then `--steps` calls of one entry point on the d24
+    shape with a reduced batch (inputs still larger than L2), for ncu captures."""
+    import torch
+
+    from causal_sliding_window_b200 import inputs, ops
+
+    dev = torch.device("cuda", 0)
+    cfg = inputs.WORKLOADS["d24"]
+    B, T, H, D, W = args.batch, cfg["T"], cfg["H"], cfg["D"], args.window
+    if args.case == "decode":
+        dc = inputs.DECODE_WORKLOAD
+        x = inputs.decode_inputs(dc["B"], dc["cap"], dc["H"], dc["D"], seed=dc["seed"])
+        q, kc, vc = to_bf16(x["q"], dev), to_bf16(x["k_cache"], dev), to_bf16(x["v_cache"], dev)
+        cl = torch.from_numpy(x["cache_len"]).to(dev)
+        ws = ops.decode_workspace(dc["B"], dc["cap"], dc["H"], dc["D"], dev)
+        call = lambda: ops.decode(q, kc, vc, cl, W, workspace=ws)  # noqa: E731
+    else:
+        x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"])
+        q, k, v, do = (to_bf16(x[n], dev) for n in ("q", "k", "v", "do"))
+        o, lse = ops.forward(q, k, v, W)
+        ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+        if args.case == "fwd":
+            call = lambda: ops.attn_fwd(q, k, v, o, lse, W)  # noqa: E731
+        else:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+            call = lambda: ops.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, W)  # noqa: E731
+    for _ in range(args.warmup + args.steps):
+        call()
+    torch.cuda.synchronize()
+    status = ops.attn_device_status(clear=True)
+    print(json.dumps({"case": args.case, "batch": B, "window": W, "calls": args.warmup + args.steps,
+                      "status": status}))
+    return 0 if status == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -208,12 +244,18 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-log", default=None)
+    ap.add_argument("--case", default="step", choices=["step", "fwd", "bwd", "decode"],
+                    help="profiling mode: run only one call repeatedly on a reduced batch (no metric line)")
+    ap.add_argument("--batch", type=int, default=8, help="batch for --case (d24 shape otherwise)")
+    ap.add_argument("--window", type=int, default=2048, help="window for --case")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.case != "step":
+        return run_case(args)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
@@ -283,6 +325,13 @@ def main():
     mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]  # noqa: E731
     evs = [{"f0": mk(len(windows)), "f1": mk(len(windows)), "bp": mk(len(windows)), "bm": mk(len(windows)),
             "b1": mk(len(windows)), "d0": mk(len(dwins)), "d1": mk(len(dwins))} for _ in range(args.steps)]
+    # torch creates the CUDA event lazily at its first record(); the library records the
+    # backward's inner events by handle, so make every handle exist before the timed region.
+    for e in evs:
+        for lst in e.values():
+            for ev in lst:
+                ev.record(stream)
+    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(gpu_uuid(dev), args.clock_log if rank == 0 else None)
     time.sleep(0.3)

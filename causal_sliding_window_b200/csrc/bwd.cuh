@@ -12,8 +12,10 @@
 //                           zeroed fp32 dQ accumulator
 //   swa_bwd_kernel          one CTA per 128-row key/value tile, walking the
 //                           query tiles of its band; P^T is recomputed from lse,
-//                           dK and dV stay in TMEM, dQ partials are added to the
-//                           fp32 accumulator with vector atomics
+//                           dK and dV stay in TMEM, and each dQ partial tile is
+//                           staged in shared memory (in the Q/dO stage it was
+//                           computed from) and added to the fp32 accumulator by a
+//                           TMA tensor reduce-add
 //   swa_bwd_dq_kernel       dQ = bf16(scale * accumulator)
 //
 // swa_bwd_kernel roles:
@@ -22,7 +24,9 @@
 //                dK += dS^T Q, dQ_i = dS K
 //   warps 0..3   thread = key row: P^T = exp2(S^T*scale*log2e - lse*log2e) with the
 //                band mask, dS^T = P^T (dP^T - Delta) to shared memory
-//   warps 4..7   thread = query row: drain dQ_i from TMEM into the accumulator
+//   warps 4..7   thread = query row: drain dQ_i from TMEM into shared memory; one
+//                thread issues the TMA reduce-add and, once it has read the tile,
+//                hands the stage back to the producer
 //   warps 0..7   epilogue: dV (warps 0..3) and scale*dK (warps 4..7) to bf16
 #pragma once
 
@@ -44,7 +48,8 @@ struct BwdCfg {
     static constexpr int OFF_DS = OFF_QD + NSTAGE * 2 * TILE;   // dS^T: 128 key rows x 128 query cols bf16
     static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;      // per stage: 128 floats lse*log2e, 128 Delta
     static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
-    static constexpr int NUM_BAR = 1 + 2 * NSTAGE + 9;
+    static constexpr int NUM_BAR = 1 + 2 * NSTAGE + 10;
+    static constexpr int DQ_BOX = 128 * 32 * 4;    // one reduce box: 128 query rows x 32 fp32 columns
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
@@ -150,7 +155,7 @@ template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdParams p) {
+               const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -169,7 +174,8 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto qd_empty = [&](int s) { return bar0 + 8u * (1 + C::NSTAGE + s); };
     const uint32_t b9 = bar0 + 8u * (1 + 2 * C::NSTAGE);
     const uint32_t s_full = b9, dp_full = b9 + 8, p_full = b9 + 16, ds_full = b9 + 24, dv_done = b9 + 32,
-                   dq_full = b9 + 40, dq_free = b9 + 48, ds_free = b9 + 56, mma_done = b9 + 64;
+                   dq_full = b9 + 40, dq_free = b9 + 48, ds_free = b9 + 56, mma_done = b9 + 64,
+                   dq_staged = b9 + 72;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
 
@@ -200,6 +206,7 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(dq_free, 128);
         mbar_init(ds_free, 1);
         mbar_init(mma_done, 1);
+        mbar_init(dq_staged, 128);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -307,9 +314,8 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int kk = 0; kk < C::BN / 16; ++kk)
                     mma_ss(tDP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024), sdesc_sw128(sK + kk * 2048, C::BOX, 1024),
                            C::IDESC_DQ, kk > 0);
-                tc_commit(dq_full);
+                tc_commit(dq_full);   // also tells the dQ warps that stage s is no longer read by MMAs
                 tc_commit(ds_free);
-                tc_commit(qd_empty(s));
             }
             tc_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
@@ -325,29 +331,40 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t par = uint32_t(n & 1);
             const long long q0 = (long long)(ilo + n) * C::BM;
             // S^T is committed after the MMA warp saw this stage's loads (Q, dO, lse, Delta) land.
-            const float* lse2_s = reinterpret_cast<const float*>(gbase + C::OFF_LSE + (n % C::NSTAGE) * 1024);
-            const float* delta_s = lse2_s + 128;
+            const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024;   // lse*log2e: 128 floats; Delta 512 bytes later
             ok = __all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
             if (!ok) break;
             tc_fence_after();
-            // Band of this key row: queries kv .. kv+W-1 (and < T).
-            const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
             float pr[C::BM];
 #pragma unroll
             for (int c = 0; c < C::BM / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tS + lane_off + c * 32, r);
+                float lz[32];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float4 t4 = lds_f32x4(sL + (c * 32 + g * 4) * 4);
+                    lz[4 * g] = t4.x;
+                    lz[4 * g + 1] = t4.y;
+                    lz[4 * g + 2] = t4.z;
+                    lz[4 * g + 3] = t4.w;
+                }
                 tmem_ld_wait(r);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int col = c * 32 + i;
-                    float v = ex2_approx(fmaf(__uint_as_float(r[i]), sl2, -lse2_s[col]));
-                    if (!full) {
-                        const long long qq = q0 + col;
-                        if (!(qq >= kv && qq - kv < W && qq < T && kv < T)) v = 0.f;
-                    }
-                    pr[col] = v;
+                    pr[col] = ex2_approx(fmaf(__uint_as_float(r[i]), sl2, -lz[i]));
                 }
+            }
+            // Tiles that cut the diagonal, the window's far edge or T: keep columns clo..chi of this
+            // key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
+            const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
+            if (!full) {
+                const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1));
+                const int chi =
+                    kv < T ? int(imin_ll(imax_ll(imin_ll(kv + W - 1, (long long)T - 1) - q0, -1), C::BM)) : -1;
+#pragma unroll
+                for (int col = 0; col < C::BM; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
             }
 #pragma unroll
             for (int c = 0; c < C::BM / 64; ++c) {
@@ -372,6 +389,15 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int c = 0; c < C::BM / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tDP + lane_off + c * 32, r);
+                float dz[32];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float4 t4 = lds_f32x4(sL + 512 + (c * 32 + g * 4) * 4);
+                    dz[4 * g] = t4.x;
+                    dz[4 * g + 1] = t4.y;
+                    dz[4 * g + 2] = t4.z;
+                    dz[4 * g + 3] = t4.w;
+                }
                 tmem_ld_wait(r);
                 // 32 query columns = four 16-byte chunks of this key row in the 128B-swizzled tile.
 #pragma unroll
@@ -380,8 +406,8 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int col = c * 32 + g * 8 + 2 * e;
-                        const float d0 = pr[col] * (__uint_as_float(r[g * 8 + 2 * e]) - delta_s[col]);
-                        const float d1 = pr[col + 1] * (__uint_as_float(r[g * 8 + 2 * e + 1]) - delta_s[col + 1]);
+                        const float d0 = pr[col] * (__uint_as_float(r[g * 8 + 2 * e]) - dz[g * 8 + 2 * e]);
+                        const float d1 = pr[col + 1] * (__uint_as_float(r[g * 8 + 2 * e + 1]) - dz[g * 8 + 2 * e + 1]);
                         w[e] = pack_bf16x2(d0, d1);
                     }
                     const int chunk = (c * 32 + g * 8) >> 3;            // 0..15 across the 128 columns
@@ -419,13 +445,36 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             tc_fence_before();
             mbar_arrive(dq_free);
-            if (qr < T) {
-                float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t(b) * T + size_t(qr)) * p.H + h) * D);
+            // Stage the fp32 dQ tile over Q_n / dO_n (no MMA reads them any more): D/32 boxes of
+            // 128 rows x 128 bytes, 128-byte swizzled like the TMA box of the reduce.
+            const int s = n % C::NSTAGE;
+            const uint32_t stg = sQD + s * 2 * C::TILE;
 #pragma unroll
-                for (int v4 = 0; v4 < D / 4; ++v4)
-                    atomicAdd(dst + v4, make_float4(acc[4 * v4], acc[4 * v4 + 1], acc[4 * v4 + 2], acc[4 * v4 + 3]));
+            for (int bx = 0; bx < D / 32; ++bx) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t addr = stg + bx * C::DQ_BOX + row * 128 + ((j ^ (row & 7)) << 4);
+                    const float* a4 = acc + bx * 32 + j * 4;
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a4[0]), "f"(a4[1]),
+                                 "f"(a4[2]), "f"(a4[3])
+                                 : "memory");
+                }
             }
+            fence_proxy_async_smem();
+            mbar_arrive(dq_staged);
+            if (threadIdx.x == 128) {
+                ok = mbar_wait(dq_staged, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue);
+                if (ok) {
+                    for (int bx = 0; bx < D / 32; ++bx)
+                        tma_reduce_add_4d(&tm_dqacc, stg + bx * C::DQ_BOX, bx * 32, h, int(qr - row), b);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();   // the stage may be refilled once the reduce has read it
+                    mbar_arrive(qd_empty(s));
+                }
+            }
+            ok = __all_sync(0xffffffffu, ok);
         }
+        if (threadIdx.x == 128) bulk_wait_group0();
     }
 
     // ------------------------------ epilogue: dV, dK ------------------------------

@@ -274,14 +274,15 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
                 }
+                // Tiles that cut the diagonal or the window's left edge: keep columns clo..chi of this
+                // row (keys k0+c with q-W < k0+c <= q).  The test is uniform across the CTA.
                 const long long k0 = (long long)j * C::BN;
                 const bool full = (k0 + C::BN - 1 <= q0[t]) && (k0 > q0[t] + C::BM - 1 - W);
                 if (!full) {
+                    const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN));
+                    const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1));
 #pragma unroll
-                    for (int c = 0; c < C::BN; ++c) {
-                        const long long kv = k0 + c;
-                        if (!(kv <= q && kv > q - W)) s[c] = -INFINITY;
-                    }
+                    for (int c = 0; c < C::BN; ++c) s[c] = (c >= clo && c <= chi) ? s[c] : -INFINITY;
                 }
                 float mx = s[0];
 #pragma unroll

@@ -38,6 +38,21 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // [B, T, H, D] bf16 viewed as a 4-D tensor (D, H, T, B), boxes of 64 x 1 x 128 x 1
 // with 128-byte swizzle (one box = 128 rows of one head, 64 columns).
+// fp32 [B, T, H, D] dQ accumulator as (D, H, T, B), boxes of 32 x 1 x 128 x 1 (128-byte swizzle),
+// target of the backward's TMA reduce-add.
+bool make_dqacc_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+    cuuint64_t strides[3] = {cuuint64_t(D) * 4, cuuint64_t(H) * D * 4, cuuint64_t(T) * H * D * 4};
+    cuuint32_t box[4] = {32, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_bthd_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
     auto enc = encode_fn();
     if (!enc) return false;
@@ -172,6 +187,8 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     float* lse2 = reinterpret_cast<float*>(workspace);
     float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + row_bytes);
     float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * row_bytes);
+    CUtensorMap mdq;
+    if (!make_dqacc_map(&mdq, dq_acc, B, T, H, D)) return ATTN_ERR_LAUNCH;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long long rows = (long long)B * T * H;
     const auto* o_b = reinterpret_cast<const __nv_bfloat16*>(o);
@@ -202,10 +219,10 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     p.wait_limit = kDefaultWaitLimit;
     if (D == 128) {
         if (!ensure_smem((const void*)swa_bwd_kernel<128>, BwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_kernel<128><<<unsigned(grid), BwdCfg<128>::THREADS, BwdCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
+        swa_bwd_kernel<128><<<unsigned(grid), BwdCfg<128>::THREADS, BwdCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, mdq, p);
     } else {
         if (!ensure_smem((const void*)swa_bwd_kernel<64>, BwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_kernel<64><<<unsigned(grid), BwdCfg<64>::THREADS, BwdCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
+        swa_bwd_kernel<64><<<unsigned(grid), BwdCfg<64>::THREADS, BwdCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, mdq, p);
     }
     if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
     if (g_ev_after_main) cudaEventRecord(g_ev_after_main, s);

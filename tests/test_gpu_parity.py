@@ -110,7 +110,10 @@ def test_small_shapes_match_oracle_elementwise(ops, B, T, H, D, W):
     assert np.max(np.abs(got["lse"] - lse)) <= LSE_ABS
     for name, ref in (("dq", dq), ("dk", dk), ("dv", dv)):
         if np.linalg.norm(ref) == 0:
-            assert np.max(np.abs(got[name])) == 0, name
+            # W = 1 (or T = 1): dQ = dK = 0 exactly, since P = 1 and Delta = dP.  The kernel
+            # rounds P, O and Delta, leaving a residue of order 1e-6; a relative norm is
+            # undefined here, so bound the residue absolutely.
+            assert np.max(np.abs(got[name])) <= 1e-4, name
         else:
             assert rel_l2(got[name], ref) <= G_REL, (name, rel_l2(got[name], ref))
 
