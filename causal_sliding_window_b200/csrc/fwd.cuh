@@ -7,17 +7,20 @@
 // "GPT model", architecture features).  Query i attends to keys
 // j in (i - W, i]; W >= T is full causal.
 //
-// One CTA owns two 128-row query tiles of one (b, h) and walks the key/value
-// tiles that intersect the band of either tile:
-//   warp 8      TMA producer: Q tiles once, then K_j, V_j into a ring of stages
+// Persistent: one CTA per SM walks work items (query block of 256 rows, b, h),
+// heaviest query blocks first.  An item is two 128-row query tiles; the CTA
+// walks the key/value tiles that intersect the band of either tile:
+//   warp 8      TMA producer: Q tiles of each item, then K_j, V_j into a ring
+//               of stages that runs on across items
 //   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM, then
 //               O_t += P_t V_j with P_t read from TMEM
 //   warps 0..7  two softmax warpgroups, one per query tile; thread = row.
 //               Online softmax in the exp2 domain, P written back to TMEM as
 //               bf16 over the first half of S_t's columns, O rescaled in TMEM
 //               only when a warp's running max grows by more than 2^8.
-// Key tiles entirely outside the band are never loaded; only tiles that cut
-// the diagonal or the window's left edge are masked element by element.
+// The next item's Q load and first S MMAs overlap the current item's last PV
+// MMAs and epilogue.  Key tiles entirely outside the band are never loaded;
+// only tiles that cut the diagonal or the window's left edge are masked.
 #pragma once
 
 #include "sm100.cuh"
@@ -28,7 +31,7 @@ template <int D>
 struct FwdCfg {
     static constexpr int BM = 128;                  // query rows per tile (one MMA M)
     static constexpr int BN = 128;                  // key rows per tile
-    static constexpr int NQ = 2;                    // query tiles per CTA
+    static constexpr int NQ = 2;                    // query tiles per item
     static constexpr int TILE = 128 * D * 2;        // bytes of a 128 x D bf16 tile
     static constexpr int BOX = 128 * 64 * 2;        // one TMA box: 128 rows x 64 columns
     static constexpr int NBOX = D / 64;
@@ -36,12 +39,13 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = NQ * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    static constexpr int NUM_BAR = 2 * NSTAGE + 4 * NQ + 1;
+    // kv_full, kv_empty per stage; q_full, q_empty; s_full, p_full, o_full, o_free per tile; mma_done
+    static constexpr int NUM_BAR = 2 * NSTAGE + 2 + 4 * NQ + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
     // the kernel checks at run time that the aligned layout fits what it was given.
-    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;   // + slack for 1024-byte alignment
+    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
     static constexpr int THREADS = 320;
     static constexpr uint32_t TMEM_COLS = 512;      // S0 | S1 | O0 | O1
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
@@ -57,8 +61,35 @@ struct FwdParams {
     long long W;
     float scale_log2;     // softmax scale * log2(e)
     int n_qblk;           // ceil(T / 256)
+    int n_items;          // n_qblk * B * H
     long long wait_limit; // clock cycles before a wait gives up
 };
+
+// Geometry of one work item: query block qblk of head (b, h).
+struct FwdItem {
+    int b, h;
+    long long q0;         // first query row of tile 0 (tile 1 starts 128 rows later)
+    bool valid1;          // tile 1 has rows below T
+    int jlo0, jhi0, jlo1, jhi1, jbeg, jend;
+};
+
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
+    FwdItem it;
+    const int BH = p.B * p.H;
+    const int qblk = p.n_qblk - 1 - item / BH;   // heaviest (latest) query blocks first
+    const int bh = item % BH;
+    it.b = bh / p.H;
+    it.h = bh % p.H;
+    it.q0 = (long long)qblk * 256;
+    it.valid1 = it.q0 + 128 < p.T;
+    it.jlo0 = int(imax_ll(0, it.q0 - p.W + 1) / 128);
+    it.jhi0 = int(imin_ll(it.q0 + 127, p.T - 1) / 128);
+    it.jlo1 = int(imax_ll(0, it.q0 + 128 - p.W + 1) / 128);
+    it.jhi1 = int(imin_ll(it.q0 + 255, p.T - 1) / 128);
+    it.jbeg = it.jlo0;
+    it.jend = it.valid1 ? it.jhi1 : it.jhi0;
+    return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
@@ -77,39 +108,21 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t sQ = base + C::OFF_Q;
     const uint32_t sKV = base + C::OFF_KV;
     const uint32_t bar0 = base + C::OFF_BAR;
-    // barrier indices
     auto kv_full = [&](int s) { return bar0 + 8u * s; };
     auto kv_empty = [&](int s) { return bar0 + 8u * (C::NSTAGE + s); };
-    auto q_full = [&](int t) { return bar0 + 8u * (2 * C::NSTAGE + t); };
-    auto s_full = [&](int t) { return bar0 + 8u * (2 * C::NSTAGE + C::NQ + t); };
-    auto p_full = [&](int t) { return bar0 + 8u * (2 * C::NSTAGE + 2 * C::NQ + t); };
-    auto o_full = [&](int t) { return bar0 + 8u * (2 * C::NSTAGE + 3 * C::NQ + t); };
-    const uint32_t mma_done = bar0 + 8u * (2 * C::NSTAGE + 4 * C::NQ);
+    const uint32_t q_full = bar0 + 8u * (2 * C::NSTAGE);
+    const uint32_t q_empty = q_full + 8u;
+    const uint32_t bt = q_full + 16u;   // per-tile barriers start here
+    auto s_full = [&](int t) { return bt + 8u * t; };
+    auto p_full = [&](int t) { return bt + 8u * (C::NQ + t); };
+    auto o_full = [&](int t) { return bt + 8u * (2 * C::NQ + t); };
+    auto o_free = [&](int t) { return bt + 8u * (3 * C::NQ + t); };
+    const uint32_t mma_done = bt + 8u * (4 * C::NQ);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
 
-    // ---- which (query block, b, h) this CTA owns; heaviest query blocks first ----
-    const int BH = p.B * p.H;
-    const int qblk = p.n_qblk - 1 - int(blockIdx.x / BH);
-    const int bh = int(blockIdx.x % BH);
-    const int b = bh / p.H, h = bh % p.H;
     const int T = p.T;
     const long long W = p.W;
-
-    long long q0[C::NQ];
-    bool tvalid[C::NQ];
-    int jlo[C::NQ], jhi[C::NQ];
-#pragma unroll
-    for (int t = 0; t < C::NQ; ++t) {
-        q0[t] = (long long)qblk * (C::BM * C::NQ) + t * C::BM;
-        tvalid[t] = q0[t] < T;
-        jlo[t] = int(imax_ll(0, q0[t] - W + 1) / C::BN);
-        jhi[t] = int(imin_ll(q0[t] + C::BM - 1, T - 1) / C::BN);
-    }
-    const int nt = tvalid[1] ? 2 : 1;
-    const int jbeg = jlo[0];
-    const int jend = jhi[nt - 1];
-
     const int warp = warp_id(), lane = lane_id();
 
     if (threadIdx.x == 0) {
@@ -117,11 +130,13 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(kv_full(s), 1);
             mbar_init(kv_empty(s), 1);
         }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int t = 0; t < C::NQ; ++t) {
-            mbar_init(q_full(t), 1);
             mbar_init(s_full(t), 1);
             mbar_init(p_full(t), 128);
             mbar_init(o_full(t), 1);
+            mbar_init(o_free(t), 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -136,8 +151,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-    const uint32_t tO[2] = {tmem + 256u, tmem + 256u + uint32_t(D)};
+    const uint32_t tS0 = tmem, tS1 = tmem + 128u;
+    const uint32_t tO0 = tmem + 256u, tO1 = tmem + 256u + uint32_t(D);
 
     if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
@@ -145,23 +160,31 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            for (int t = 0; t < nt; ++t) {
-                mbar_arrive_expect_tx(q_full(t), C::TILE);
-                for (int x = 0; x < C::NBOX; ++x)
-                    tma_load_4d(sQ + t * C::TILE + x * C::BOX, &tm_q, q_full(t), x * 64, h, int(q0[t]), b);
-            }
-            int it = 0;
+            int it = 0, qi = 0;
             bool ok = true;
-            for (int j = jbeg; j <= jend && ok; ++j) {
-                for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
-                    const int s = it % C::NSTAGE;
-                    const uint32_t ph = (it / C::NSTAGE) & 1;
-                    ok = mbar_wait(kv_empty(s), ph ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++qi) {
+                const FwdItem g = fwd_item(p, item);
+                // The Q tiles of the previous item are free once its S MMAs completed.
+                if (qi > 0) {
+                    ok = mbar_wait(q_empty, uint32_t((qi - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(kv_full(s), C::TILE);
-                    const CUtensorMap* m = kv ? &tm_v : &tm_k;
+                }
+                mbar_arrive_expect_tx(q_full, (g.valid1 ? 2 : 1) * C::TILE);
+                for (int t = 0; t < (g.valid1 ? 2 : 1); ++t)
                     for (int x = 0; x < C::NBOX; ++x)
-                        tma_load_4d(sKV + s * C::TILE + x * C::BOX, m, kv_full(s), x * 64, h, j * C::BN, b);
+                        tma_load_4d(sQ + t * C::TILE + x * C::BOX, &tm_q, q_full, x * 64, g.h, int(g.q0) + t * 128,
+                                    g.b);
+                for (int j = g.jbeg; j <= g.jend && ok; ++j) {
+                    for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
+                        const int s = it % C::NSTAGE;
+                        const uint32_t ph = (it / C::NSTAGE) & 1;
+                        ok = mbar_wait(kv_empty(s), ph ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(kv_full(s), C::TILE);
+                        const CUtensorMap* m = kv ? &tm_v : &tm_k;
+                        for (int x = 0; x < C::NBOX; ++x)
+                            tma_load_4d(sKV + s * C::TILE + x * C::BOX, m, kv_full(s), x * 64, g.h, j * C::BN, g.b);
+                    }
                 }
             }
             // Drain: make sure no copy is still landing when the CTA exits.
@@ -169,80 +192,114 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int fills = (it - s + C::NSTAGE - 1) / C::NSTAGE;
                 mbar_wait(kv_full(s), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
             }
-            for (int t = 0; t < nt; ++t) mbar_wait(q_full(t), 0, abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            if (qi > 0) mbar_wait(q_full, uint32_t((qi - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             bool ok = true;
-            for (int t = 0; t < nt && ok; ++t) ok = mbar_wait(q_full(t), 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
-            int it = 0;            // ring position of the next tile to consume
-            int npv[2] = {0, 0};   // PV MMAs issued per query tile
+            int it = 0, qi = 0;
+            int npv0 = 0, npv1 = 0;   // PV MMAs issued per tile (all items)
+            int nep0 = 0, nep1 = 0;   // items processed per tile (= epilogues owed)
             auto issue_s = [&](int t, int stage) {
                 const uint32_t qa = sQ + t * C::TILE, ka = sKV + stage * C::TILE;
+                const uint32_t d = t ? tS1 : tS0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), C::IDESC_S,
-                           kk > 0);
+                    mma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), C::IDESC_S, kk > 0);
                 }
                 tc_commit(s_full(t));
             };
-            auto issue_pv = [&](int t, int stage) {
+            auto issue_pv = [&](int t, int stage, bool first) {
                 const uint32_t va = sKV + stage * C::TILE;
+                const uint32_t a = t ? tS1 : tS0, d = t ? tO1 : tO0;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX, 1024), C::IDESC_PV,
-                           (npv[t] > 0 || kk > 0) ? 1u : 0u);
-                ++npv[t];
+                    mma_ts(d, a + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX, 1024), C::IDESC_PV,
+                           (!first || kk > 0) ? 1u : 0u);
                 tc_commit(o_full(t));
             };
-            // Prologue: S_t(jbeg) for the tiles whose band starts there.
-            int sk = 0;
-            if (ok) {
-                sk = it % C::NSTAGE;
+            // S_t overwrites the columns the last PV_t read P from: wait for that PV first.
+            auto s_ready = [&](int t) -> bool {
+                const int n = t ? npv1 : npv0;
+                if (n == 0) return true;
+                if (!mbar_wait(o_full(t), uint32_t((n - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutMma))
+                    return false;
+                tc_fence_after();
+                return true;
+            };
+            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++qi) {
+                const FwdItem g = fwd_item(p, item);
+                auto act = [&](int t, int j) {
+                    return t ? (g.valid1 && j >= g.jlo1 && j <= g.jhi1) : (j >= g.jlo0 && j <= g.jhi0);
+                };
+                ok = mbar_wait(q_full, uint32_t(qi & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+                if (!ok) break;
+                bool first0 = true, first1 = true;
+                int sk = it % C::NSTAGE;
                 ok = mbar_wait(kv_full(sk), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
                 ++it;
-                tc_fence_after();
-                for (int t = 0; t < nt && ok; ++t)
-                    if (jbeg >= jlo[t] && jbeg <= jhi[t]) issue_s(t, sk);
-            }
-            for (int j = jbeg; j <= jend && ok; ++j) {
-                const int sv = it % C::NSTAGE;
-                ok = mbar_wait(kv_full(sv), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                ++it;
                 if (!ok) break;
-                const bool more = j + 1 <= jend;
-                int sk_next = 0;
-                if (more) {
-                    sk_next = it % C::NSTAGE;
-                    ok = mbar_wait(kv_full(sk_next), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                tc_fence_after();
+                if (act(0, g.jbeg)) {
+                    if (!(ok = s_ready(0))) break;
+                    issue_s(0, sk);
+                }
+                if (act(1, g.jbeg)) {
+                    if (!(ok = s_ready(1))) break;
+                    issue_s(1, sk);
+                }
+                for (int j = g.jbeg; j <= g.jend && ok; ++j) {
+                    const int sv = it % C::NSTAGE;
+                    ok = mbar_wait(kv_full(sv), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
                     ++it;
                     if (!ok) break;
-                }
-                for (int t = 0; t < nt && ok; ++t) {
-                    if (j >= jlo[t] && j <= jhi[t]) {
-                        ok = mbar_wait(p_full(t), uint32_t((npv[t]) & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    const bool more = j + 1 <= g.jend;
+                    int sk_next = 0;
+                    if (more) {
+                        sk_next = it % C::NSTAGE;
+                        ok = mbar_wait(kv_full(sk_next), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit,
+                                       kStatusTimeoutMma);
+                        ++it;
                         if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(t, sv);
                     }
-                    if (more && j + 1 >= jlo[t] && j + 1 <= jhi[t]) {
-                        // S_t(j+1) overwrites the columns PV_t(j) reads P from: wait for it.
-                        if (npv[t] > 0) {
-                            ok = mbar_wait(o_full(t), uint32_t((npv[t] - 1) & 1), abort_flag, p.wait_limit,
-                                           kStatusTimeoutMma);
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (!ok) break;
+                        int& npv = t ? npv1 : npv0;
+                        bool& first = t ? first1 : first0;
+                        if (act(t, j)) {
+                            ok = mbar_wait(p_full(t), uint32_t(npv & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
                             if (!ok) break;
+                            if (first) {
+                                // O_t is overwritten: the previous item's epilogue must have read it.
+                                const int nep = t ? nep1 : nep0;
+                                if (nep > 0) {
+                                    ok = mbar_wait(o_free(t), uint32_t((nep - 1) & 1), abort_flag, p.wait_limit,
+                                                   kStatusTimeoutMma);
+                                    if (!ok) break;
+                                }
+                            }
                             tc_fence_after();
+                            issue_pv(t, sv, first);
+                            first = false;
+                            ++npv;
                         }
-                        issue_s(t, sk_next);
+                        if (more && act(t, j + 1)) {
+                            if (!(ok = s_ready(t))) break;
+                            issue_s(t, sk_next);
+                        }
                     }
+                    // K_j (read by the S MMAs issued one step earlier) and V_j are free once the
+                    // MMAs issued so far complete.
+                    tc_commit(kv_empty(sk));
+                    tc_commit(kv_empty(sv));
+                    sk = sk_next;
                 }
-                // K_{j} (consumed by the S MMAs issued one step earlier) and V_j are free once
-                // the MMAs issued so far complete.
-                tc_commit(kv_empty(sk));
-                tc_commit(kv_empty(sv));
-                sk = sk_next;
+                tc_commit(q_empty);   // every S MMA of this item has been issued
+                ++nep0;
+                if (g.valid1) ++nep1;
             }
             tc_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
@@ -252,24 +309,29 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int t = warp >> 2;            // query tile of this warpgroup
         const int quarter = warp & 3;       // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;
-        const long long q = q0[t] + row;    // global query index of this thread
         const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+        const uint32_t tS = (t ? tS1 : tS0) + lane_off, tO = (t ? tO1 : tO0) + lane_off;
         const float sl2 = p.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;
-        int n = 0;
-        bool ok = tvalid[t];
-        const bool active = tvalid[t];
-        if (active) {
-            for (int j = jlo[t]; j <= jhi[t] && ok; ++j, ++n) {
+        int ns = 0;      // S tiles consumed so far (all items): parity of s_full / o_full
+        bool ok = true;
+        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+            const FwdItem g = fwd_item(p, item);
+            if (t == 1 && !g.valid1) continue;
+            const long long qt0 = g.q0 + t * 128;    // first row of this tile
+            const long long q = qt0 + row;           // global query index of this thread
+            const int jlo = t ? g.jlo1 : g.jlo0, jhi = t ? g.jhi1 : g.jhi0;
+            float m_run = -INFINITY, l_run = 0.f;
+            int nloc = 0;
+            for (int j = jlo; j <= jhi && ok; ++j, ++ns, ++nloc) {
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait(s_full(t), uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                                mbar_wait(s_full(t), uint32_t(ns & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
                 float s[C::BN];
 #pragma unroll
                 for (int c = 0; c < C::BN / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld32(tS[t] + lane_off + c * 32, r);
+                    tmem_ld32(tS + c * 32, r);
                     tmem_ld_wait(r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
@@ -277,7 +339,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // Tiles that cut the diagonal or the window's left edge: keep columns clo..chi of this
                 // row (keys k0+c with q-W < k0+c <= q).  The test is uniform across the CTA.
                 const long long k0 = (long long)j * C::BN;
-                const bool full = (k0 + C::BN - 1 <= q0[t]) && (k0 > q0[t] + C::BM - 1 - W);
+                const bool full = (k0 + C::BN - 1 <= qt0) && (k0 > qt0 + C::BM - 1 - W);
                 if (!full) {
                     const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN));
                     const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1));
@@ -305,24 +367,24 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         rowsum += p0 + p1;
                         pk[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st32(tS[t] + lane_off + c * 32, pk);
+                    tmem_st32(tS + c * 32, pk);
                 }
                 l_run = l_run * alpha + rowsum;
                 tmem_st_wait();
-                if (warp_need && n > 0) {
+                if (warp_need && nloc > 0) {
                     // O_t holds the sum up to key tile j-1: wait for PV_t(j-1), then rescale.
-                    ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((n - 1) & 1), abort_flag,
+                    ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((ns - 1) & 1), abort_flag,
                                                            p.wait_limit, kStatusTimeoutSoftmax));
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t r[32];
-                        tmem_ld32(tO[t] + lane_off + c * 32, r);
+                        tmem_ld32(tO + c * 32, r);
                         tmem_ld_wait(r);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(tO[t] + lane_off + c * 32, r);
+                        tmem_st32(tO + c * 32, r);
                     }
                     tmem_st_wait();
                 }
@@ -330,34 +392,36 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tc_fence_before();
                 mbar_arrive(p_full(t));
             }
+            if (!ok || nloc == 0) break;
             // ---- epilogue: O = O / l, lse = ln(sum exp S) ----
-            if (ok && n > 0)
-                ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((n - 1) & 1), abort_flag, p.wait_limit,
-                                                       kStatusTimeoutEpilogue));
-            if (ok && n > 0) {
-                tc_fence_after();
+            ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((ns - 1) & 1), abort_flag, p.wait_limit,
+                                                   kStatusTimeoutEpilogue));
+            if (!ok) break;
+            tc_fence_after();
+            float ov[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tO + c * 32, r);
+                tmem_ld_wait(r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ov[c * 32 + i] = __uint_as_float(r[i]);
+            }
+            tc_fence_before();
+            mbar_arrive(o_free(t));   // the next item's first PV may overwrite O_t now
+            if (q < T) {
                 const float inv_l = 1.f / l_run;
-                const bool in_range = q < T;
-                __nv_bfloat16* orow = p.o + ((size_t(b) * T + size_t(in_range ? q : 0)) * p.H + h) * D;
+                __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tO[t] + lane_off + c * 32, r);
-                    tmem_ld_wait(r);
-                    if (in_range) {
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * inv_l, __uint_as_float(r[v4 * 8 + 1]) * inv_l);
-                            w.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * inv_l, __uint_as_float(r[v4 * 8 + 3]) * inv_l);
-                            w.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * inv_l, __uint_as_float(r[v4 * 8 + 5]) * inv_l);
-                            w.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * inv_l, __uint_as_float(r[v4 * 8 + 7]) * inv_l);
-                            *reinterpret_cast<uint4*>(orow + c * 32 + v4 * 8) = w;
-                        }
-                    }
+                for (int v8 = 0; v8 < D / 8; ++v8) {
+                    uint4 w;
+                    w.x = pack_bf16x2(ov[v8 * 8 + 0] * inv_l, ov[v8 * 8 + 1] * inv_l);
+                    w.y = pack_bf16x2(ov[v8 * 8 + 2] * inv_l, ov[v8 * 8 + 3] * inv_l);
+                    w.z = pack_bf16x2(ov[v8 * 8 + 4] * inv_l, ov[v8 * 8 + 5] * inv_l);
+                    w.w = pack_bf16x2(ov[v8 * 8 + 6] * inv_l, ov[v8 * 8 + 7] * inv_l);
+                    *reinterpret_cast<uint4*>(orow + v8 * 8) = w;
                 }
-                if (in_range)
-                    p.lse[(size_t(b) * p.H + h) * T + q] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+                p.lse[(size_t(g.b) * p.H + g.h) * T + q] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
             }
         }
     }

@@ -79,6 +79,20 @@ bool ensure_smem(const void* func, int bytes) {
     return true;
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
 bool valid_common(int B, int T, int H, int D, int W, float scale) {
     if (B < 1 || T < 1 || H < 1 || W < 1) return false;
     if (!(scale > 0.f) || scale != scale || scale > 3.4e38f) return false;
@@ -130,8 +144,9 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     if (!valid_common(B, T, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     const int n_qblk = (T + 255) / 256;
-    const long long grid = (long long)n_qblk * B * H;
-    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long n_items = (long long)n_qblk * B * H;
+    if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
     CUtensorMap mq, mk, mv;
     if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, H, D) || !make_bthd_map(&mv, v, B, T, H, D))
         return ATTN_ERR_LAUNCH;
@@ -144,6 +159,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_qblk = n_qblk;
+    p.n_items = int(n_items);
     p.wait_limit = kDefaultWaitLimit;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (D == 128) {
