@@ -59,6 +59,23 @@ def decode_bytes(cache_len, H, D, W):
     return int(n.sum()) * H * D * 2 * 2 + 2 * B * H * D * 2
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_rank_step * world * steps / (max_ms * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -82,7 +99,7 @@ class ClockSampler:
             self.out = open(path, "w") if path else subprocess.PIPE
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=self.out, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
@@ -238,7 +255,7 @@ def run_case(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -352,10 +369,7 @@ def main():
     t_bmain = sum(e["bp"][i].elapsed_time(e["bm"][i]) for e in evs for i in range(len(windows)))
     t_conv = sum(e["bm"][i].elapsed_time(e["b1"][i]) for e in evs for i in range(len(windows)))
     t_dec = sum(e["d0"][i].elapsed_time(e["d1"][i]) for e in evs for i in range(len(dwins)))
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dev)
     finite = bool(torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all()
                   and torch.isfinite(d_o.float()).all())
 
@@ -390,14 +404,12 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
         K = args.steps
-        value = step_flops * world * K / (ms_max * 1e-3) / 1e12
+        value = weak_scaling_value(step_flops, world, K, ms_max)
         fwd_tf = step_fwd_flops * K / (t_fwd * 1e-3) / 1e12
         bmain_tf = step_bwd_flops * K / (t_bmain * 1e-3) / 1e12
         bwd_tf = step_bwd_flops * K / ((t_pre + t_bmain + t_conv) * 1e-3) / 1e12
@@ -424,7 +436,7 @@ def main():
             cb = cpu_baseline_sample(cfg, att)
             cb.pop("seconds")
             cpu = cb
-        e2e_val = step_flops * world / (float(e2e_ms.item()) * 1e-3) / 1e12
+        e2e_val = weak_scaling_value(step_flops, world, 1, e2e_ms)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
