@@ -248,7 +248,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
 }
 
 size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
-    if (B < 1 || cap < 1 || H < 1 || D < 1) return 0;
+    if (B < 1 || cap < 1 || H < 1 || (D != 64 && D != 128)) return 0;
     const size_t nsm = size_t((cap + kDecodeChunk - 1) / kDecodeChunk);
     const size_t nhg = size_t((H + kDecodeThreads / (D / 8) - 1) / (kDecodeThreads / (D / 8)));
     return align256(size_t(B) * nhg * 4) + align256(size_t(B) * nsm * H * 2 * 4) +

@@ -88,7 +88,8 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
              void* workspace, size_t ws_bytes, int B, int T, int H, int D, int W, float scale,
              void* stream);
 
-/* Bytes of workspace attn_decode needs for B sequences of capacity cap (any W). */
+/* Bytes of workspace attn_decode needs for B sequences of capacity cap (any W); 0 for
+ * sizes attn_decode rejects (B, cap or H below 1, D not 64 or 128). */
 size_t attn_decode_workspace_bytes(int B, int cap, int H, int D);
 
 /*

@@ -77,6 +77,8 @@ def test_workspace_sizes():
     assert ops.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
     assert ops.attn_decode_workspace_bytes(32, 2048, 12, 128) > 32 * 32 * 12 * 128 * 4
     assert ops.attn_decode_workspace_bytes(1, 0, 1, 64) == 0
+    for bad_d in (0, 4, 7, 96):
+        assert ops.attn_decode_workspace_bytes(1, 16, 1, bad_d) == 0
 
 
 def dec(q=A, cl=A, ws=A, ws_bytes=None, B=2, cap=64, H=2, D=128, W=8, scale=0.1, lse=A):
