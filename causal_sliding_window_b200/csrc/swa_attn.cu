@@ -132,6 +132,31 @@ __global__ void swa_selftest_wait_kernel(long long limit_cycles) {
     __syncthreads();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed decode scratch for callers that cannot allocate device memory
+// (attn_decode_noalloc).  Every GPU that loads this library holds the array
+// until the process exits.  Host code may not pass the array's name to a
+// kernel (on the host it is only a stand-in symbol); its device address is
+// looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+// Device address of g_decode_scratch on the current device (set up on first use per device).
+void* noalloc_scratch() {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    if (addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -299,6 +324,24 @@ int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v
     else
         swa_decode_kernel<64><<<grid, threads, 0, s>>>(p);
     return launch_status();
+}
+
+int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                        const int32_t* cache_len, attn_bf16* o, float* lse, int B, int cap, int H, int D, int W,
+                        float scale, void* stream) {
+    const size_t need = attn_decode_workspace_bytes(B, cap, H, D);
+    if (need == 0) return (D != 64 && D != 128 && B >= 1 && cap >= 1 && H >= 1) ? ATTN_ERR_UNSUPPORTED
+                                                                                : ATTN_ERR_INVALID_ARG;
+    if (need > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;
+    void* ws = noalloc_scratch();
+    if (ws == nullptr) return ATTN_ERR_LAUNCH;
+    // The ticket counters at the start of the scratch must be zero when a call begins.
+    const int heads_per_cta = kDecodeThreads / (D / 8);
+    const size_t counter_bytes = size_t(B) * ((H + heads_per_cta - 1) / heads_per_cta) * 4;
+    if (cudaMemsetAsync(ws, 0, counter_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
+    return attn_decode(q, k_cache, v_cache, cache_len, o, lse, ws, kNoAllocScratchBytes, B, cap, H, D, W, scale,
+                       stream);
 }
 
 int attn_bwd_set_profile_events(void* after_pre, void* after_main) {

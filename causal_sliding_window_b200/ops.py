@@ -41,6 +41,8 @@ _lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
 _lib.attn_decode_workspace_bytes.restype = _sz
 _lib.attn_decode.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode.restype = _i
+_lib.attn_decode_noalloc.argtypes = [_p] * 6 + [_i, _i, _i, _i, _i, _f, _p]
+_lib.attn_decode_noalloc.restype = _i
 _lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
 _lib.attn_bwd_set_profile_events.restype = _i
 _lib.attn_device_status.argtypes = [_i]
@@ -51,7 +53,7 @@ _lib.attn_status_string.argtypes = [_i]
 _lib.attn_status_string.restype = ctypes.c_char_p
 
 EXPORTED = ["attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_decode_workspace_bytes", "attn_decode",
-            "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
+            "attn_decode_noalloc", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
             "attn_status_string"]
 
 
@@ -126,6 +128,21 @@ def attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W: int, scale
     _check(_lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), _ptr(o), _ptr(lse),
                             _ptr(workspace), ws_bytes, B, cap, H, D, int(W), _scale(scale, D), _stream(stream)),
            "attn_decode")
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, cache_len, o, lse, W: int, scale=None, stream=None):
+    """attn_decode on the library's fixed 8 MiB scratch, for callers that cannot allocate.
+
+    Shares one scratch array across calls: do not overlap calls on the GPU.  The first
+    call on a device performs a one-time address lookup; make it before stream capture.
+    """
+    B, cap, H, D = _bthd(k_cache, v_cache)
+    if tuple(q.shape) != (B, H, D) or tuple(o.shape) != (B, H, D) or q.dtype != torch.bfloat16:
+        raise ValueError("q and o must be bf16 [B, H, D]")
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or not cache_len.is_cuda:
+        raise ValueError("cache_len must be an int32 CUDA tensor of shape [B]")
+    _check(_lib.attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), _ptr(o), _ptr(lse),
+                                    B, cap, H, D, int(W), _scale(scale, D), _stream(stream)), "attn_decode_noalloc")
 
 
 def attn_bwd_set_profile_events(after_pre=None, after_main=None):

@@ -112,6 +112,29 @@ int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v
                 int B, int cap, int H, int D, int W, float scale, void* stream);
 
 /*
+ * attn_decode without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code that issues its work while a CUDA graph is
+ * being captured (cudaMalloc is not allowed there), plugins whose host engine
+ * owns a fixed device-memory arena and forbids allocation, and latency-bound
+ * token loops where an allocation would synchronise the device.
+ * The paper has no counterpart: this is a deployment convenience.
+ *   Arguments as for attn_decode, minus workspace / ws_bytes.
+ *   Scratch: a fixed 8 MiB device array inside the library (held by every GPU
+ *   that loads it until exit).  Sizes whose attn_decode_workspace_bytes
+ *   exceeds 8 MiB return ATTN_ERR_WORKSPACE; unsupported D returns
+ *   ATTN_ERR_UNSUPPORTED, other bad sizes ATTN_ERR_INVALID_ARG.
+ *   The first call on a device looks up the array's device address (set-up,
+ *   with that device current); make that first call before any stream capture.
+ *   Each call zeroes the scratch's ticket counters on `stream`, then runs
+ *   attn_decode on it.  All calls share the one array: calls that overlap on
+ *   the GPU (other streams, other threads) race and must be serialised by the
+ *   caller.  Allocates nothing.
+ */
+int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                        const int32_t* cache_len, attn_bf16* o, float* lse, int B, int cap, int H, int D, int W,
+                        float scale, void* stream);
+
+/*
  * Profiling aid: when set (non-NULL cudaEvent_t handles), every later
  * attn_bwd call made from this host thread records `after_pre` on its stream
  * right after the Delta / accumulator-zeroing launch and `after_main` right
