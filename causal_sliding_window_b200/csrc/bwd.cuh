@@ -10,8 +10,10 @@
 //   swa_bwd_pre_kernel      Delta and lse*log2(e) as fp32 rows [B*H, Tp] padded to
 //                           Tp = 128*ceil(T/128) (padding: Delta 0, lse +inf), and a
 //                           zeroed fp32 dQ accumulator
-//   swa_bwd_kernel          one CTA per 128-row key/value tile, walking the
-//                           query tiles of its band; P^T is recomputed from lse,
+//   swa_bwd_kernel          persistent (one CTA per SM) drawing items = 128-row key/value
+//                           tile of one (b, h) from a launch-wide counter (head-major,
+//                           lowest key tiles first), walking the
+//                           query tiles of each item's band; P^T is recomputed from lse,
 //                           dK and dV stay in TMEM, and each dQ partial tile is
 //                           staged in shared memory (in the Q/dO stage it was
 //                           computed from) and added to the fp32 accumulator by a
@@ -27,7 +29,8 @@
 //   warps 4..7   thread = query row: drain dQ_i from TMEM into shared memory; one
 //                thread issues the TMA reduce-add and, once it has read the tile,
 //                hands the stage back to the producer
-//   warps 0..7   epilogue: dV (warps 0..3) and scale*dK (warps 4..7) to bf16
+//   warps 0..7   per-item epilogue: dV (warps 0..3) and scale*dK (warps 4..7) to bf16,
+//                overlapping the next item's first steps (acc_full / acc_free barriers)
 #pragma once
 
 #include "sm100.cuh"
@@ -48,7 +51,9 @@ struct BwdCfg {
     static constexpr int OFF_DS = OFF_QD + NSTAGE * 2 * TILE;   // dS^T: 128 key rows x 128 query cols bf16
     static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;      // per stage: 128 floats lse*log2e, 128 Delta
     static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
-    static constexpr int NUM_BAR = 1 + 2 * NSTAGE + 10;
+    // kv_full, kv_empty, qd_full x2, qd_empty x2, s_full, dp_full, p_full, ds_full, dv_done, dq_full,
+    // dq_free, ds_free, mma_done, dq_staged, acc_full, acc_free; item_full, item_empty per ring entry
+    static constexpr int NUM_BAR = 2 + 2 * NSTAGE + 12 + 2 * kItemRing;
     static constexpr int DQ_BOX = 128 * 32 * 4;    // one reduce box: 128 query rows x 32 fp32 columns
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
@@ -74,9 +79,33 @@ struct BwdParams {
     float scale;
     float scale_log2;
     int n_kblk;
+    int n_items;          // n_kblk * B * H
+    int work_slot;        // index into g_work_slots for this launch
     int Tp;               // T rounded up to 128
     long long wait_limit;
 };
+
+// Geometry of one work item: key block kblk of head (b, h).  Items are head-major (all key
+// blocks of one head, lowest first, then the next head), so the CTAs that run at the same
+// time read the same head's Q / dO tiles and share them through L2.
+struct BwdItem {
+    int b, h, bh;
+    long long k0;         // first key row
+    int ilo, nsteps;      // first query tile and number of query tiles in the band
+};
+
+__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
+    BwdItem it;
+    const int kblk = item % p.n_kblk;
+    it.bh = item / p.n_kblk;
+    it.b = it.bh / p.H;
+    it.h = it.bh % p.H;
+    it.k0 = (long long)kblk * 128;
+    it.ilo = int(it.k0 / 128);
+    const int ihi = int(imin_ll(p.T - 1, it.k0 + 127 + p.W - 1) / 128);
+    it.nsteps = ihi - it.ilo + 1;
+    return it;
+}
 
 // ---------------------------------------------------------------------------
 // Delta_i = sum_d dO_id * O_id and zeroing of the dQ accumulator.
@@ -169,30 +198,24 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQD = base + C::OFF_QD, sDS = base + C::OFF_DS;
     const uint32_t sLSE = base + C::OFF_LSE;   // stage s: lse2 at sLSE + s*1024, Delta 512 bytes later
     const uint32_t bar0 = base + C::OFF_BAR;
-    const uint32_t kv_full = bar0;
-    auto qd_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto qd_empty = [&](int s) { return bar0 + 8u * (1 + C::NSTAGE + s); };
-    const uint32_t b9 = bar0 + 8u * (1 + 2 * C::NSTAGE);
-    const uint32_t s_full = b9, dp_full = b9 + 8, p_full = b9 + 16, ds_full = b9 + 24, dv_done = b9 + 32,
-                   dq_full = b9 + 40, dq_free = b9 + 48, ds_free = b9 + 56, mma_done = b9 + 64,
-                   dq_staged = b9 + 72;
+    const uint32_t kv_full = bar0, kv_empty = bar0 + 8;
+    auto qd_full = [&](int s) { return bar0 + 8u * (2 + s); };
+    auto qd_empty = [&](int s) { return bar0 + 8u * (2 + C::NSTAGE + s); };
+    const uint32_t bb = bar0 + 8u * (2 + 2 * C::NSTAGE);
+    const uint32_t s_full = bb, dp_full = bb + 8, p_full = bb + 16, ds_full = bb + 24, dv_done = bb + 32,
+                   dq_full = bb + 40, dq_free = bb + 48, ds_free = bb + 56, mma_done = bb + 64,
+                   dq_staged = bb + 72, acc_full = bb + 80, acc_free = bb + 88;
+    const uint32_t item_full0 = bb + 96, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
+    volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
 
-    const int BH = p.B * p.H;
-    const int kblk = int(blockIdx.x / BH);          // low key blocks have the most query tiles: first
-    const int bh = int(blockIdx.x % BH);
-    const int b = bh / p.H, h = bh % p.H;
     const int T = p.T;
     const long long W = p.W;
-    const long long k0 = (long long)kblk * C::BN;
-    const int ilo = int(k0 / C::BM);
-    const int ihi = int(imin_ll(T - 1, k0 + C::BN - 1 + W - 1) / C::BM);
-    const int nsteps = ihi - ilo + 1;
-
     const int warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
+        mbar_init(kv_empty, 1);
         for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(qd_full(s), 1);
             mbar_init(qd_empty(s), 1);
@@ -207,6 +230,12 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(ds_free, 1);
         mbar_init(mma_done, 1);
         mbar_init(dq_staged, 128);
+        mbar_init(acc_full, 1);
+        mbar_init(acc_free, 256);
+        for (int e = 0; e < kItemRing; ++e) {
+            mbar_init(item_full0 + 8u * e, 1);
+            mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and warps 0..7
+        }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -228,94 +257,122 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
-            for (int x = 0; x < C::NBOX; ++x) {
-                tma_load_4d(sK + x * C::BOX, &tm_k, kv_full, x * 64, h, int(k0), b);
-                tma_load_4d(sV + x * C::BOX, &tm_v, kv_full, x * 64, h, int(k0), b);
-            }
-            int n = 0;
-            for (; n < nsteps; ++n) {
-                const int s = n % C::NSTAGE;
-                if (!mbar_wait(qd_empty(s), ((n / C::NSTAGE) & 1) ^ 1u, abort_flag, p.wait_limit,
-                               kStatusTimeoutProducer))
-                    break;
-                const int qrow = (ilo + n) * C::BM;
-                mbar_arrive_expect_tx(qd_full(s), 2 * C::TILE + 1024);
-                const uint32_t dst = sQD + s * 2 * C::TILE;
-                for (int x = 0; x < C::NBOX; ++x) {
-                    tma_load_4d(dst + x * C::BOX, &tm_q, qd_full(s), x * 64, h, qrow, b);
-                    tma_load_4d(dst + C::TILE + x * C::BOX, &tm_do, qd_full(s), x * 64, h, qrow, b);
+            int n = 0, ki = 0;   // query-tile steps and items issued so far
+            bool ok = true;
+            for (;; ++ki) {
+                const int item =
+                    item_produce(p.work_slot, ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                if (!ok || item >= p.n_items) break;
+                const BwdItem g = bwd_item(p, item);
+                // K/V of the previous item are free once its last MMA completed.
+                if (ki > 0) {
+                    ok = mbar_wait(kv_empty, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                    if (!ok) break;
                 }
-                const size_t row = size_t(bh) * p.Tp + size_t(qrow);
-                bulk_load(sLSE + s * 1024, p.lse2 + row, 512, qd_full(s));
-                bulk_load(sLSE + s * 1024 + 512, p.delta + row, 512, qd_full(s));
+                mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+                for (int x = 0; x < C::NBOX; ++x) {
+                    tma_load_4d(sK + x * C::BOX, &tm_k, kv_full, x * 64, g.h, int(g.k0), g.b);
+                    tma_load_4d(sV + x * C::BOX, &tm_v, kv_full, x * 64, g.h, int(g.k0), g.b);
+                }
+                for (int l = 0; l < g.nsteps; ++l, ++n) {
+                    const int s = n % C::NSTAGE;
+                    if (!(ok = mbar_wait(qd_empty(s), ((n / C::NSTAGE) & 1) ^ 1u, abort_flag, p.wait_limit,
+                                         kStatusTimeoutProducer)))
+                        break;
+                    const int qrow = (g.ilo + l) * C::BM;
+                    mbar_arrive_expect_tx(qd_full(s), 2 * C::TILE + 1024);
+                    const uint32_t dst = sQD + s * 2 * C::TILE;
+                    for (int x = 0; x < C::NBOX; ++x) {
+                        tma_load_4d(dst + x * C::BOX, &tm_q, qd_full(s), x * 64, g.h, qrow, g.b);
+                        tma_load_4d(dst + C::TILE + x * C::BOX, &tm_do, qd_full(s), x * 64, g.h, qrow, g.b);
+                    }
+                    const size_t row = size_t(g.bh) * p.Tp + size_t(qrow);
+                    bulk_load(sLSE + s * 1024, p.lse2 + row, 512, qd_full(s));
+                    bulk_load(sLSE + s * 1024 + 512, p.delta + row, 512, qd_full(s));
+                }
             }
+            work_slot_finish(p.work_slot);
+            // Drain: make sure no copy is still landing when the CTA exits.
             for (int s = 0; s < C::NSTAGE && s < n; ++s) {
                 const int fills = (n - s + C::NSTAGE - 1) / C::NSTAGE;
                 mbar_wait(qd_full(s), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
             }
-            mbar_wait(kv_full, 0, abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            if (ki > 0) mbar_wait(kv_full, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            bool ok = mbar_wait(kv_full, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
-            for (int n = 0; n < nsteps && ok; ++n) {
-                const int s = n % C::NSTAGE;
-                const uint32_t par = uint32_t(n & 1);
-                ok = mbar_wait(qd_full(s), (n / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                if (!ok) break;
-                const uint32_t sQ = sQD + s * 2 * C::TILE, sDO = sQ + C::TILE;
-                // S^T overwrites the P^T columns read by dV of the previous step.
-                if (n > 0) {
-                    ok = mbar_wait(dv_done, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
+            bool ok = true;
+            int n = 0, ki = 0;
+            for (;; ++ki) {
+                const int item = item_consume_thread(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                                     kStatusTimeoutMma, ok);
+                if (!ok || item >= p.n_items) break;
+                const BwdItem g = bwd_item(p, item);
+                ok = mbar_wait(kv_full, uint32_t(ki & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+                for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
+                    const int s = n % C::NSTAGE;
+                    const uint32_t par = uint32_t(n & 1);
+                    ok = mbar_wait(qd_full(s), (n / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
                     if (!ok) break;
-                }
-                tc_fence_after();
+                    const uint32_t sQ = sQD + s * 2 * C::TILE, sDO = sQ + C::TILE;
+                    // S^T overwrites the P^T columns read by dV of the previous step.
+                    if (n > 0) {
+                        ok = mbar_wait(dv_done, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), C::IDESC_S, kk > 0);
-                }
-                tc_commit(s_full);
-                // dP^T reuses the columns the dQ drain of the previous step reads.
-                if (n > 0) {
-                    ok = mbar_wait(dq_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                        mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), C::IDESC_S,
+                               kk > 0);
+                    }
+                    tc_commit(s_full);
+                    // dP^T reuses the columns the dQ drain of the previous step reads.
+                    if (n > 0) {
+                        ok = mbar_wait(dq_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                        mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), C::IDESC_S,
+                               kk > 0);
+                    }
+                    tc_commit(dp_full);
+                    // dV += P^T dO  (the previous item's epilogue must have read dV / dK first)
+                    ok = mbar_wait(p_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    if (ok && l == 0 && ki > 0)
+                        ok = mbar_wait(acc_free, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
                     if (!ok) break;
                     tc_fence_after();
-                }
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), C::IDESC_S,
-                           kk > 0);
+                    for (int kk = 0; kk < C::BM / 16; ++kk)
+                        mma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
+                               (l > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(dv_done);
+                    // dK += dS^T Q ; dQ_i = dS K
+                    ok = mbar_wait(ds_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C::BM / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                        mma_ss(tDK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, C::BOX, 1024),
+                               C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; ++kk)
+                        mma_ss(tDP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
+                               sdesc_sw128(sK + kk * 2048, C::BOX, 1024), C::IDESC_DQ, kk > 0);
+                    tc_commit(dq_full);   // also tells the dQ warps that stage s is no longer read by MMAs
+                    tc_commit(ds_free);
                 }
-                tc_commit(dp_full);
-                // dV += P^T dO
-                ok = mbar_wait(p_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
                 if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; ++kk)
-                    mma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
-                           (n > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(dv_done);
-                // dK += dS^T Q ; dQ_i = dS K
-                ok = mbar_wait(ds_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < C::BM / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tDK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, C::BOX, 1024),
-                           C::IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ss(tDP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024), sdesc_sw128(sK + kk * 2048, C::BOX, 1024),
-                           C::IDESC_DQ, kk > 0);
-                tc_commit(dq_full);   // also tells the dQ warps that stage s is no longer read by MMAs
-                tc_commit(ds_free);
+                tc_commit(acc_full);   // dV, dK of this item are final
+                tc_commit(kv_empty);   // K, V may be replaced by the next item's
             }
             tc_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
@@ -323,192 +380,231 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp < 4) {
         // ------------------------------ key-row warps: P^T and dS^T ------------------------------
         const int row = warp * 32 + lane;
-        const long long kv = k0 + row;
         const uint32_t lane_off = uint32_t(warp * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
-        for (int n = 0; n < nsteps && ok; ++n) {
-            const uint32_t par = uint32_t(n & 1);
-            const long long q0 = (long long)(ilo + n) * C::BM;
-            // S^T is committed after the MMA warp saw this stage's loads (Q, dO, lse, Delta) land.
-            const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024;   // lse*log2e: 128 floats; Delta 512 bytes later
-            ok = __all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
-            if (!ok) break;
-            tc_fence_after();
-            float pr[C::BM];
-#pragma unroll
-            for (int c = 0; c < C::BM / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tS + lane_off + c * 32, r);
-                float lz[32];
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const float4 t4 = lds_f32x4(sL + (c * 32 + g * 4) * 4);
-                    lz[4 * g] = t4.x;
-                    lz[4 * g + 1] = t4.y;
-                    lz[4 * g + 2] = t4.z;
-                    lz[4 * g + 3] = t4.w;
-                }
-                tmem_ld_wait(r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int col = c * 32 + i;
-                    pr[col] = ex2_approx(fmaf(__uint_as_float(r[i]), sl2, -lz[i]));
-                }
-            }
-            // Tiles that cut the diagonal, the window's far edge or T: keep columns clo..chi of this
-            // key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
-            const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
-            if (!full) {
-                const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1));
-                const int chi =
-                    kv < T ? int(imin_ll(imax_ll(imin_ll(kv + W - 1, (long long)T - 1) - q0, -1), C::BM)) : -1;
-#pragma unroll
-                for (int col = 0; col < C::BM; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
-            }
-#pragma unroll
-            for (int c = 0; c < C::BM / 64; ++c) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[c * 64 + 2 * i], pr[c * 64 + 2 * i + 1]);
-                tmem_st32(tS + lane_off + c * 32, pk);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(p_full);
-            // dS^T = P^T (dP^T - Delta)
-            ok = __all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
-            if (!ok) break;
-            tc_fence_after();
-            if (n > 0) {
+        int n = 0, ki = 0;
+        for (;; ++ki) {
+            const int item = item_consume_warp(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                               kStatusTimeoutSoftmax, ok);
+            if (!ok || item >= p.n_items) break;
+            const BwdItem g = bwd_item(p, item);
+            const long long k0 = g.k0;
+            const long long kv = k0 + row;
+            for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
+                const uint32_t par = uint32_t(n & 1);
+                const long long q0 = (long long)(g.ilo + l) * C::BM;
+                const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024;   // lse*log2e: 128 floats; Delta 512 bytes later
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait(ds_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                                mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
-            }
+                tc_fence_after();
+                float pr[C::BM];
 #pragma unroll
-            for (int c = 0; c < C::BM / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tDP + lane_off + c * 32, r);
-                float dz[32];
+                for (int c = 0; c < C::BM / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + lane_off + c * 32, r);
+                    float lz[32];
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const float4 t4 = lds_f32x4(sL + 512 + (c * 32 + g * 4) * 4);
-                    dz[4 * g] = t4.x;
-                    dz[4 * g + 1] = t4.y;
-                    dz[4 * g + 2] = t4.z;
-                    dz[4 * g + 3] = t4.w;
-                }
-                tmem_ld_wait(r);
-                // 32 query columns = four 16-byte chunks of this key row in the 128B-swizzled tile.
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int col = c * 32 + g * 8 + 2 * e;
-                        const float d0 = pr[col] * (__uint_as_float(r[g * 8 + 2 * e]) - dz[g * 8 + 2 * e]);
-                        const float d1 = pr[col + 1] * (__uint_as_float(r[g * 8 + 2 * e + 1]) - dz[g * 8 + 2 * e + 1]);
-                        w[e] = pack_bf16x2(d0, d1);
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 t4 = lds_f32x4(sL + (c * 32 + gq * 4) * 4);
+                        lz[4 * gq] = t4.x;
+                        lz[4 * gq + 1] = t4.y;
+                        lz[4 * gq + 2] = t4.z;
+                        lz[4 * gq + 3] = t4.w;
                     }
-                    const int chunk = (c * 32 + g * 8) >> 3;            // 0..15 across the 128 columns
-                    const int box = chunk >> 3, cib = chunk & 7;
-                    const uint32_t addr = sDS + box * C::BOX + row * 128 + ((cib ^ (row & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
-                                 "r"(w[2]), "r"(w[3])
-                                 : "memory");
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) pr[c * 32 + i] = ex2_approx(fmaf(__uint_as_float(r[i]), sl2, -lz[i]));
+                }
+                // Tiles that cut the diagonal, the window's far edge or T: keep columns clo..chi of this
+                // key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
+                const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
+                if (!full) {
+                    const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1));
+                    const int chi =
+                        kv < T ? int(imin_ll(imax_ll(imin_ll(kv + W - 1, (long long)T - 1) - q0, -1), C::BM)) : -1;
+#pragma unroll
+                    for (int col = 0; col < C::BM; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < C::BM / 64; ++c) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[c * 64 + 2 * i], pr[c * 64 + 2 * i + 1]);
+                    tmem_st32(tS + lane_off + c * 32, pk);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(p_full);
+                // dS^T = P^T (dP^T - Delta)
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                if (!ok) break;
+                tc_fence_after();
+                if (n > 0) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(ds_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                    if (!ok) break;
+                }
+#pragma unroll
+                for (int c = 0; c < C::BM / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tDP + lane_off + c * 32, r);
+                    float dz[32];
+#pragma unroll
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 t4 = lds_f32x4(sL + 512 + (c * 32 + gq * 4) * 4);
+                        dz[4 * gq] = t4.x;
+                        dz[4 * gq + 1] = t4.y;
+                        dz[4 * gq + 2] = t4.z;
+                        dz[4 * gq + 3] = t4.w;
+                    }
+                    tmem_ld_wait(r);
+                    // 32 query columns = four 16-byte chunks of this key row in the 128B-swizzled tile.
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int col = c * 32 + gq * 8 + 2 * e;
+                            const float d0 = pr[col] * (__uint_as_float(r[gq * 8 + 2 * e]) - dz[gq * 8 + 2 * e]);
+                            const float d1 =
+                                pr[col + 1] * (__uint_as_float(r[gq * 8 + 2 * e + 1]) - dz[gq * 8 + 2 * e + 1]);
+                            w[e] = pack_bf16x2(d0, d1);
+                        }
+                        const int chunk = (c * 32 + gq * 8) >> 3;            // 0..15 across the 128 columns
+                        const int box = chunk >> 3, cib = chunk & 7;
+                        const uint32_t addr = sDS + box * C::BOX + row * 128 + ((cib ^ (row & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
+                                     "r"(w[2]), "r"(w[3])
+                                     : "memory");
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(ds_full);
+            }
+            if (!ok) break;
+            // ---- epilogue of the item: dV ----
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(acc_full, uint32_t(ki & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t dvr[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tDV + lane_off + c * 32, r);
+                tmem_ld_wait(r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) dvr[c * 32 + i] = r[i];
+            }
+            tc_fence_before();
+            mbar_arrive(acc_free);
+            if (kv < T) {
+                __nv_bfloat16* dst = p.dv + ((size_t(g.b) * T + size_t(kv)) * p.H + g.h) * D;
+#pragma unroll
+                for (int v8 = 0; v8 < D / 8; ++v8) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 0]), __uint_as_float(dvr[v8 * 8 + 1]));
+                    w.y = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 2]), __uint_as_float(dvr[v8 * 8 + 3]));
+                    w.z = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 4]), __uint_as_float(dvr[v8 * 8 + 5]));
+                    w.w = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 6]), __uint_as_float(dvr[v8 * 8 + 7]));
+                    *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
                 }
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(ds_full);
         }
     } else {
-        // ------------------------------ query-row warps: dQ drain ------------------------------
+        // ------------------------------ query-row warps: dQ drain; dK epilogue ------------------------------
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const uint32_t lane_off = uint32_t(quarter * 32) << 16;
         bool ok = true;
-        for (int n = 0; n < nsteps && ok; ++n) {
-            const long long qr = (long long)(ilo + n) * C::BM + row;
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(dq_full, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
-            if (!ok) break;
-            tc_fence_after();
-            float acc[D];
+        int n = 0, ki = 0;
+        for (;; ++ki) {
+            const int item = item_consume_warp(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                               kStatusTimeoutSoftmax, ok);
+            if (!ok || item >= p.n_items) break;
+            const BwdItem g = bwd_item(p, item);
+            for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(dq_full, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
+                if (!ok) break;
+                tc_fence_after();
+                // Stage the fp32 dQ tile over Q_n / dO_n (no MMA reads them any more): D/32 boxes of
+                // 128 rows x 128 bytes, 128-byte swizzled like the TMA box of the reduce.
+                const int s = n % C::NSTAGE;
+                const uint32_t stg = sQD + s * 2 * C::TILE;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tDP + lane_off + c * 32, r);
-                tmem_ld_wait(r);
+                for (int hh = 0; hh < D / 64; ++hh) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tDP + lane_off + hh * 64, r0);
+                    tmem_ld32(tDP + lane_off + hh * 64 + 32, r1);
+                    tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) acc[c * 32 + i] = __uint_as_float(r[i]);
-            }
-            tc_fence_before();
-            mbar_arrive(dq_free);
-            // Stage the fp32 dQ tile over Q_n / dO_n (no MMA reads them any more): D/32 boxes of
-            // 128 rows x 128 bytes, 128-byte swizzled like the TMA box of the reduce.
-            const int s = n % C::NSTAGE;
-            const uint32_t stg = sQD + s * 2 * C::TILE;
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t* rr = half ? r1 : r0;
+                        const int bx = hh * 2 + half;
 #pragma unroll
-            for (int bx = 0; bx < D / 32; ++bx) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t addr = stg + bx * C::DQ_BOX + row * 128 + ((j ^ (row & 7)) << 4);
-                    const float* a4 = acc + bx * 32 + j * 4;
-                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a4[0]), "f"(a4[1]),
-                                 "f"(a4[2]), "f"(a4[3])
-                                 : "memory");
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(dq_staged);
-            if (threadIdx.x == 128) {
-                ok = mbar_wait(dq_staged, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue);
-                if (ok) {
-                    for (int bx = 0; bx < D / 32; ++bx)
-                        tma_reduce_add_4d(&tm_dqacc, stg + bx * C::DQ_BOX, bx * 32, h, int(qr - row), b);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();   // the stage may be refilled once the reduce has read it
-                    mbar_arrive(qd_empty(s));
-                }
-            }
-            ok = __all_sync(0xffffffffu, ok);
-        }
-        if (threadIdx.x == 128) bulk_wait_group0();
-    }
-
-    // ------------------------------ epilogue: dV, dK ------------------------------
-    if (warp < 8) {
-        const bool ok = __all_sync(0xffffffffu,
-                                   mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
-        if (ok) {
-            tc_fence_after();
-            const int quarter = warp & 3;
-            const int row = quarter * 32 + lane;
-            const long long kv = k0 + row;
-            const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-            const bool is_dv = warp < 4;
-            const uint32_t src = (is_dv ? tDV : tDK) + lane_off;
-            const float mul = is_dv ? 1.f : p.scale;
-            __nv_bfloat16* dst = (is_dv ? p.dv : p.dk) + ((size_t(b) * T + size_t(kv < T ? kv : 0)) * p.H + h) * D;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(src + c * 32, r);
-                tmem_ld_wait(r);
-                if (kv < T) {
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * mul, __uint_as_float(r[v4 * 8 + 1]) * mul);
-                        w.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * mul, __uint_as_float(r[v4 * 8 + 3]) * mul);
-                        w.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * mul, __uint_as_float(r[v4 * 8 + 5]) * mul);
-                        w.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * mul, __uint_as_float(r[v4 * 8 + 7]) * mul);
-                        *reinterpret_cast<uint4*>(dst + c * 32 + v4 * 8) = w;
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t addr = stg + bx * C::DQ_BOX + row * 128 + ((j ^ (row & 7)) << 4);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(rr[j * 4]),
+                                         "r"(rr[j * 4 + 1]), "r"(rr[j * 4 + 2]), "r"(rr[j * 4 + 3])
+                                         : "memory");
+                        }
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(dq_free);
+                fence_proxy_async_smem();
+                mbar_arrive(dq_staged);
+                if (threadIdx.x == 128) {
+                    ok = mbar_wait(dq_staged, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue);
+                    if (ok) {
+                        for (int bx = 0; bx < D / 32; ++bx)
+                            tma_reduce_add_4d(&tm_dqacc, stg + bx * C::DQ_BOX, bx * 32, g.h, (g.ilo + l) * C::BM, g.b);
+                        bulk_commit_group();
+                        bulk_wait_group_read0();   // the stage may be refilled once the reduce has read it
+                        mbar_arrive(qd_empty(s));
+                    }
+                }
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            if (!ok) break;
+            // ---- epilogue of the item: scale * dK ----
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(acc_full, uint32_t(ki & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t dkr[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tDK + lane_off + c * 32, r);
+                tmem_ld_wait(r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) dkr[c * 32 + i] = r[i];
+            }
+            tc_fence_before();
+            mbar_arrive(acc_free);
+            const long long kv = g.k0 + row;
+            if (kv < T) {
+                const float sc = p.scale;
+                __nv_bfloat16* dst = p.dk + ((size_t(g.b) * T + size_t(kv)) * p.H + g.h) * D;
+#pragma unroll
+                for (int v8 = 0; v8 < D / 8; ++v8) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 0]) * sc, __uint_as_float(dkr[v8 * 8 + 1]) * sc);
+                    w.y = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 2]) * sc, __uint_as_float(dkr[v8 * 8 + 3]) * sc);
+                    w.z = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 4]) * sc, __uint_as_float(dkr[v8 * 8 + 5]) * sc);
+                    w.w = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 6]) * sc, __uint_as_float(dkr[v8 * 8 + 7]) * sc);
+                    *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
+                }
             }
         }
+        if (threadIdx.x == 128) bulk_wait_group0();
     }
 
     tc_fence_before();

@@ -7,8 +7,9 @@
 // "GPT model", architecture features).  Query i attends to keys
 // j in (i - W, i]; W >= T is full causal.
 //
-// Persistent: one CTA per SM walks work items (query block of 256 rows, b, h),
-// heaviest query blocks first.  An item is two 128-row query tiles; the CTA
+// Persistent: one CTA per SM draws work items (query block of 256 rows, b, h) from a
+// launch-wide counter; items are head-major so that concurrent CTAs share a head's K/V
+// in L2, heaviest query blocks of a head first.  An item is two 128-row query tiles; the CTA
 // walks the key/value tiles that intersect the band of either tile:
 //   warp 8      TMA producer: Q tiles of each item, then K_j, V_j into a ring
 //               of stages that runs on across items
@@ -39,8 +40,9 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = NQ * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    // kv_full, kv_empty per stage; q_full, q_empty; s_full, p_full, o_full, o_free per tile; mma_done
-    static constexpr int NUM_BAR = 2 * NSTAGE + 2 + 4 * NQ + 1;
+    // kv_full, kv_empty per stage; q_full, q_empty; s_full, p_full, o_full, o_free per tile; mma_done;
+    // item_full, item_empty per entry of the item ring
+    static constexpr int NUM_BAR = 2 * NSTAGE + 2 + 4 * NQ + 1 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
@@ -62,6 +64,7 @@ struct FwdParams {
     float scale_log2;     // softmax scale * log2(e)
     int n_qblk;           // ceil(T / 256)
     int n_items;          // n_qblk * B * H
+    int work_slot;        // index into g_work_slots for this launch
     long long wait_limit; // clock cycles before a wait gives up
 };
 
@@ -73,11 +76,13 @@ struct FwdItem {
     int jlo0, jhi0, jlo1, jhi1, jbeg, jend;
 };
 
+// Items are head-major (all query blocks of one (b, h), then the next head), so the CTAs that
+// run at the same time read the same head's K/V tiles and share them through L2; within a
+// head the heaviest (latest) query blocks come first.
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
     FwdItem it;
-    const int BH = p.B * p.H;
-    const int qblk = p.n_qblk - 1 - item / BH;   // heaviest (latest) query blocks first
-    const int bh = item % BH;
+    const int bh = item / p.n_qblk;
+    const int qblk = p.n_qblk - 1 - item % p.n_qblk;
     it.b = bh / p.H;
     it.h = bh % p.H;
     it.q0 = (long long)qblk * 256;
@@ -118,8 +123,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto o_full = [&](int t) { return bt + 8u * (2 * C::NQ + t); };
     auto o_free = [&](int t) { return bt + 8u * (3 * C::NQ + t); };
     const uint32_t mma_done = bt + 8u * (4 * C::NQ);
+    const uint32_t item_full0 = mma_done + 8u, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
+    volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
 
     const int T = p.T;
     const long long W = p.W;
@@ -139,6 +146,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(o_free(t), 128);
         }
         mbar_init(mma_done, 1);
+        for (int e = 0; e < kItemRing; ++e) {
+            mbar_init(item_full0 + 8u * e, 1);
+            mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and the 8 softmax warps
+        }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -162,7 +173,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_prefetch_desc(&tm_v);
             int it = 0, qi = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++qi) {
+            for (;; ++qi) {
+                const int item =
+                    item_produce(p.work_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                if (!ok || item >= p.n_items) break;
                 const FwdItem g = fwd_item(p, item);
                 // The Q tiles of the previous item are free once its S MMAs completed.
                 if (qi > 0) {
@@ -187,6 +201,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
             }
+            work_slot_finish(p.work_slot);
             // Drain: make sure no copy is still landing when the CTA exits.
             for (int s = 0; s < C::NSTAGE && s < it; ++s) {
                 const int fills = (it - s + C::NSTAGE - 1) / C::NSTAGE;
@@ -229,7 +244,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tc_fence_after();
                 return true;
             };
-            for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++qi) {
+            for (;; ++qi) {
+                const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                                     kStatusTimeoutMma, ok);
+                if (!ok || item >= p.n_items) break;
                 const FwdItem g = fwd_item(p, item);
                 auto act = [&](int t, int j) {
                     return t ? (g.valid1 && j >= g.jlo1 && j <= g.jhi1) : (j >= g.jlo0 && j <= g.jhi0);
@@ -314,7 +332,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float sl2 = p.scale_log2;
         int ns = 0;      // S tiles consumed so far (all items): parity of s_full / o_full
         bool ok = true;
-        for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        for (int k = 0;; ++k) {
+            const int item = item_consume_warp(k, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                               kStatusTimeoutSoftmax, ok);
+            if (!ok || item >= p.n_items) break;
             const FwdItem g = fwd_item(p, item);
             if (t == 1 && !g.valid1) continue;
             const long long qt0 = g.q0 + t * 128;    // first row of this tile

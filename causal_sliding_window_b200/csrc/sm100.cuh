@@ -91,6 +91,70 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // ---------------------------------------------------------------------------
+// Dynamic work distribution for persistent kernels.
+//
+// A launch of a persistent kernel draws item indices 0, 1, 2, ... from one counter in
+// g_work_slots (atomicAdd), so whichever CTA is free takes the next item: items keep the
+// kernel's order (head-major, heaviest first) and the load balances itself.  Inside a CTA
+// the producer thread draws the index and hands it to the other roles through a small
+// shared-memory ring (item_full / item_empty mbarriers).  When a CTA stops drawing it
+// counts itself done; the last CTA of the launch zeroes the slot for a later launch.  The
+// host gives concurrent launches different slots (kWorkSlots of them, round robin).
+// ---------------------------------------------------------------------------
+constexpr int kWorkSlots = 64;
+constexpr int kItemRing = 4;
+struct WorkSlot {
+    int next;
+    int done;
+};
+__device__ WorkSlot g_work_slots[kWorkSlots];
+
+// Producer side: draw the k-th item of this CTA and publish it in ring entry k % kItemRing.
+__device__ __forceinline__ int item_produce(int slot, int k, volatile int* ring, uint32_t full0, uint32_t empty0,
+                                            volatile int* abort_flag, long long limit, bool& ok) {
+    const int e = k % kItemRing;
+    if (k >= kItemRing)
+        ok = ok && mbar_wait(empty0 + 8u * e, uint32_t(((k / kItemRing) - 1) & 1), abort_flag, limit,
+                             kStatusTimeoutProducer);
+    const int item = ok ? atomicAdd(&g_work_slots[slot].next, 1) : 0x7fffffff;
+    ring[e] = item;
+    mbar_arrive(full0 + 8u * e);
+    return item;
+}
+
+// Consumer side (every lane of a consuming warp calls it; lane 0 releases the entry).
+__device__ __forceinline__ int item_consume_warp(int k, volatile int* ring, uint32_t full0, uint32_t empty0,
+                                                 volatile int* abort_flag, long long limit, int code, bool& ok) {
+    const int e = k % kItemRing;
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(full0 + 8u * e, uint32_t((k / kItemRing) & 1), abort_flag,
+                                                 limit, code));
+    const int item = ok ? ring[e] : 0x7fffffff;
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(empty0 + 8u * e);
+    return item;
+}
+
+// Consumer side for a single thread (one arrival).
+__device__ __forceinline__ int item_consume_thread(int k, volatile int* ring, uint32_t full0, uint32_t empty0,
+                                                   volatile int* abort_flag, long long limit, int code, bool& ok) {
+    const int e = k % kItemRing;
+    ok = ok && mbar_wait(full0 + 8u * e, uint32_t((k / kItemRing) & 1), abort_flag, limit, code);
+    const int item = ok ? ring[e] : 0x7fffffff;
+    mbar_arrive(empty0 + 8u * e);
+    return item;
+}
+
+// Called once per CTA by the producer thread after its last draw.
+__device__ __forceinline__ void work_slot_finish(int slot) {
+    __threadfence();
+    if (atomicAdd(&g_work_slots[slot].done, 1) == int(gridDim.x) - 1) {
+        g_work_slots[slot].next = 0;
+        g_work_slots[slot].done = 0;
+        __threadfence();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // TMA: 4-D tiled load global -> shared, completion counted on an mbarrier.
 // Coordinates are innermost first.  (No cluster multicast anywhere.)
 // ---------------------------------------------------------------------------
@@ -250,6 +314,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// 2^x on the FMA/ALU pipes, to take load off the MUFU unit (which executes ex2.approx).
+// Range reduction x = n + f with n = round(x), |f| <= 1/2 (Cody and Waite's additive
+// reduction; n is read from the mantissa after adding 1.5 * 2^23), then
+// 2^f ~= c0 + c1 f + c2 f^2 + c3 f^3 and 2^n is added to the exponent field.  The
+// coefficients minimise the maximum relative error of 2^f on [-1/2, 1/2] (Remez
+// exchange): max relative error 7.5e-5, well below half a bf16 ulp (2^-9), which is
+// the precision the probabilities are rounded to.  x is clamped below at -125, so
+// masked (-inf) entries give 2^-125 (about 2e-38) rather than 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+    constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+    x = fmaxf(x, -125.0f);
+    const float t = x + kRound;
+    const float f = x - (t - kRound);
+    const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Pack two fp32 into bf16x2 with round-to-nearest-even; `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -77,6 +78,13 @@ bool ensure_smem(const void* func, int bytes) {
     if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
     done.insert({dev, func});
     return true;
+}
+
+// Work-counter slot for the next persistent launch (round robin over kWorkSlots, so that
+// up to kWorkSlots launches may be in flight at once on different streams).
+int next_work_slot() {
+    static std::atomic<unsigned> ctr{0};
+    return int(ctr.fetch_add(1, std::memory_order_relaxed) % unsigned(kWorkSlots));
 }
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -185,6 +193,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_qblk = n_qblk;
     p.n_items = int(n_items);
+    p.work_slot = next_work_slot();
     p.wait_limit = kDefaultWaitLimit;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (D == 128) {
@@ -217,8 +226,9 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_bwd_workspace_bytes(B, T, H, D)) return ATTN_ERR_WORKSPACE;
     const int n_kblk = (T + 127) / 128;
-    const long long grid = (long long)n_kblk * B * H;
-    if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long n_items = (long long)n_kblk * B * H;
+    if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
     CUtensorMap mq, mk, mv, mdo;
     if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, H, D) ||
         !make_bthd_map(&mv, v, B, T, H, D) || !make_bthd_map(&mdo, dout, B, T, H, D))
@@ -256,6 +266,8 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_kblk = n_kblk;
+    p.n_items = int(n_items);
+    p.work_slot = next_work_slot();
     p.Tp = Tp;
     p.wait_limit = kDefaultWaitLimit;
     if (D == 128) {

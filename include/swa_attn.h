@@ -30,6 +30,9 @@
  *    (or ATTN_ERR_UNSUPPORTED for an unsupported D) before anything is
  *    launched.  A failed launch returns ATTN_ERR_LAUNCH.
  *  - Outputs are written with round-to-nearest-even to bf16; lse is fp32.
+ *  - attn_fwd and attn_bwd run persistent kernels that draw work from one of 64
+ *    counters inside the library (round robin per call); at most 64 such calls may
+ *    be executing on the device at the same time (on different streams).
  *  - Device-side waits are bounded.  If one gives up (a condition that
  *    correct use never produces), the kernel stops early and records a flag
  *    that attn_device_status() reports as ATTN_ERR_DEVICE_TIMEOUT.
