@@ -399,23 +399,29 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
+                // Both halves of the row (64 columns each) are requested before one wait.
                 float pr[C::BM];
 #pragma unroll
-                for (int c = 0; c < C::BM / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + lane_off + c * 32, r);
-                    float lz[32];
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tS + lane_off + hh * 64, r0);
+                    tmem_ld32(tS + lane_off + hh * 64 + 32, r1);
+                    float lz[64];
 #pragma unroll
-                    for (int gq = 0; gq < 8; ++gq) {
-                        const float4 t4 = lds_f32x4(sL + (c * 32 + gq * 4) * 4);
+                    for (int gq = 0; gq < 16; ++gq) {
+                        const float4 t4 = lds_f32x4(sL + (hh * 64 + gq * 4) * 4);
                         lz[4 * gq] = t4.x;
                         lz[4 * gq + 1] = t4.y;
                         lz[4 * gq + 2] = t4.z;
                         lz[4 * gq + 3] = t4.w;
                     }
-                    tmem_ld_wait(r);
+                    tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pr[c * 32 + i] = ex2_approx(fmaf(__uint_as_float(r[i]), sl2, -lz[i]));
+                    for (int i = 0; i < 32; ++i) {
+                        pr[hh * 64 + i] = ex2_approx(fmaf(__uint_as_float(r0[i]), sl2, -lz[i]));
+                        pr[hh * 64 + 32 + i] = ex2_approx(fmaf(__uint_as_float(r1[i]), sl2, -lz[32 + i]));
+                    }
                 }
                 // Tiles that cut the diagonal, the window's far edge or T: keep columns clo..chi of this
                 // key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.

@@ -348,14 +348,26 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 mbar_wait(s_full(t), uint32_t(ns & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
+                // All 128 columns are requested before the single wait, so the TMEM load
+                // latency is paid once per tile.
                 float s[C::BN];
+                {
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld32(tS, r0);
+                    tmem_ld32(tS + 32, r1);
+                    tmem_ld32(tS + 64, r2);
+                    tmem_ld32(tS + 96, r3);
+                    tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
+                    tmem_ld_wait(r2);
+                    tmem_ld_wait(r3);
 #pragma unroll
-                for (int c = 0; c < C::BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + c * 32, r);
-                    tmem_ld_wait(r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        s[i] = __uint_as_float(r0[i]);
+                        s[32 + i] = __uint_as_float(r1[i]);
+                        s[64 + i] = __uint_as_float(r2[i]);
+                        s[96 + i] = __uint_as_float(r3[i]);
+                    }
                 }
                 // Tiles that cut the diagonal or the window's left edge: keep columns clo..chi of this
                 // row (keys k0+c with q-W < k0+c <= q).  The test is uniform across the CTA.
@@ -367,9 +379,14 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int c = 0; c < C::BN; ++c) s[c] = (c >= clo && c <= chi) ? s[c] : -INFINITY;
                 }
-                float mx = s[0];
+                // Row max and row sum over 8 independent partials (short dependency chains).
+                float mp[8];
 #pragma unroll
-                for (int c = 1; c < C::BN; ++c) mx = fmaxf(mx, s[c]);
+                for (int u = 0; u < 8; ++u) mp[u] = s[u];
+#pragma unroll
+                for (int c = 8; c < C::BN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+                const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
                 const float m_tile = mx * sl2;
                 const float m_new = fmaxf(m_run, m_tile);
                 const bool need = m_new > m_run + 8.0f;
@@ -377,7 +394,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float m_use = warp_need ? m_new : m_run;
                 const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
                 const float alpha = (m_use == -INFINITY) ? 1.f : ex2_approx(m_run - m_use);
-                float rowsum = 0.f;
+                float sp[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) sp[u] = 0.f;
 #pragma unroll
                 for (int c = 0; c < C::BN / 64; ++c) {
                     uint32_t pk[32];
@@ -385,11 +404,13 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int i = 0; i < 32; ++i) {
                         const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_sub));
                         const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
-                        rowsum += p0 + p1;
+                        sp[(2 * i) & 7] += p0;
+                        sp[(2 * i + 1) & 7] += p1;
                         pk[i] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(tS + c * 32, pk);
                 }
+                const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
                 l_run = l_run * alpha + rowsum;
                 tmem_st_wait();
                 if (warp_need && nloc > 0) {

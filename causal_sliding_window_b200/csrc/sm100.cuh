@@ -314,25 +314,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// 2^x on the FMA/ALU pipes, to take load off the MUFU unit (which executes ex2.approx).
-// Range reduction x = n + f with n = round(x), |f| <= 1/2 (Cody and Waite's additive
-// reduction; n is read from the mantissa after adding 1.5 * 2^23), then
-// 2^f ~= c0 + c1 f + c2 f^2 + c3 f^3 and 2^n is added to the exponent field.  The
-// coefficients minimise the maximum relative error of 2^f on [-1/2, 1/2] (Remez
-// exchange): max relative error 7.5e-5, well below half a bf16 ulp (2^-9), which is
-// the precision the probabilities are rounded to.  x is clamped below at -125, so
-// masked (-inf) entries give 2^-125 (about 2e-38) rather than 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-    constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
-    constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    x = fmaxf(x, -125.0f);
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Pack two fp32 into bf16x2 with round-to-nearest-even; `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
