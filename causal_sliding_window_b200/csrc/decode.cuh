@@ -24,8 +24,8 @@
 
 namespace swa {
 
-constexpr int kDecodeChunk = 64;   // cache slots per CTA
-constexpr int kDecodeUnroll = 8;   // slots in flight per thread
+constexpr int kDecodeChunk = 128;  // cache slots per CTA
+constexpr int kDecodeUnroll = 4;   // slots per batch (two batches in flight per thread)
 
 struct DecParams {
     const __nv_bfloat16* q;        // [B,H,D]
@@ -93,14 +93,17 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
     const __nv_bfloat16* kb = p.kc + size_t(b) * p.cap * row_elems + size_t(h) * D + c * 8;
     const __nv_bfloat16* vb = p.vc + size_t(b) * p.cap * row_elems + size_t(h) * D + c * 8;
 
-    for (int pos = start; pos < end; pos += kDecodeUnroll) {
-        uint4 ku[kDecodeUnroll], vu[kDecodeUnroll];
+    // Two batches of kDecodeUnroll slots are in flight: the next batch's loads are issued
+    // before the current batch is consumed.
+    auto load = [&](int pos, uint4 (&ku)[kDecodeUnroll], uint4 (&vu)[kDecodeUnroll]) {
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) {
             const bool in = live && (pos + u < end);
             ku[u] = in ? __ldcs(reinterpret_cast<const uint4*>(kb + size_t(pos + u) * row_elems)) : make_uint4(0, 0, 0, 0);
             vu[u] = in ? __ldcs(reinterpret_cast<const uint4*>(vb + size_t(pos + u) * row_elems)) : make_uint4(0, 0, 0, 0);
         }
+    };
+    auto consume = [&](int pos, const uint4 (&ku)[kDecodeUnroll], const uint4 (&vu)[kDecodeUnroll]) {
         float s[kDecodeUnroll];
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) {
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
         float mx = m;
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) mx = fmaxf(mx, s[u]);
-        const float alpha = ex2_approx(m - mx);   // m = -inf on the first pass: alpha = 0
+        const float alpha = ex2_approx(m - mx);   // m = -inf on the first batch: alpha = 0
         l *= alpha;
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] *= alpha;
@@ -130,6 +133,14 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
             for (int i = 0; i < 8; ++i) acc[i] = fmaf(pu, vf[i], acc[i]);
         }
         m = mx;
+    };
+    uint4 ka[kDecodeUnroll], va[kDecodeUnroll], kn[kDecodeUnroll], vn[kDecodeUnroll];
+    if (start < end) load(start, ka, va);
+    for (int pos = start; pos < end; pos += 2 * kDecodeUnroll) {   // CTA-uniform trip count
+        if (pos + kDecodeUnroll < end) load(pos + kDecodeUnroll, kn, vn);
+        consume(pos, ka, va);
+        if (pos + 2 * kDecodeUnroll < end) load(pos + 2 * kDecodeUnroll, ka, va);
+        if (pos + kDecodeUnroll < end) consume(pos + kDecodeUnroll, kn, vn);
     }
 
     // ---- partial of this chunk ----
@@ -158,28 +169,46 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
     const int n = L - lo;
     const int used = (n + kDecodeChunk - 1) / kDecodeChunk;
     if (live) {
+        // Partials are read in batches so their load latencies overlap.
+        const size_t pbase = (size_t(b) * p.nsplit_max) * H + h;   // partial (split sp) at pbase + sp * H
         float M = -INFINITY;
-        for (int sp = 0; sp < used; ++sp) {
-            const size_t q = (size_t(b) * p.nsplit_max + sp) * H + h;
-            M = fmaxf(M, __ldcg(p.part_ml + 2 * q));
+        for (int sp0 = 0; sp0 < used; sp0 += 8) {
+            float mv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                mv[u] = (sp0 + u < used) ? __ldcg(p.part_ml + 2 * (pbase + size_t(sp0 + u) * H)) : -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) M = fmaxf(M, mv[u]);
         }
         float lsum = 0.f, o8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) o8[i] = 0.f;
-        for (int sp = 0; sp < used; ++sp) {
-            const size_t q = (size_t(b) * p.nsplit_max + sp) * H + h;
-            const float w = ex2_approx(__ldcg(p.part_ml + 2 * q) - M);
-            lsum = fmaf(w, __ldcg(p.part_ml + 2 * q + 1), lsum);
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(p.part_o + q * D + c * 8));
-            const float4 bb = __ldcg(reinterpret_cast<const float4*>(p.part_o + q * D + c * 8) + 1);
-            o8[0] = fmaf(w, a.x, o8[0]);
-            o8[1] = fmaf(w, a.y, o8[1]);
-            o8[2] = fmaf(w, a.z, o8[2]);
-            o8[3] = fmaf(w, a.w, o8[3]);
-            o8[4] = fmaf(w, bb.x, o8[4]);
-            o8[5] = fmaf(w, bb.y, o8[5]);
-            o8[6] = fmaf(w, bb.z, o8[6]);
-            o8[7] = fmaf(w, bb.w, o8[7]);
+        for (int sp0 = 0; sp0 < used; sp0 += 4) {
+            float ml[4][2];
+            float4 oa[4], ob[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const bool in = sp0 + u < used;
+                const size_t q = pbase + size_t(sp0 + u) * H;
+                ml[u][0] = in ? __ldcg(p.part_ml + 2 * q) : -INFINITY;
+                ml[u][1] = in ? __ldcg(p.part_ml + 2 * q + 1) : 0.f;
+                oa[u] = in ? __ldcg(reinterpret_cast<const float4*>(p.part_o + q * D + c * 8)) : make_float4(0, 0, 0, 0);
+                ob[u] = in ? __ldcg(reinterpret_cast<const float4*>(p.part_o + q * D + c * 8) + 1)
+                           : make_float4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float w = ex2_approx(ml[u][0] - M);   // 0 for empty partials (m = -inf)
+                lsum = fmaf(w, ml[u][1], lsum);
+                o8[0] = fmaf(w, oa[u].x, o8[0]);
+                o8[1] = fmaf(w, oa[u].y, o8[1]);
+                o8[2] = fmaf(w, oa[u].z, o8[2]);
+                o8[3] = fmaf(w, oa[u].w, o8[3]);
+                o8[4] = fmaf(w, ob[u].x, o8[4]);
+                o8[5] = fmaf(w, ob[u].y, o8[5]);
+                o8[6] = fmaf(w, ob[u].z, o8[6]);
+                o8[7] = fmaf(w, ob[u].w, o8[7]);
+            }
         }
         const float inv = used > 0 ? 1.f / lsum : 0.f;
         uint4 w;

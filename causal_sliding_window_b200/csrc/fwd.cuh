@@ -36,13 +36,14 @@ struct FwdCfg {
     static constexpr int TILE = 128 * D * 2;        // bytes of a 128 x D bf16 tile
     static constexpr int BOX = 128 * 64 * 2;        // one TMA box: 128 rows x 64 columns
     static constexpr int NBOX = D / 64;
+    static constexpr int NQBUF = 1;                 // Q buffers (2: the next item's Q loads a whole item ahead)
     static constexpr int NSTAGE = D == 128 ? 5 : 8; // K/V ring (a stage holds one K or one V tile)
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = NQ * TILE;
+    static constexpr int OFF_KV = NQBUF * NQ * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    // kv_full, kv_empty per stage; q_full, q_empty; s_full, p_full, o_full, o_free per tile; mma_done;
-    // item_full, item_empty per entry of the item ring
-    static constexpr int NUM_BAR = 2 * NSTAGE + 2 + 4 * NQ + 1 + 2 * kItemRing;
+    // kv_full, kv_empty per stage; q_full, q_empty per Q buffer; s_full, p_full, o_full, o_free per
+    // tile; mma_done; item_full, item_empty per entry of the item ring
+    static constexpr int NUM_BAR = 2 * NSTAGE + 2 * NQBUF + 4 * NQ + 1 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
@@ -115,9 +116,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t bar0 = base + C::OFF_BAR;
     auto kv_full = [&](int s) { return bar0 + 8u * s; };
     auto kv_empty = [&](int s) { return bar0 + 8u * (C::NSTAGE + s); };
-    const uint32_t q_full = bar0 + 8u * (2 * C::NSTAGE);
-    const uint32_t q_empty = q_full + 8u;
-    const uint32_t bt = q_full + 16u;   // per-tile barriers start here
+    auto q_full = [&](int qb) { return bar0 + 8u * (2 * C::NSTAGE + qb); };
+    auto q_empty = [&](int qb) { return bar0 + 8u * (2 * C::NSTAGE + C::NQBUF + qb); };
+    const uint32_t bt = bar0 + 8u * (2 * C::NSTAGE + 2 * C::NQBUF);   // per-tile barriers start here
     auto s_full = [&](int t) { return bt + 8u * t; };
     auto p_full = [&](int t) { return bt + 8u * (C::NQ + t); };
     auto o_full = [&](int t) { return bt + 8u * (2 * C::NQ + t); };
@@ -137,8 +138,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(kv_full(s), 1);
             mbar_init(kv_empty(s), 1);
         }
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        for (int qb = 0; qb < C::NQBUF; ++qb) {
+            mbar_init(q_full(qb), 1);
+            mbar_init(q_empty(qb), 1);
+        }
         for (int t = 0; t < C::NQ; ++t) {
             mbar_init(s_full(t), 1);
             mbar_init(p_full(t), 128);
@@ -178,16 +181,18 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     item_produce(p.work_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
                 const FwdItem g = fwd_item(p, item);
-                // The Q tiles of the previous item are free once its S MMAs completed.
-                if (qi > 0) {
-                    ok = mbar_wait(q_empty, uint32_t((qi - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                // A Q buffer is free once the S MMAs of the item that used it completed.
+                const int qb = qi % C::NQBUF;
+                if (qi >= C::NQBUF) {
+                    ok = mbar_wait(q_empty(qb), uint32_t(((qi / C::NQBUF) - 1) & 1), abort_flag, p.wait_limit,
+                                   kStatusTimeoutProducer);
                     if (!ok) break;
                 }
-                mbar_arrive_expect_tx(q_full, (g.valid1 ? 2 : 1) * C::TILE);
+                mbar_arrive_expect_tx(q_full(qb), (g.valid1 ? 2 : 1) * C::TILE);
                 for (int t = 0; t < (g.valid1 ? 2 : 1); ++t)
                     for (int x = 0; x < C::NBOX; ++x)
-                        tma_load_4d(sQ + t * C::TILE + x * C::BOX, &tm_q, q_full, x * 64, g.h, int(g.q0) + t * 128,
-                                    g.b);
+                        tma_load_4d(sQ + (qb * C::NQ + t) * C::TILE + x * C::BOX, &tm_q, q_full(qb), x * 64, g.h,
+                                    int(g.q0) + t * 128, g.b);
                 for (int j = g.jbeg; j <= g.jend && ok; ++j) {
                     for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
                         const int s = it % C::NSTAGE;
@@ -207,7 +212,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int fills = (it - s + C::NSTAGE - 1) / C::NSTAGE;
                 mbar_wait(kv_full(s), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
             }
-            if (qi > 0) mbar_wait(q_full, uint32_t((qi - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            for (int qb = 0; qb < C::NQBUF && qb < qi; ++qb) {
+                const int fills = (qi - qb + C::NQBUF - 1) / C::NQBUF;
+                mbar_wait(q_full(qb), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            }
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
@@ -216,8 +224,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             int it = 0, qi = 0;
             int npv0 = 0, npv1 = 0;   // PV MMAs issued per tile (all items)
             int nep0 = 0, nep1 = 0;   // items processed per tile (= epilogues owed)
+            int qbuf = 0;   // Q buffer of the current item
             auto issue_s = [&](int t, int stage) {
-                const uint32_t qa = sQ + t * C::TILE, ka = sKV + stage * C::TILE;
+                const uint32_t qa = sQ + (qbuf * C::NQ + t) * C::TILE, ka = sKV + stage * C::TILE;
                 const uint32_t d = t ? tS1 : tS0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -252,7 +261,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 auto act = [&](int t, int j) {
                     return t ? (g.valid1 && j >= g.jlo1 && j <= g.jhi1) : (j >= g.jlo0 && j <= g.jhi0);
                 };
-                ok = mbar_wait(q_full, uint32_t(qi & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+                qbuf = qi % C::NQBUF;
+                ok = mbar_wait(q_full(qbuf), uint32_t((qi / C::NQBUF) & 1), abort_flag, p.wait_limit,
+                               kStatusTimeoutMma);
                 if (!ok) break;
                 bool first0 = true, first1 = true;
                 int sk = it % C::NSTAGE;
@@ -315,7 +326,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tc_commit(kv_empty(sv));
                     sk = sk_next;
                 }
-                tc_commit(q_empty);   // every S MMA of this item has been issued
+                tc_commit(q_empty(qbuf));   // every S MMA of this item has been issued
                 ++nep0;
                 if (g.valid1) ++nep1;
             }
