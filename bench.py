@@ -366,8 +366,8 @@ def main():
     assert status == 0, "device wait timed out during the timed region"
     t_fwd = sum(e["f0"][i].elapsed_time(e["f1"][i]) for e in evs for i in range(len(windows)))
     t_pre = sum(e["f1"][i].elapsed_time(e["bp"][i]) for e in evs for i in range(len(windows)))
-    t_bmain = sum(e["bp"][i].elapsed_time(e["bm"][i]) for e in evs for i in range(len(windows)))
-    t_conv = sum(e["bm"][i].elapsed_time(e["b1"][i]) for e in evs for i in range(len(windows)))
+    t_dkdv = sum(e["bp"][i].elapsed_time(e["bm"][i]) for e in evs for i in range(len(windows)))
+    t_dqk = sum(e["bm"][i].elapsed_time(e["b1"][i]) for e in evs for i in range(len(windows)))
     t_dec = sum(e["d0"][i].elapsed_time(e["d1"][i]) for e in evs for i in range(len(dwins)))
     ms_max = max_over_ranks(ms, dev)
     finite = bool(torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all()
@@ -411,11 +411,14 @@ def main():
         K = args.steps
         value = weak_scaling_value(step_flops, world, K, ms_max)
         fwd_tf = step_fwd_flops * K / (t_fwd * 1e-3) / 1e12
-        bmain_tf = step_bwd_flops * K / (t_bmain * 1e-3) / 1e12
-        bwd_tf = step_bwd_flops * K / ((t_pre + t_bmain + t_conv) * 1e-3) / 1e12
+        # Per-kernel algorithmic work: the dK/dV kernel needs S, dP, dV, dK (8*D flops per in-band
+        # pair), the dQ kernel S, dP, dQ (6*D); the backward as a whole counts 10*D.
+        dkdv_tf = step_bwd_flops * 0.8 * K / (t_dkdv * 1e-3) / 1e12
+        dqk_tf = step_bwd_flops * 0.6 * K / (t_dqk * 1e-3) / 1e12
+        bwd_tf = step_bwd_flops * K / ((t_pre + t_dkdv + t_dqk) * 1e-3) / 1e12
         dec_gbs = step_dec_bytes * K / (t_dec * 1e-3) / 1e9
-        parts = {"fwd_ms": t_fwd / K, "bwd_pre_ms": t_pre / K, "bwd_main_ms": t_bmain / K,
-                 "bwd_dq_convert_ms": t_conv / K, "decode_ms": t_dec / K}
+        parts = {"fwd_ms": t_fwd / K, "bwd_pre_ms": t_pre / K, "bwd_dkdv_ms": t_dkdv / K,
+                 "bwd_dq_ms": t_dqk / K, "decode_ms": t_dec / K}
         dominant = max(parts, key=parts.get)
         peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -425,8 +428,11 @@ def main():
         elif dominant == "decode_ms":
             roof = {"kernel": "swa_decode_kernel<128>", "bound": "hbm", "achieved": dec_gbs, "peak": peak_h,
                     "unit": "GB/s"}
+        elif dominant == "bwd_dq_ms":
+            roof = {"kernel": "swa_bwd_dq_kernel<128>", "bound": "tensor", "achieved": dqk_tf, "peak": peak_t,
+                    "unit": "TFLOP/s"}
         else:
-            roof = {"kernel": "swa_bwd_kernel<128>", "bound": "tensor", "achieved": bmain_tf, "peak": peak_t,
+            roof = {"kernel": "swa_bwd_dkdv_kernel<128>", "bound": "tensor", "achieved": dkdv_tf, "peak": peak_t,
                     "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["traffic"] = None
@@ -449,7 +455,7 @@ def main():
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "parts": {
                 **{k2: round(v2, 4) for k2, v2 in parts.items()},
-                "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "bwd_main_tflops": bmain_tf, "decode_gbs": dec_gbs,
+                "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "bwd_dkdv_tflops": dkdv_tf, "bwd_dq_tflops": dqk_tf, "decode_gbs": dec_gbs,
                 "fwd_frac_spec_2250": fwd_tf / SPEC_BF16_TFLOPS, "bwd_frac_spec_2250": bwd_tf / SPEC_BF16_TFLOPS,
                 "decode_frac_spec_8000": dec_gbs / SPEC_HBM_GBS,
                 "fwd_frac_measured": fwd_tf / peak_t, "bwd_frac_measured": bwd_tf / peak_t,

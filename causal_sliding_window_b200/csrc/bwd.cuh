@@ -6,109 +6,52 @@
 //   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - Delta),
 //   dK = scale * dS^T Q,   dQ = scale * dS K.
 //
-// Three launches:
-//   swa_bwd_pre_kernel      Delta and lse*log2(e) as fp32 rows [B*H, Tp] padded to
-//                           Tp = 128*ceil(T/128) (padding: Delta 0, lse +inf), and a
-//                           zeroed fp32 dQ accumulator
-//   swa_bwd_kernel          persistent (one CTA per SM) drawing items = 128-row key/value
-//                           tile of one (b, h) from a launch-wide counter (head-major,
-//                           lowest key tiles first), walking the
-//                           query tiles of each item's band; P^T is recomputed from lse,
-//                           dK and dV stay in TMEM, and each dQ partial tile is
-//                           staged in shared memory (in the Q/dO stage it was
-//                           computed from) and added to the fp32 accumulator by a
-//                           TMA tensor reduce-add
-//   swa_bwd_dq_kernel       dQ = bf16(scale * accumulator)
+// Three launches, no atomics and no fp32 gradient accumulator in memory:
+//   swa_bwd_pre_kernel    Delta and lse*log2(e) as fp32 rows [B*H, Tp], Tp = 128*ceil(T/128)
+//                         (padding: Delta 0, lse +inf), so every 128-query slice is one
+//                         aligned 512-byte bulk copy
+//   swa_bwd_dkdv_kernel   key-stationary: an item is a 128-row key/value tile of one (b, h);
+//                         it walks the query tiles of its band, recomputes P^T from lse and
+//                         keeps dV, dK in TMEM (4 MMAs per step)
+//   swa_bwd_dq_kernel     query-stationary: an item is a 128-row query tile; it walks the key
+//                         tiles of its band, recomputes P and dS and keeps dQ in TMEM
+//                         (3 MMAs per step)
+// Splitting dQ off costs recomputing S and dP (2 extra MMAs per tile pair) and saves
+// the fp32 dQ accumulator round trip: a TMA reduce-add of one 64 KB fp32 dQ partial per
+// tile pair is bound by L2 atomics, and it pins the shared memory it reads from.
 //
-// swa_bwd_kernel roles:
-//   warp 8       TMA producer: K, V once; Q_i and dO_i per query tile into a ring
-//   warp 9       MMA issuer: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO (P^T from TMEM),
-//                dK += dS^T Q, dQ_i = dS K
-//   warps 0..3   thread = key row: P^T = exp2(S^T*scale*log2e - lse*log2e) with the
-//                band mask, dS^T = P^T (dP^T - Delta) to shared memory
-//   warps 4..7   thread = query row: drain dQ_i from TMEM into shared memory; one
-//                thread issues the TMA reduce-add and, once it has read the tile,
-//                hands the stage back to the producer
-//   warps 0..7   per-item epilogue: dV (warps 0..3) and scale*dK (warps 4..7) to bf16,
-//                overlapping the next item's first steps (acc_full / acc_free barriers)
+// Both main kernels are persistent (one CTA per SM) and draw head-major items from a
+// launch-wide counter (sm100.cuh), so CTAs that run at the same time share a head's
+// tiles through L2.  Roles (320 threads):
+//   warp 8       TMA producer
+//   warp 9       MMA issuer (one thread)
+//   warps 0..7   two warpgroups on the same 128 TMEM lanes (one row per lane): warps 0..3
+//                take columns 0..63 of the 128-column score tiles, warps 4..7 columns 64..127.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace swa {
 
-template <int D>
-struct BwdCfg {
-    static constexpr int BN = 128;                 // key rows per CTA (MMA M for S^T, dP^T, dV, dK)
-    static constexpr int BM = 128;                 // query rows per step
-    static constexpr int TILE = 128 * D * 2;
-    static constexpr int BOX = 128 * 64 * 2;
-    static constexpr int NBOX = D / 64;
-    static constexpr int NSTAGE = 2;               // Q_i / dO_i ring
-    static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = TILE;
-    static constexpr int OFF_QD = 2 * TILE;        // stage s: Q at OFF_QD + s*2*TILE, dO after it
-    static constexpr int OFF_DS = OFF_QD + NSTAGE * 2 * TILE;   // dS^T: 128 key rows x 128 query cols bf16
-    static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;      // per stage: 128 floats lse*log2e, 128 Delta
-    static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
-    // kv_full, kv_empty, qd_full x2, qd_empty x2, s_full, dp_full, p_full, ds_full, dv_done, dq_full,
-    // dq_free, ds_free, mma_done, dq_staged, acc_full, acc_free; item_full, item_empty per ring entry
-    static constexpr int NUM_BAR = 2 + 2 * NSTAGE + 12 + 2 * kItemRing;
-    static constexpr int DQ_BOX = 128 * 32 * 4;    // one reduce box: 128 query rows x 32 fp32 columns
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
-    static constexpr int SMEM_USED = OFF_MISC + 64;
-    // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
-    // the kernel checks at run time that the aligned layout fits what it was given.
-    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
-    static constexpr int THREADS = 320;
-    static constexpr uint32_t TMEM_COLS = 512;     // S^T | dP^T (then dQ) | dV | dK
-    static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BM, 0, 0);       // K-major A, K-major B
-    static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);      // K-major A, MN-major B
-    static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 1, 1);       // MN-major A, MN-major B
-    static_assert(SMEM_USED <= 232448, "shared memory");
-};
-
 struct BwdParams {
     const float* lse2;    // [B*H, Tp] lse * log2(e), +inf past T
     const float* delta;   // [B*H, Tp], 0 past T
-    float* dq_acc;        // [B,T,H,D]
+    __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     int B, T, H;
     long long W;
     float scale;
     float scale_log2;
-    int n_kblk;
-    int n_items;          // n_kblk * B * H
+    int n_blk;            // ceil(T / 128)
+    int n_items;          // n_blk * B * H
     int work_slot;        // index into g_work_slots for this launch
     int Tp;               // T rounded up to 128
     long long wait_limit;
 };
 
-// Geometry of one work item: key block kblk of head (b, h).  Items are head-major (all key
-// blocks of one head, lowest first, then the next head), so the CTAs that run at the same
-// time read the same head's Q / dO tiles and share them through L2.
-struct BwdItem {
-    int b, h, bh;
-    long long k0;         // first key row
-    int ilo, nsteps;      // first query tile and number of query tiles in the band
-};
-
-__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int item) {
-    BwdItem it;
-    const int kblk = item % p.n_kblk;
-    it.bh = item / p.n_kblk;
-    it.b = it.bh / p.H;
-    it.h = it.bh % p.H;
-    it.k0 = (long long)kblk * 128;
-    it.ilo = int(it.k0 / 128);
-    const int ihi = int(imin_ll(p.T - 1, it.k0 + 127 + p.W - 1) / 128);
-    it.nsteps = ihi - it.ilo + 1;
-    return it;
-}
-
 // ---------------------------------------------------------------------------
-// Delta_i = sum_d dO_id * O_id and zeroing of the dQ accumulator.
+// Delta_i = sum_d dO_id * O_id and lse * log2(e), as padded fp32 rows.
 // One thread per 8 consecutive elements (16 bytes) of a [B,T,H,D] row.
 // ---------------------------------------------------------------------------
 template <int D>
@@ -116,12 +59,11 @@ __global__ void __launch_bounds__(256) swa_bwd_pre_kernel(const __nv_bfloat16* _
                                                           const __nv_bfloat16* __restrict__ dout,
                                                           const float* __restrict__ lse,
                                                           float* __restrict__ lse2, float* __restrict__ delta,
-                                                          float* __restrict__ dq_acc, int B, int T, int H, int Tp) {
+                                                          int B, int T, int H, int Tp) {
     constexpr int LPR = D / 8;   // lanes per row
     const long long nrows = (long long)B * T * H;
     const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long stride = (long long)gridDim.x * blockDim.x;
-    // lse * log2(e) into the padded rows; padding columns get +inf (and Delta 0).
     for (long long e = tid; e < (long long)B * H * Tp; e += stride) {
         const long long bh = e / Tp, t = e % Tp;
         if (t < T) {
@@ -148,9 +90,6 @@ __global__ void __launch_bounds__(256) swa_bwd_pre_kernel(const __nv_bfloat16* _
                 acc = fmaf(fa.x, fg.x, acc);
                 acc = fmaf(fa.y, fg.y, acc);
             }
-            float4* z = reinterpret_cast<float4*>(dq_acc + row * D + c * 8);
-            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -163,29 +102,88 @@ __global__ void __launch_bounds__(256) swa_bwd_pre_kernel(const __nv_bfloat16* _
     }
 }
 
-// dq = bf16(scale * dq_acc), 8 elements per thread.
-__global__ void __launch_bounds__(256) swa_bwd_dq_kernel(const float* __restrict__ dq_acc,
-                                                         __nv_bfloat16* __restrict__ dq, long long n8,
-                                                         float scale) {
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8; e += stride) {
-        const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * e];
-        const float4 b = reinterpret_cast<const float4*>(dq_acc)[2 * e + 1];
+// Store 32 fp32 values (bit patterns) of one row as bf16, times `mul`, 16 bytes at a time.
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint32_t (&r)[32], float mul) {
+#pragma unroll
+    for (int v4 = 0; v4 < 4; ++v4) {
         uint4 w;
-        w.x = pack_bf16x2(a.x * scale, a.y * scale);
-        w.y = pack_bf16x2(a.z * scale, a.w * scale);
-        w.z = pack_bf16x2(b.x * scale, b.y * scale);
-        w.w = pack_bf16x2(b.z * scale, b.w * scale);
-        reinterpret_cast<uint4*>(dq)[e] = w;
+        w.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * mul, __uint_as_float(r[v4 * 8 + 1]) * mul);
+        w.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * mul, __uint_as_float(r[v4 * 8 + 3]) * mul);
+        w.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * mul, __uint_as_float(r[v4 * 8 + 5]) * mul);
+        w.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * mul, __uint_as_float(r[v4 * 8 + 7]) * mul);
+        *reinterpret_cast<uint4*>(dst + v4 * 8) = w;
     }
 }
 
+// ===========================================================================
+// dK, dV: key-stationary
+// ===========================================================================
 template <int D>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
-swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
-    using C = BwdCfg<D>;
+struct BwdKVCfg {
+    static constexpr int BN = 128;                 // key rows per item (MMA M of S^T, dP^T, dV, dK)
+    static constexpr int BM = 128;                 // query rows per step
+    static constexpr int TILE = 128 * D * 2;
+    static constexpr int BOX = 128 * 64 * 2;
+    static constexpr int NBOX = D / 64;
+    static constexpr int NSTAGE = 2;               // Q_n / dO_n ring
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = TILE;
+    static constexpr int OFF_QD = 2 * TILE;        // stage s: Q at OFF_QD + s*2*TILE, dO after it
+    static constexpr int OFF_LSE = OFF_QD + NSTAGE * 2 * TILE;   // per stage: 128 floats lse*log2e, 128 Delta
+    static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
+    // k_full, k_empty, v_full, v_empty, qd_full x NSTAGE, qd_empty x NSTAGE, s_full, s_read, dp_full,
+    // dp_read, p_full, ds_full, dv_done, dk_done, mma_done, acc_full, acc_free; item_full, item_empty
+    // per ring entry
+    static constexpr int NUM_BAR = 4 + 2 * NSTAGE + 11 + 2 * kItemRing;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 64;
+    // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
+    // the kernel checks at run time that the aligned layout fits what it was given.
+    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;     // S^T (then P^T) | dP^T (then dS^T) | dV | dK
+    static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BM, 0, 0);       // K-major A, K-major B
+    static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);      // K-major A, MN-major B
+    static_assert(SMEM_USED <= 232448, "shared memory");
+};
+
+// Item of the key-stationary kernel: key block kblk of head (b, h); head-major, lowest key
+// blocks (the most query tiles under causal masking) first.
+struct BwdKVItem {
+    int b, h, bh;
+    long long k0;         // first key row
+    int ilo, nsteps;      // first query tile and number of query tiles in the band
+};
+
+__device__ __forceinline__ BwdKVItem bwd_kv_item(const BwdParams& p, int item) {
+    BwdKVItem it;
+    const int kblk = item % p.n_blk;
+    it.bh = item / p.n_blk;
+    it.b = it.bh / p.H;
+    it.h = it.bh % p.H;
+    it.k0 = (long long)kblk * 128;
+    it.ilo = kblk;
+    const int ihi = int(imin_ll(p.T - 1, it.k0 + 127 + p.W - 1) / 128);
+    it.nsteps = ihi - it.ilo + 1;
+    return it;
+}
+
+// Per step n (one query tile of the item):
+//   S^T = K Q^T -> TMEM S,   dP^T = V dO^T -> TMEM dP
+//   P^T = exp2(S^T scale log2e - lse2), masked; bf16 into TMEM S columns 0..63
+//   dV += P^T dO             (A operand from TMEM)
+//   dS^T = P^T (dP^T - Delta); bf16 into TMEM dP columns 0..63
+//   dK += dS^T Q             (A operand from TMEM)
+// With both products' left operands in TMEM only Q, dO, K and V are read from shared memory,
+// which keeps the tensor pipe within the SM's shared-memory bandwidth.  S^T(n+1) overwrites
+// P^T(n) and dP^T(n+1) overwrites dS^T(n), so MMA order dV(n) | S(n+1) | dK(n) | dP(n+1), each
+// after the MMA whose operand it overwrites has completed.
+template <int D>
+__global__ void __launch_bounds__(BwdKVCfg<D>::THREADS, 1)
+swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+    using C = BwdKVCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -195,17 +193,17 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return;
     }
 
-    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQD = base + C::OFF_QD, sDS = base + C::OFF_DS;
+    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQD = base + C::OFF_QD;
     const uint32_t sLSE = base + C::OFF_LSE;   // stage s: lse2 at sLSE + s*1024, Delta 512 bytes later
     const uint32_t bar0 = base + C::OFF_BAR;
-    const uint32_t kv_full = bar0, kv_empty = bar0 + 8;
-    auto qd_full = [&](int s) { return bar0 + 8u * (2 + s); };
-    auto qd_empty = [&](int s) { return bar0 + 8u * (2 + C::NSTAGE + s); };
-    const uint32_t bb = bar0 + 8u * (2 + 2 * C::NSTAGE);
-    const uint32_t s_full = bb, dp_full = bb + 8, p_full = bb + 16, ds_full = bb + 24, dv_done = bb + 32,
-                   dq_full = bb + 40, dq_free = bb + 48, ds_free = bb + 56, mma_done = bb + 64,
-                   dq_staged = bb + 72, acc_full = bb + 80, acc_free = bb + 88;
-    const uint32_t item_full0 = bb + 96, item_empty0 = item_full0 + 8u * kItemRing;
+    const uint32_t k_full = bar0, k_empty = bar0 + 8, v_full = bar0 + 16, v_empty = bar0 + 24;
+    auto qd_full = [&](int s) { return bar0 + 8u * (4 + s); };
+    auto qd_empty = [&](int s) { return bar0 + 8u * (4 + C::NSTAGE + s); };
+    const uint32_t bb = bar0 + 8u * (4 + 2 * C::NSTAGE);
+    const uint32_t s_full = bb, s_read = bb + 8, dp_full = bb + 16, dp_read = bb + 24, p_full = bb + 32,
+                   ds_full = bb + 40, dv_done = bb + 48, dk_done = bb + 56, mma_done = bb + 64,
+                   acc_full = bb + 72, acc_free = bb + 80;
+    const uint32_t item_full0 = bb + 88, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
     volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
@@ -214,22 +212,23 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const long long W = p.W;
     const int warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
-        mbar_init(kv_full, 1);
-        mbar_init(kv_empty, 1);
+        mbar_init(k_full, 1);
+        mbar_init(k_empty, 1);
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
         for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(qd_full(s), 1);
             mbar_init(qd_empty(s), 1);
         }
         mbar_init(s_full, 1);
+        mbar_init(s_read, 128);
         mbar_init(dp_full, 1);
-        mbar_init(p_full, 128);
-        mbar_init(ds_full, 128);
+        mbar_init(dp_read, 128);
+        mbar_init(p_full, 256);
+        mbar_init(ds_full, 256);
         mbar_init(dv_done, 1);
-        mbar_init(dq_full, 1);
-        mbar_init(dq_free, 128);
-        mbar_init(ds_free, 1);
+        mbar_init(dk_done, 1);
         mbar_init(mma_done, 1);
-        mbar_init(dq_staged, 128);
         mbar_init(acc_full, 1);
         mbar_init(acc_free, 256);
         for (int e = 0; e < kItemRing; ++e) {
@@ -252,29 +251,36 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
+        // Per item: K, the first Q/dO stage, V, then the other stages, so that S of the
+        // item's first step waits for K and one stage only.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            int n = 0, ki = 0;   // query-tile steps and items issued so far
+            int n = 0, nk = 0, nv = 0;   // stages, K tiles and V tiles issued so far
             bool ok = true;
-            for (;; ++ki) {
+            for (int ki = 0;; ++ki) {
                 const int item =
                     item_produce(p.work_slot, ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
-                const BwdItem g = bwd_item(p, item);
-                // K/V of the previous item are free once its last MMA completed.
-                if (ki > 0) {
-                    ok = mbar_wait(kv_empty, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
-                    if (!ok) break;
-                }
-                mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+                const BwdKVItem g = bwd_kv_item(p, item);
+                // K and V are read by this CTA alone: start them towards L2 while the previous
+                // item's last steps still hold the shared-memory tiles.
                 for (int x = 0; x < C::NBOX; ++x) {
-                    tma_load_4d(sK + x * C::BOX, &tm_k, kv_full, x * 64, g.h, int(g.k0), g.b);
-                    tma_load_4d(sV + x * C::BOX, &tm_v, kv_full, x * 64, g.h, int(g.k0), g.b);
+                    tma_prefetch_l2_4d(&tm_k, x * 64, g.h, int(g.k0), g.b);
+                    tma_prefetch_l2_4d(&tm_v, x * 64, g.h, int(g.k0), g.b);
                 }
-                for (int l = 0; l < g.nsteps; ++l, ++n) {
+                for (int l = 0; l < g.nsteps && ok; ++l) {
+                    if (l == 0) {   // K of the previous item is free once its last S completed
+                        if (ki > 0 && !(ok = mbar_wait(k_empty, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit,
+                                                       kStatusTimeoutProducer)))
+                            break;
+                        mbar_arrive_expect_tx(k_full, C::TILE);
+                        for (int x = 0; x < C::NBOX; ++x)
+                            tma_load_4d(sK + x * C::BOX, &tm_k, k_full, x * 64, g.h, int(g.k0), g.b);
+                        ++nk;
+                    }
                     const int s = n % C::NSTAGE;
                     if (!(ok = mbar_wait(qd_empty(s), ((n / C::NSTAGE) & 1) ^ 1u, abort_flag, p.wait_limit,
                                          kStatusTimeoutProducer)))
@@ -289,328 +295,636 @@ swa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const size_t row = size_t(g.bh) * p.Tp + size_t(qrow);
                     bulk_load(sLSE + s * 1024, p.lse2 + row, 512, qd_full(s));
                     bulk_load(sLSE + s * 1024 + 512, p.delta + row, 512, qd_full(s));
+                    ++n;
+                    if (l == 0) {   // V of the previous item is free once its last dP completed
+                        if (ki > 0 && !(ok = mbar_wait(v_empty, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit,
+                                                       kStatusTimeoutProducer)))
+                            break;
+                        mbar_arrive_expect_tx(v_full, C::TILE);
+                        for (int x = 0; x < C::NBOX; ++x)
+                            tma_load_4d(sV + x * C::BOX, &tm_v, v_full, x * 64, g.h, int(g.k0), g.b);
+                        ++nv;
+                    }
                 }
+                if (!ok) break;
             }
             work_slot_finish(p.work_slot);
-            // Drain: make sure no copy is still landing when the CTA exits.
+            // Drain: no copy of this CTA may still be landing when it exits.
             for (int s = 0; s < C::NSTAGE && s < n; ++s) {
                 const int fills = (n - s + C::NSTAGE - 1) / C::NSTAGE;
-                mbar_wait(qd_full(s), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                mbar_drain(qd_full(s), uint32_t((fills - 1) & 1), p.wait_limit);
             }
-            if (ki > 0) mbar_wait(kv_full, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            if (nk > 0) mbar_drain(k_full, uint32_t((nk - 1) & 1), p.wait_limit);
+            if (nv > 0) mbar_drain(v_full, uint32_t((nv - 1) & 1), p.wait_limit);
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             bool ok = true;
-            int n = 0, ki = 0;
-            for (;; ++ki) {
+            int n = 0;
+            auto stage_q = [&](int m) { return sQD + (m % C::NSTAGE) * 2 * C::TILE; };
+            auto wait = [&](uint32_t bar, int phase) {
+                return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+            };
+            // S^T(m) overwrites P^T(m-1): dV(m-1) must have completed.
+            auto issue_s = [&](int m, bool last) -> bool {
+                if (!wait(qd_full(m % C::NSTAGE), m / C::NSTAGE) || (m > 0 && !wait(dv_done, m - 1))) return false;
+                tc_fence_after();
+                const uint32_t sQ = stage_q(m);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), C::IDESC_S, kk > 0);
+                }
+                tc_commit(s_full);
+                if (last) tc_commit(k_empty);
+                return true;
+            };
+            // dP^T(m) overwrites dS^T(m-1): dK(m-1) must have completed.
+            auto issue_dp = [&](int m, bool last) -> bool {
+                if (m > 0 && !wait(dk_done, m - 1)) return false;
+                tc_fence_after();
+                const uint32_t sDO = stage_q(m) + C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), C::IDESC_S,
+                           kk > 0);
+                }
+                tc_commit(dp_full);
+                if (last) tc_commit(v_empty);
+                return true;
+            };
+            for (int ki = 0;; ++ki) {
                 const int item = item_consume_thread(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                      kStatusTimeoutMma, ok);
                 if (!ok || item >= p.n_items) break;
-                const BwdItem g = bwd_item(p, item);
-                ok = mbar_wait(kv_full, uint32_t(ki & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+                const BwdKVItem g = bwd_kv_item(p, item);
+                ok = wait(k_full, ki) && issue_s(n, g.nsteps == 1) && wait(v_full, ki) && issue_dp(n, g.nsteps == 1);
                 for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
-                    const int s = n % C::NSTAGE;
-                    const uint32_t par = uint32_t(n & 1);
-                    ok = mbar_wait(qd_full(s), (n / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                    if (!ok) break;
-                    const uint32_t sQ = sQD + s * 2 * C::TILE, sDO = sQ + C::TILE;
-                    // S^T overwrites the P^T columns read by dV of the previous step.
-                    if (n > 0) {
-                        ok = mbar_wait(dv_done, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                        if (!ok) break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                        mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), C::IDESC_S,
-                               kk > 0);
-                    }
-                    tc_commit(s_full);
-                    // dP^T reuses the columns the dQ drain of the previous step reads.
-                    if (n > 0) {
-                        ok = mbar_wait(dq_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                        mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), C::IDESC_S,
-                               kk > 0);
-                    }
-                    tc_commit(dp_full);
-                    // dV += P^T dO  (the previous item's epilogue must have read dV / dK first)
-                    ok = mbar_wait(p_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                    if (ok && l == 0 && ki > 0)
-                        ok = mbar_wait(acc_free, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
-                    if (!ok) break;
+                    const uint32_t sQ = stage_q(n), sDO = sQ + C::TILE;
+                    const bool more = l + 1 < g.nsteps;
+                    // dV += P^T dO  (the previous item's epilogue must have read dV / dK)
+                    if (!(ok = wait(p_full, n)) || (l == 0 && ki > 0 && !(ok = wait(acc_free, ki - 1)))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < C::BM / 16; ++kk)
                         mma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
                                (l > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(dv_done);
-                    // dK += dS^T Q ; dQ_i = dS K
-                    ok = mbar_wait(ds_full, par, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                    if (!ok) break;
+                    if (more && !(ok = issue_s(n + 1, l + 2 == g.nsteps))) break;
+                    // dK += dS^T Q
+                    if (!(ok = wait(ds_full, n))) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < C::BM / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                        mma_ss(tDK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, C::BOX, 1024),
-                               C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk)
-                        mma_ss(tDP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
-                               sdesc_sw128(sK + kk * 2048, C::BOX, 1024), C::IDESC_DQ, kk > 0);
-                    tc_commit(dq_full);   // also tells the dQ warps that stage s is no longer read by MMAs
-                    tc_commit(ds_free);
+                    for (int kk = 0; kk < C::BM / 16; ++kk)
+                        mma_ts(tDK, tDP + kk * 8, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
+                               (l > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(dk_done);
+                    tc_commit(qd_empty(n % C::NSTAGE));   // Q_n, dO_n, lse and Delta of step n are read
+                    if (more && !(ok = issue_dp(n + 1, l + 2 == g.nsteps))) break;
                 }
                 if (!ok) break;
                 tc_commit(acc_full);   // dV, dK of this item are final
-                tc_commit(kv_empty);   // K, V may be replaced by the next item's
             }
             tc_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
         }
-    } else if (warp < 4) {
-        // ------------------------------ key-row warps: P^T and dS^T ------------------------------
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    } else {
+        // ------------------------------ key-row warps: P^T, dS^T, epilogue ------------------------------
+        // Thread = key row (TMEM lane); warps 0..3 take query columns 0..63, warps 4..7 columns 64..127.
+        const int rh = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const float sl2 = p.scale_log2;
+        // Epilogue of the pki-th item (index pitem): warps 0..3 write this row's dV,
+        // warps 4..7 scale * dK.  It runs after P^T of the next item's first step, so the
+        // next item's S^T / P^T overlap the last dK of this one.
+        auto epilogue = [&](int pki, int pitem) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(acc_full, uint32_t(pki & 1), abort_flag, p.wait_limit,
+                                                   kStatusTimeoutEpilogue)))
+                return false;
+            tc_fence_after();
+            const BwdKVItem pg = bwd_kv_item(p, pitem);
+            const long long pkv = pg.k0 + row;
+            __nv_bfloat16* dst =
+                pkv < T ? (rh == 0 ? p.dv : p.dk) + ((size_t(pg.b) * T + size_t(pkv)) * p.H + pg.h) * D : nullptr;
+            const uint32_t src = (rh == 0 ? tDV : tDK) + lane_off;
+            const float mul = rh == 0 ? 1.f : p.scale;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {   // 32 columns at a time: P^T of the next step is live
+                uint32_t a[32];
+                tmem_ld32(src + c * 32, a);
+                tmem_ld_wait(a);
+                if (c == D / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(acc_free);
+                }
+                if (dst) store_row32_bf16(dst + c * 32, a, mul);
+            }
+            return true;
+        };
         bool ok = true;
-        int n = 0, ki = 0;
-        for (;; ++ki) {
+        int n = 0;
+        int prev_ki = -1, prev_item = 0;   // item whose epilogue is still pending
+        for (int ki = 0;; ++ki) {
             const int item = item_consume_warp(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                kStatusTimeoutSoftmax, ok);
             if (!ok || item >= p.n_items) break;
-            const BwdItem g = bwd_item(p, item);
+            const BwdKVItem g = bwd_kv_item(p, item);
             const long long k0 = g.k0;
             const long long kv = k0 + row;
             for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
                 const uint32_t par = uint32_t(n & 1);
                 const long long q0 = (long long)(g.ilo + l) * C::BM;
-                const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024;   // lse*log2e: 128 floats; Delta 512 bytes later
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024 + rh * 256;   // this half's 64 lse2 values
+                ok = __all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                // Both halves of the row (64 columns each) are requested before one wait.
-                float pr[C::BM];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
+                float pr[64];
+                {
                     uint32_t r0[32], r1[32];
-                    tmem_ld32(tS + lane_off + hh * 64, r0);
-                    tmem_ld32(tS + lane_off + hh * 64 + 32, r1);
-                    float lz[64];
-#pragma unroll
-                    for (int gq = 0; gq < 16; ++gq) {
-                        const float4 t4 = lds_f32x4(sL + (hh * 64 + gq * 4) * 4);
-                        lz[4 * gq] = t4.x;
-                        lz[4 * gq + 1] = t4.y;
-                        lz[4 * gq + 2] = t4.z;
-                        lz[4 * gq + 3] = t4.w;
-                    }
+                    tmem_ld32(tS + lane_off + rh * 64, r0);
+                    tmem_ld32(tS + lane_off + rh * 64 + 32, r1);
                     tmem_ld_wait(r0);
                     tmem_ld_wait(r1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        pr[hh * 64 + i] = ex2_approx(fmaf(__uint_as_float(r0[i]), sl2, -lz[i]));
-                        pr[hh * 64 + 32 + i] = ex2_approx(fmaf(__uint_as_float(r1[i]), sl2, -lz[32 + i]));
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 a = lds_f32x4(sL + gq * 16);
+                        const float4 b = lds_f32x4(sL + 128 + gq * 16);
+                        pr[4 * gq + 0] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 0]), sl2, -a.x));
+                        pr[4 * gq + 1] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 1]), sl2, -a.y));
+                        pr[4 * gq + 2] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 2]), sl2, -a.z));
+                        pr[4 * gq + 3] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 3]), sl2, -a.w));
+                        pr[32 + 4 * gq + 0] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 0]), sl2, -b.x));
+                        pr[32 + 4 * gq + 1] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 1]), sl2, -b.y));
+                        pr[32 + 4 * gq + 2] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 2]), sl2, -b.z));
+                        pr[32 + 4 * gq + 3] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 3]), sl2, -b.w));
                     }
                 }
-                // Tiles that cut the diagonal, the window's far edge or T: keep columns clo..chi of this
-                // key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
+                // Packed P^T of query columns 64..127 goes to TMEM columns 32..63, which hold S^T of
+                // query columns 32..63 that warps 0..3 read: those warps say when they have.
+                if (rh == 0) {
+                    tc_fence_before();
+                    mbar_arrive(s_read);
+                }
+                // Tiles that cut the diagonal, the window's far edge or T: keep query columns clo..chi
+                // of this key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
                 const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
                 if (!full) {
-                    const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1));
+                    const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1)) - rh * 64;
                     const int chi =
-                        kv < T ? int(imin_ll(imax_ll(imin_ll(kv + W - 1, (long long)T - 1) - q0, -1), C::BM)) : -1;
+                        (kv < T ? int(imin_ll(imax_ll(imin_ll(kv + W - 1, (long long)T - 1) - q0, -1), C::BM)) : -1) -
+                        rh * 64;
 #pragma unroll
-                    for (int col = 0; col < C::BM; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
+                    for (int col = 0; col < 64; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
                 }
-#pragma unroll
-                for (int c = 0; c < C::BM / 64; ++c) {
+                if (rh == 1) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(s_read, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                {
                     uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[c * 64 + 2 * i], pr[c * 64 + 2 * i + 1]);
-                    tmem_st32(tS + lane_off + c * 32, pk);
+                    for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
+                    tmem_st32(tS + lane_off + rh * 32, pk);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(p_full);
+                if (l == 0 && prev_ki >= 0) {
+                    if (!(ok = epilogue(prev_ki, prev_item))) break;
+                    prev_ki = -1;
+                }
                 // dS^T = P^T (dP^T - Delta)
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                ok = __all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                if (n > 0) {
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(ds_free, par ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
-                    if (!ok) break;
-                }
-#pragma unroll
-                for (int c = 0; c < C::BM / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tDP + lane_off + c * 32, r);
-                    float dz[32];
+                uint32_t w[32];
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tDP + lane_off + rh * 64, r0);
+                    tmem_ld32(tDP + lane_off + rh * 64 + 32, r1);
+                    tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
+                    if (rh == 0) {   // packed dS^T of columns 64..127 goes over dP^T columns 32..63
+                        tc_fence_before();
+                        mbar_arrive(dp_read);
+                    }
 #pragma unroll
                     for (int gq = 0; gq < 8; ++gq) {
-                        const float4 t4 = lds_f32x4(sL + 512 + (c * 32 + gq * 4) * 4);
-                        dz[4 * gq] = t4.x;
-                        dz[4 * gq + 1] = t4.y;
-                        dz[4 * gq + 2] = t4.z;
-                        dz[4 * gq + 3] = t4.w;
-                    }
-                    tmem_ld_wait(r);
-                    // 32 query columns = four 16-byte chunks of this key row in the 128B-swizzled tile.
-#pragma unroll
-                    for (int gq = 0; gq < 4; ++gq) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int col = c * 32 + gq * 8 + 2 * e;
-                            const float d0 = pr[col] * (__uint_as_float(r[gq * 8 + 2 * e]) - dz[gq * 8 + 2 * e]);
-                            const float d1 =
-                                pr[col + 1] * (__uint_as_float(r[gq * 8 + 2 * e + 1]) - dz[gq * 8 + 2 * e + 1]);
-                            w[e] = pack_bf16x2(d0, d1);
-                        }
-                        const int chunk = (c * 32 + gq * 8) >> 3;            // 0..15 across the 128 columns
-                        const int box = chunk >> 3, cib = chunk & 7;
-                        const uint32_t addr = sDS + box * C::BOX + row * 128 + ((cib ^ (row & 7)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
-                                     "r"(w[2]), "r"(w[3])
-                                     : "memory");
+                        const float4 a = lds_f32x4(sL + 512 + gq * 16);
+                        const float4 b = lds_f32x4(sL + 512 + 128 + gq * 16);
+                        const int c = 4 * gq;
+                        w[2 * gq] = pack_bf16x2(pr[c] * (__uint_as_float(r0[c]) - a.x),
+                                                pr[c + 1] * (__uint_as_float(r0[c + 1]) - a.y));
+                        w[2 * gq + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(r0[c + 2]) - a.z),
+                                                    pr[c + 3] * (__uint_as_float(r0[c + 3]) - a.w));
+                        w[16 + 2 * gq] = pack_bf16x2(pr[32 + c] * (__uint_as_float(r1[c]) - b.x),
+                                                     pr[33 + c] * (__uint_as_float(r1[c + 1]) - b.y));
+                        w[17 + 2 * gq] = pack_bf16x2(pr[34 + c] * (__uint_as_float(r1[c + 2]) - b.z),
+                                                     pr[35 + c] * (__uint_as_float(r1[c + 3]) - b.w));
                     }
                 }
-                fence_proxy_async_smem();
+                if (rh == 1) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(dp_read, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                tmem_st32(tDP + lane_off + rh * 32, w);
+                tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(ds_full);
             }
             if (!ok) break;
-            // ---- epilogue of the item: dV ----
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(acc_full, uint32_t(ki & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t dvr[D];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tDV + lane_off + c * 32, r);
-                tmem_ld_wait(r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) dvr[c * 32 + i] = r[i];
-            }
-            tc_fence_before();
-            mbar_arrive(acc_free);
-            if (kv < T) {
-                __nv_bfloat16* dst = p.dv + ((size_t(g.b) * T + size_t(kv)) * p.H + g.h) * D;
-#pragma unroll
-                for (int v8 = 0; v8 < D / 8; ++v8) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 0]), __uint_as_float(dvr[v8 * 8 + 1]));
-                    w.y = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 2]), __uint_as_float(dvr[v8 * 8 + 3]));
-                    w.z = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 4]), __uint_as_float(dvr[v8 * 8 + 5]));
-                    w.w = pack_bf16x2(__uint_as_float(dvr[v8 * 8 + 6]), __uint_as_float(dvr[v8 * 8 + 7]));
-                    *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
+            prev_ki = ki;
+            prev_item = item;
+        }
+        if (ok && prev_ki >= 0) epilogue(prev_ki, prev_item);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ===========================================================================
+// dQ: query-stationary
+// ===========================================================================
+template <int D>
+struct BwdQCfg {
+    static constexpr int BM = 128;                  // query rows per item (MMA M)
+    static constexpr int BN = 128;                  // key rows per step
+    static constexpr int TILE = 128 * D * 2;
+    static constexpr int BOX = 128 * 64 * 2;
+    static constexpr int NBOX = D / 64;
+    // Separate K and V rings: K_j is read by S(j) and dQ(j), V_j by dP(j) alone, so with one ring
+    // V_{j+1} would wait for the slot dQ(j-1) frees.
+    static constexpr int NK = D == 128 ? 3 : 6;
+    static constexpr int NV = D == 128 ? 2 : 4;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_DO = TILE;
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = OFF_K + NK * TILE;
+    static constexpr int OFF_BAR = OFF_V + NV * TILE;
+    // k_full, k_empty per K stage; v_full, v_empty per V stage; q_full, q_empty, do_full, do_empty;
+    // s_full x2, s_read x2, dq_done x2; dp_full, dp_free, ds_full, dq_full, dq_free, mma_done;
+    // item_full, item_empty per ring entry
+    static constexpr int NUM_BAR = 2 * (NK + NV) + 4 + 6 + 6 + 2 * kItemRing;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 64;
+    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
+    static constexpr int THREADS = 320;
+    static constexpr uint32_t TMEM_COLS = 512;      // S buffer 0 | S buffer 1 | dP | dQ
+    static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);    // K-major A, K-major B
+    static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);    // A from TMEM, MN-major B
+    static_assert(SMEM_USED <= 232448, "shared memory");
+};
+
+// Item of the query-stationary kernel: query tile qt of head (b, h); head-major, latest
+// query tiles (the most key tiles under causal masking) first.
+struct BwdQItem {
+    int b, h, bh;
+    long long q0;         // first query row
+    int jlo, jhi;         // key tiles of the band
+};
+
+__device__ __forceinline__ BwdQItem bwd_q_item(const BwdParams& p, int item) {
+    BwdQItem it;
+    const int qt = p.n_blk - 1 - item % p.n_blk;
+    it.bh = item / p.n_blk;
+    it.b = it.bh / p.H;
+    it.h = it.bh % p.H;
+    it.q0 = (long long)qt * 128;
+    it.jlo = int(imax_ll(0, it.q0 - p.W + 1) / 128);
+    it.jhi = qt;
+    return it;
+}
+
+// Per step n (one key tile j of the item):
+//   S = Q K_j^T -> TMEM S buffer n%2,   dP = dO V_j^T -> TMEM dP
+//   dS = exp2(S scale log2e - lse2) (dP - Delta), masked; bf16 back into the S buffer
+//   dQ += dS K_j                (A operand from TMEM)
+// The row warps hold dP in registers as soon as they have loaded it, so dP(n+1) is issued
+// before dQ(n): MMA order S(n+1) | dP(n+1) | dQ(n).
+template <int D>
+__global__ void __launch_bounds__(BwdQCfg<D>::THREADS, 1)
+swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+    using C = BwdQCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    if (int(base - raw) + C::SMEM_USED > C::SMEM) {   // uniform across the CTA: nothing started yet
+        if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusSmemLayout);
+        return;
+    }
+
+    const uint32_t sQ = base + C::OFF_Q, sDO = base + C::OFF_DO;
+    auto sK = [&](int m) { return base + C::OFF_K + uint32_t(m % C::NK) * C::TILE; };   // K of step m
+    auto sV = [&](int m) { return base + C::OFF_V + uint32_t(m % C::NV) * C::TILE; };   // V of step m
+    const uint32_t bar0 = base + C::OFF_BAR;
+    auto k_full = [&](int m) { return bar0 + 8u * (m % C::NK); };
+    auto k_empty = [&](int m) { return bar0 + 8u * (C::NK + m % C::NK); };
+    auto v_full = [&](int m) { return bar0 + 8u * (2 * C::NK + m % C::NV); };
+    auto v_empty = [&](int m) { return bar0 + 8u * (2 * C::NK + C::NV + m % C::NV); };
+    const uint32_t bb = bar0 + 8u * (2 * (C::NK + C::NV));
+    const uint32_t q_full = bb, q_empty = bb + 8, do_full = bb + 16, do_empty = bb + 24;
+    auto s_full = [&](int buf) { return bb + 32u + 8u * buf; };
+    auto s_read = [&](int buf) { return bb + 48u + 8u * buf; };
+    auto dq_done = [&](int buf) { return bb + 64u + 8u * buf; };
+    const uint32_t dp_full = bb + 80, dp_free = bb + 88, ds_full = bb + 96, dq_full = bb + 104,
+                   dq_free = bb + 112, mma_done = bb + 120;
+    const uint32_t item_full0 = bb + 128, item_empty0 = item_full0 + 8u * kItemRing;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
+    volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
+
+    const int T = p.T;
+    const long long W = p.W;
+    const int warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NK; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
+        }
+        for (int s = 0; s < C::NV; ++s) {
+            mbar_init(v_full(s), 1);
+            mbar_init(v_empty(s), 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        mbar_init(do_full, 1);
+        mbar_init(do_empty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full(b), 1);
+            mbar_init(s_read(b), 128);
+            mbar_init(dq_done(b), 1);
+        }
+        mbar_init(dp_full, 1);
+        mbar_init(dp_free, 256);
+        mbar_init(ds_full, 256);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_free, 256);
+        mbar_init(mma_done, 1);
+        for (int e = 0; e < kItemRing; ++e) {
+            mbar_init(item_full0 + 8u * e, 1);
+            mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and warps 0..7
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto tSb = [&](int buf) { return tmem + uint32_t(buf) * 128u; };
+    const uint32_t tDP = tmem + 256u, tDQ = tmem + 384u;
+
+    if (warp == 8) {
+        // ------------------------------ TMA producer ------------------------------
+        // Order per item: Q, K_jlo, dO, V_jlo, then K_j, V_j per step (Q and dO have their own buffers).
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            int n = 0, nq = 0, ndo = 0, nk = 0, nv = 0;   // steps, Q, dO, K and V tiles issued so far
+            bool ok = true;
+            auto wait_p = [&](uint32_t bar, int phase) {
+                return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+            };
+            for (int qi = 0;; ++qi) {
+                const int item =
+                    item_produce(p.work_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                if (!ok || item >= p.n_items) break;
+                const BwdQItem g = bwd_q_item(p, item);
+                // Q and dO are read by this CTA alone: start them towards L2 while the previous
+                // item's last steps still hold the shared-memory tiles.
+                for (int x = 0; x < C::NBOX; ++x) {
+                    tma_prefetch_l2_4d(&tm_q, x * 64, g.h, int(g.q0), g.b);
+                    tma_prefetch_l2_4d(&tm_do, x * 64, g.h, int(g.q0), g.b);
                 }
+                for (int j = g.jlo; j <= g.jhi; ++j, ++n) {
+                    if (j == g.jlo) {
+                        if (qi > 0 && !(ok = wait_p(q_empty, qi - 1))) break;
+                        mbar_arrive_expect_tx(q_full, C::TILE);
+                        for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sQ + x * C::BOX, &tm_q, q_full, x * 64, g.h, int(g.q0), g.b);
+                        ++nq;
+                    }
+                    if (!(ok = wait_p(k_empty(n), n / C::NK + 1))) break;   // first pass: the phase before 0
+                    mbar_arrive_expect_tx(k_full(n), C::TILE);
+                    for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sK(n) + x * C::BOX, &tm_k, k_full(n), x * 64, g.h, j * C::BN, g.b);
+                    ++nk;
+                    if (j == g.jlo) {
+                        if (qi > 0 && !(ok = wait_p(do_empty, qi - 1))) break;
+                        mbar_arrive_expect_tx(do_full, C::TILE);
+                        for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sDO + x * C::BOX, &tm_do, do_full, x * 64, g.h, int(g.q0), g.b);
+                        ++ndo;
+                    }
+                    if (!(ok = wait_p(v_empty(n), n / C::NV + 1))) break;
+                    mbar_arrive_expect_tx(v_full(n), C::TILE);
+                    for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sV(n) + x * C::BOX, &tm_v, v_full(n), x * 64, g.h, j * C::BN, g.b);
+                    ++nv;
+                }
+                if (!ok) break;
             }
+            work_slot_finish(p.work_slot);
+            // Drain: no copy of this CTA may still be landing when it exits.
+            for (int s = 0; s < C::NK && s < nk; ++s) mbar_drain(k_full(s), uint32_t(((nk - s + C::NK - 1) / C::NK - 1) & 1), p.wait_limit);
+            for (int s = 0; s < C::NV && s < nv; ++s) mbar_drain(v_full(s), uint32_t(((nv - s + C::NV - 1) / C::NV - 1) & 1), p.wait_limit);
+            if (nq > 0) mbar_drain(q_full, uint32_t((nq - 1) & 1), p.wait_limit);
+            if (ndo > 0) mbar_drain(do_full, uint32_t((ndo - 1) & 1), p.wait_limit);
+        }
+    } else if (warp == 9) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            bool ok = true;
+            int n = 0;   // steps (all items)
+            auto wait = [&](uint32_t bar, int phase) {
+                return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+            };
+            // S(m) goes to buffer m%2, which held dS(m-2) for dQ(m-2).
+            auto issue_s = [&](int m, bool last) -> bool {
+                if (!wait(k_full(m), m / C::NK) || (m >= 2 && !wait(dq_done(m & 1), (m - 2) >> 1))) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tSb(m & 1), sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK(m) + off, 16, 1024), C::IDESC_S,
+                           kk > 0);
+                }
+                tc_commit(s_full(m & 1));
+                if (last) tc_commit(q_empty);
+                return true;
+            };
+            // dP(m) overwrites dP(m-1), which the row warps have loaded once dp_free(m-1) completes.
+            auto issue_dp = [&](int m, bool last) -> bool {
+                if (!wait(v_full(m), m / C::NV) || (m > 0 && !wait(dp_free, m - 1))) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tDP, sdesc_sw128(sDO + off, 16, 1024), sdesc_sw128(sV(m) + off, 16, 1024), C::IDESC_S,
+                           kk > 0);
+                }
+                tc_commit(dp_full);
+                tc_commit(v_empty(m));   // V_j is read by this dP only
+                if (last) tc_commit(do_empty);
+                return true;
+            };
+            for (int qi = 0;; ++qi) {
+                const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                                     kStatusTimeoutMma, ok);
+                if (!ok || item >= p.n_items) break;
+                const BwdQItem g = bwd_q_item(p, item);
+                const int nsteps = g.jhi - g.jlo + 1;
+                ok = wait(q_full, qi) && issue_s(n, nsteps == 1) && wait(do_full, qi) && issue_dp(n, nsteps == 1);
+                for (int l = 0; l < nsteps && ok; ++l, ++n) {
+                    const bool more = l + 1 < nsteps;
+                    if (more && !(ok = issue_s(n + 1, l + 2 == nsteps) && issue_dp(n + 1, l + 2 == nsteps))) break;
+                    // dQ += dS K_j  (the previous item's epilogue must have read dQ)
+                    if (!(ok = wait(ds_full, n)) || (l == 0 && qi > 0 && !(ok = wait(dq_free, qi - 1)))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / 16; ++kk)
+                        mma_ts(tDQ, tSb(n & 1) + kk * 8, sdesc_sw128(sK(n) + kk * 2048, C::BOX, 1024), C::IDESC_DQ,
+                               (l > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(dq_done(n & 1));
+                    tc_commit(k_empty(n));   // K_j: read by S(n) and dQ(n)
+                }
+                if (!ok) break;
+                tc_commit(dq_full);   // dQ of this item is final
+            }
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
         }
     } else {
-        // ------------------------------ query-row warps: dQ drain; dK epilogue ------------------------------
-        const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
-        const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+        // ------------------------------ query-row warps: dS, epilogue ------------------------------
+        // Thread = query row (TMEM lane); warps 0..3 take key columns 0..63, warps 4..7 columns 64..127.
+        const int rh = warp >> 2;
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+        const float sl2 = p.scale_log2;
+        // Epilogue of item pqi (this row's half of dQ at dst, null past T): dQ = scale * acc.  It
+        // runs after P of the next item's first step, so that P overlaps the last dQ MMA.
+        auto epilogue = [&](int pqi, __nv_bfloat16* dst) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(dq_full, uint32_t(pqi & 1), abort_flag, p.wait_limit,
+                                                   kStatusTimeoutEpilogue)))
+                return false;
+            tc_fence_after();
+            uint32_t acc[D / 64][32];
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tmem_ld32(tDQ + lane_off + rh * (D / 2) + c * 32, acc[c]);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tmem_ld_wait(acc[c]);
+            tc_fence_before();
+            mbar_arrive(dq_free);
+            if (dst) {
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) store_row32_bf16(dst + c * 32, acc[c], p.scale);
+            }
+            return true;
+        };
         bool ok = true;
-        int n = 0, ki = 0;
-        for (;; ++ki) {
-            const int item = item_consume_warp(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+        int n = 0;
+        int prev_qi = -1;                  // item whose epilogue is still pending
+        __nv_bfloat16* prev_dst = nullptr;
+        for (int qi = 0;; ++qi) {
+            const int item = item_consume_warp(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                kStatusTimeoutSoftmax, ok);
             if (!ok || item >= p.n_items) break;
-            const BwdItem g = bwd_item(p, item);
-            for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
+            const BwdQItem g = bwd_q_item(p, item);
+            const long long q = g.q0 + row;
+            const size_t prow = size_t(g.bh) * p.Tp + size_t(q);   // padded rows: in bounds for every q
+            const float lse2_q = p.lse2[prow];
+            const float delta_q = p.delta[prow];
+            for (int j = g.jlo; j <= g.jhi && ok; ++j, ++n) {
+                const int buf = n & 1;
+                const uint32_t ph = uint32_t((n >> 1) & 1);
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait(dq_full, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
+                                mbar_wait(s_full(buf), ph, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                // Stage the fp32 dQ tile over Q_n / dO_n (no MMA reads them any more): D/32 boxes of
-                // 128 rows x 128 bytes, 128-byte swizzled like the TMA box of the reduce.
-                const int s = n % C::NSTAGE;
-                const uint32_t stg = sQD + s * 2 * C::TILE;
-#pragma unroll
-                for (int hh = 0; hh < D / 64; ++hh) {
+                float pr[64];
+                {
                     uint32_t r0[32], r1[32];
-                    tmem_ld32(tDP + lane_off + hh * 64, r0);
-                    tmem_ld32(tDP + lane_off + hh * 64 + 32, r1);
+                    tmem_ld32(tSb(buf) + lane_off + rh * 64, r0);
+                    tmem_ld32(tSb(buf) + lane_off + rh * 64 + 32, r1);
                     tmem_ld_wait(r0);
                     tmem_ld_wait(r1);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const uint32_t* rr = half ? r1 : r0;
-                        const int bx = hh * 2 + half;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint32_t addr = stg + bx * C::DQ_BOX + row * 128 + ((j ^ (row & 7)) << 4);
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(rr[j * 4]),
-                                         "r"(rr[j * 4 + 1]), "r"(rr[j * 4 + 2]), "r"(rr[j * 4 + 3])
-                                         : "memory");
-                        }
+                    for (int i = 0; i < 32; ++i) {
+                        pr[i] = ex2_approx(fmaf(__uint_as_float(r0[i]), sl2, -lse2_q));
+                        pr[32 + i] = ex2_approx(fmaf(__uint_as_float(r1[i]), sl2, -lse2_q));
                     }
                 }
+                // Packed dS of key columns 64..127 goes to TMEM columns 32..63 of the buffer, which hold
+                // S of key columns 32..63 that warps 0..3 read: those warps say when they have.
+                if (rh == 0) {
+                    tc_fence_before();
+                    mbar_arrive(s_read(buf));
+                }
+                // Tiles that cut the diagonal or the window's far edge: keep key columns clo..chi of this
+                // query row (keys q-W+1 .. q).  The test is uniform across the CTA.
+                const long long k0 = (long long)j * C::BN;
+                const bool full = (k0 + C::BN - 1 <= g.q0) && (k0 > g.q0 + C::BM - 1 - W);
+                if (!full) {
+                    const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN)) - rh * 64;
+                    const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1)) - rh * 64;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) pr[c] = (c >= clo && c <= chi) ? pr[c] : 0.f;
+                }
+                if (j == g.jlo && prev_qi >= 0) {
+                    if (!(ok = epilogue(prev_qi, prev_dst))) break;
+                    prev_qi = -1;
+                }
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(dp_full, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t pk[32];
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tDP + lane_off + rh * 64, r0);
+                    tmem_ld32(tDP + lane_off + rh * 64 + 32, r1);
+                    tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
+                    tc_fence_before();
+                    mbar_arrive(dp_free);   // dP(n+1) may be written
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        pk[i] = pack_bf16x2(pr[2 * i] * (__uint_as_float(r0[2 * i]) - delta_q),
+                                            pr[2 * i + 1] * (__uint_as_float(r0[2 * i + 1]) - delta_q));
+                        pk[16 + i] = pack_bf16x2(pr[32 + 2 * i] * (__uint_as_float(r1[2 * i]) - delta_q),
+                                                 pr[33 + 2 * i] * (__uint_as_float(r1[2 * i + 1]) - delta_q));
+                    }
+                }
+                if (rh == 1) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(s_read(buf), ph, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                tmem_st32(tSb(buf) + lane_off + rh * 32, pk);
+                tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(dq_free);
-                fence_proxy_async_smem();
-                mbar_arrive(dq_staged);
-                if (threadIdx.x == 128) {
-                    ok = mbar_wait(dq_staged, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue);
-                    if (ok) {
-                        for (int bx = 0; bx < D / 32; ++bx)
-                            tma_reduce_add_4d(&tm_dqacc, stg + bx * C::DQ_BOX, bx * 32, g.h, (g.ilo + l) * C::BM, g.b);
-                        bulk_commit_group();
-                        bulk_wait_group_read0();   // the stage may be refilled once the reduce has read it
-                        mbar_arrive(qd_empty(s));
-                    }
-                }
-                ok = __all_sync(0xffffffffu, ok);
+                mbar_arrive(ds_full);
             }
             if (!ok) break;
-            // ---- epilogue of the item: scale * dK ----
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(acc_full, uint32_t(ki & 1), abort_flag, p.wait_limit, kStatusTimeoutEpilogue));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t dkr[D];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tDK + lane_off + c * 32, r);
-                tmem_ld_wait(r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) dkr[c * 32 + i] = r[i];
-            }
-            tc_fence_before();
-            mbar_arrive(acc_free);
-            const long long kv = g.k0 + row;
-            if (kv < T) {
-                const float sc = p.scale;
-                __nv_bfloat16* dst = p.dk + ((size_t(g.b) * T + size_t(kv)) * p.H + g.h) * D;
-#pragma unroll
-                for (int v8 = 0; v8 < D / 8; ++v8) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 0]) * sc, __uint_as_float(dkr[v8 * 8 + 1]) * sc);
-                    w.y = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 2]) * sc, __uint_as_float(dkr[v8 * 8 + 3]) * sc);
-                    w.z = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 4]) * sc, __uint_as_float(dkr[v8 * 8 + 5]) * sc);
-                    w.w = pack_bf16x2(__uint_as_float(dkr[v8 * 8 + 6]) * sc, __uint_as_float(dkr[v8 * 8 + 7]) * sc);
-                    *reinterpret_cast<uint4*>(dst + v8 * 8) = w;
-                }
-            }
+            prev_qi = qi;
+            prev_dst = q < T ? p.dq + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D + rh * (D / 2) : nullptr;
         }
-        if (threadIdx.x == 128) bulk_wait_group0();
+        if (ok && prev_qi >= 0) epilogue(prev_qi, prev_dst);
     }
 
     tc_fence_before();

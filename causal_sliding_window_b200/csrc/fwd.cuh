@@ -210,11 +210,11 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // Drain: make sure no copy is still landing when the CTA exits.
             for (int s = 0; s < C::NSTAGE && s < it; ++s) {
                 const int fills = (it - s + C::NSTAGE - 1) / C::NSTAGE;
-                mbar_wait(kv_full(s), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                mbar_drain(kv_full(s), uint32_t((fills - 1) & 1), p.wait_limit);
             }
             for (int qb = 0; qb < C::NQBUF && qb < qi; ++qb) {
                 const int fills = (qi - qb + C::NQBUF - 1) / C::NQBUF;
-                mbar_wait(q_full(qb), uint32_t((fills - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                mbar_drain(q_full(qb), uint32_t((fills - 1) & 1), p.wait_limit);
             }
         }
     } else if (warp == 9) {
@@ -417,7 +417,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
                         sp[(2 * i) & 7] += p0;
                         sp[(2 * i + 1) & 7] += p1;
-                        pk[i] = pack_bf16x2(p0, p1);
+                        pk[i] = pack_bf16x2_alu(p0, p1);   // integer pipe: exp2 keeps the SFU
                     }
                     tmem_st32(tS + c * 32, pk);
                 }

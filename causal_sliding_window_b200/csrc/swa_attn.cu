@@ -39,21 +39,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // [B, T, H, D] bf16 viewed as a 4-D tensor (D, H, T, B), boxes of 64 x 1 x 128 x 1
 // with 128-byte swizzle (one box = 128 rows of one head, 64 columns).
-// fp32 [B, T, H, D] dQ accumulator as (D, H, T, B), boxes of 32 x 1 x 128 x 1 (128-byte swizzle),
-// target of the backward's TMA reduce-add.
-bool make_dqacc_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
-    auto enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
-    cuuint64_t strides[3] = {cuuint64_t(D) * 4, cuuint64_t(H) * D * 4, cuuint64_t(T) * H * D * 4};
-    cuuint32_t box[4] = {32, 1, 128, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 bool make_bthd_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
     auto enc = encode_fn();
     if (!enc) return false;
@@ -206,12 +191,11 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     return launch_status();
 }
 
-// Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128),
-// then the fp32 dQ accumulator [B, T, H, D].
+// Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128).
 size_t attn_bwd_workspace_bytes(int B, int T, int H, int D) {
     if (B < 1 || T < 1 || H < 1 || D < 1) return 0;
     const size_t Tp = (size_t(T) + 127) / 128 * 128;
-    return 2 * align256(size_t(B) * H * Tp * 4) + align256(size_t(B) * T * H * D * 4);
+    return 2 * align256(size_t(B) * H * Tp * 4);
 }
 
 int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
@@ -225,8 +209,8 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     if (!valid_common(B, T, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_bwd_workspace_bytes(B, T, H, D)) return ATTN_ERR_WORKSPACE;
-    const int n_kblk = (T + 127) / 128;
-    const long long n_items = (long long)n_kblk * B * H;
+    const int n_blk = (T + 127) / 128;
+    const long long n_items = (long long)n_blk * B * H;
     if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
     CUtensorMap mq, mk, mv, mdo;
@@ -237,26 +221,21 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     const size_t row_bytes = align256(size_t(B) * H * Tp * 4);
     float* lse2 = reinterpret_cast<float*>(workspace);
     float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + row_bytes);
-    float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * row_bytes);
-    CUtensorMap mdq;
-    if (!make_dqacc_map(&mdq, dq_acc, B, T, H, D)) return ATTN_ERR_LAUNCH;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long long rows = (long long)B * T * H;
     const auto* o_b = reinterpret_cast<const __nv_bfloat16*>(o);
     const auto* do_b = reinterpret_cast<const __nv_bfloat16*>(dout);
     if (D == 128)
-        swa_bwd_pre_kernel<128><<<grid_for(rows * 16, 256), 256, 0, s>>>(o_b, do_b, lse, lse2, delta, dq_acc, B,
-                                                                         T, H, Tp);
+        swa_bwd_pre_kernel<128><<<grid_for(rows * 16, 256), 256, 0, s>>>(o_b, do_b, lse, lse2, delta, B, T, H, Tp);
     else
-        swa_bwd_pre_kernel<64><<<grid_for(rows * 8, 256), 256, 0, s>>>(o_b, do_b, lse, lse2, delta, dq_acc, B, T,
-                                                                       H, Tp);
+        swa_bwd_pre_kernel<64><<<grid_for(rows * 8, 256), 256, 0, s>>>(o_b, do_b, lse, lse2, delta, B, T, H, Tp);
     if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
     if (g_ev_after_pre) cudaEventRecord(g_ev_after_pre, s);
 
     BwdParams p;
     p.lse2 = lse2;
     p.delta = delta;
-    p.dq_acc = dq_acc;
+    p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
     p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
     p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
     p.B = B;
@@ -265,22 +244,29 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     p.W = W;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.n_kblk = n_kblk;
+    p.n_blk = n_blk;
     p.n_items = int(n_items);
-    p.work_slot = next_work_slot();
     p.Tp = Tp;
     p.wait_limit = kDefaultWaitLimit;
+    // dK, dV (key-stationary), then dQ (query-stationary); each launch draws from its own counter.
+    p.work_slot = next_work_slot();
     if (D == 128) {
-        if (!ensure_smem((const void*)swa_bwd_kernel<128>, BwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_kernel<128><<<unsigned(grid), BwdCfg<128>::THREADS, BwdCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, mdq, p);
+        if (!ensure_smem((const void*)swa_bwd_dkdv_kernel<128>, BwdKVCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_bwd_dkdv_kernel<128><<<unsigned(grid), BwdKVCfg<128>::THREADS, BwdKVCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
     } else {
-        if (!ensure_smem((const void*)swa_bwd_kernel<64>, BwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_kernel<64><<<unsigned(grid), BwdCfg<64>::THREADS, BwdCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, mdq, p);
+        if (!ensure_smem((const void*)swa_bwd_dkdv_kernel<64>, BwdKVCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_bwd_dkdv_kernel<64><<<unsigned(grid), BwdKVCfg<64>::THREADS, BwdKVCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
     }
     if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
     if (g_ev_after_main) cudaEventRecord(g_ev_after_main, s);
-    const long long n8 = rows * D / 8;
-    swa_bwd_dq_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, reinterpret_cast<__nv_bfloat16*>(dq), n8, scale);
+    p.work_slot = next_work_slot();
+    if (D == 128) {
+        if (!ensure_smem((const void*)swa_bwd_dq_kernel<128>, BwdQCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_bwd_dq_kernel<128><<<unsigned(grid), BwdQCfg<128>::THREADS, BwdQCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
+    } else {
+        if (!ensure_smem((const void*)swa_bwd_dq_kernel<64>, BwdQCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_bwd_dq_kernel<64><<<unsigned(grid), BwdQCfg<64>::THREADS, BwdQCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
+    }
     return launch_status();
 }
 

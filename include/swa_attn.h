@@ -71,7 +71,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
              int B, int T, int H, int D, int W, float scale, void* stream);
 
 /* Bytes of workspace attn_bwd needs: fp32 rows of lse*log2(e) and Delta, [B*H, T rounded up
- * to 128] each, and the fp32 dQ accumulator [B,T,H,D]. */
+ * to 128] each (256-byte padded). */
 size_t attn_bwd_workspace_bytes(int B, int T, int H, int D);
 
 /*
@@ -82,7 +82,9 @@ size_t attn_bwd_workspace_bytes(int B, int T, int H, int D);
  *   workspace         device buffer of at least attn_bwd_workspace_bytes(B,T,H,D)
  *                     bytes, 256-byte aligned, contents need not be initialised;
  *                     ws_bytes smaller than required returns ATTN_ERR_WORKSPACE.
- * Probabilities are recomputed from lse; dQ is accumulated in fp32.
+ * Probabilities are recomputed from lse.  dK, dV and dQ are each accumulated in fp32
+ * on chip (tensor memory) and written once as bf16; no atomics, so results are
+ * bitwise reproducible run to run.
  * Defined by: training through flash_attn_func (apidog guide, section 5; the
  * training runs of its "scripts.base_train" walkthrough).
  */
@@ -140,9 +142,9 @@ int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn
 /*
  * Profiling aid: when set (non-NULL cudaEvent_t handles), every later
  * attn_bwd call made from this host thread records `after_pre` on its stream
- * right after the Delta / accumulator-zeroing launch and `after_main` right
- * after the main backward launch, so a caller that brackets attn_bwd with its
- * own events can time the three launches separately.  Pass NULLs to stop.
+ * right after the Delta / lse launch and `after_main` right after the dK/dV
+ * launch (the dQ launch follows it), so a caller that brackets attn_bwd with
+ * its own events can time the three launches separately.  Pass NULLs to stop.
  * Nothing else changes; no work is skipped.
  */
 int attn_bwd_set_profile_events(void* after_pre, void* after_main);

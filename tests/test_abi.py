@@ -71,9 +71,10 @@ def test_bwd_rejects_bad_arguments():
 
 
 def test_workspace_sizes():
-    # lse*log2e and Delta [B*H, Tp] fp32 + dQ accumulator [B,T,H,D] fp32, each 256-byte padded.
-    assert ops.attn_bwd_workspace_bytes(32, 2048, 12, 128) == 2 * 32 * 12 * 2048 * 4 + 32 * 2048 * 12 * 128 * 4
-    assert ops.attn_bwd_workspace_bytes(1, 130, 1, 64) == 2 * 256 * 4 + 130 * 64 * 4   # Tp = 256
+    # lse*log2e and Delta [B*H, Tp] fp32, each 256-byte padded.
+    assert ops.attn_bwd_workspace_bytes(32, 2048, 12, 128) == 2 * 32 * 12 * 2048 * 4
+    assert ops.attn_bwd_workspace_bytes(1, 130, 1, 64) == 2 * 256 * 4   # Tp = 256
+    assert ops.attn_bwd_workspace_bytes(1, 1, 1, 128) == 2 * 512   # 128 floats per row, no 256-byte padding needed
     assert ops.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
     # ticket counters [B] + partial (m, l) and o for ceil(cap / 128) chunks of 128 cache slots
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
