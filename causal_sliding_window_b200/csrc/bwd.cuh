@@ -132,9 +132,8 @@ struct BwdKVCfg {
     static constexpr int OFF_LSE = OFF_QD + NSTAGE * 2 * TILE;   // per stage: 128 floats lse*log2e, 128 Delta
     static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
     // k_full, k_empty, v_full, v_empty, qd_full x NSTAGE, qd_empty x NSTAGE, s_full, s_read, dp_full,
-    // dp_read, p_full, ds_full, dv_done, dk_done, mma_done, acc_full, acc_free; item_full, item_empty
-    // per ring entry
-    static constexpr int NUM_BAR = 4 + 2 * NSTAGE + 11 + 2 * kItemRing;
+    // dp_read, p_full, ds_full, mma_done, acc_full, acc_free; item_full, item_empty per ring entry
+    static constexpr int NUM_BAR = 4 + 2 * NSTAGE + 9 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
@@ -175,9 +174,10 @@ __device__ __forceinline__ BwdKVItem bwd_kv_item(const BwdParams& p, int item) {
 //   dS^T = P^T (dP^T - Delta); bf16 into TMEM dP columns 0..63
 //   dK += dS^T Q             (A operand from TMEM)
 // With both products' left operands in TMEM only Q, dO, K and V are read from shared memory,
-// which keeps the tensor pipe within the SM's shared-memory bandwidth.  S^T(n+1) overwrites
-// P^T(n) and dP^T(n+1) overwrites dS^T(n), so MMA order dV(n) | S(n+1) | dK(n) | dP(n+1), each
-// after the MMA whose operand it overwrites has completed.
+// which keeps the tensor pipe within the SM's shared-memory bandwidth.  MMA order
+// dV(n) | S(n+1) | dK(n) | dP(n+1): S^T(n+1) overwrites P^T(n) and dP^T(n+1) overwrites dS^T(n),
+// and the MMAs one thread issues execute in issue order, so neither waits for the MMA that
+// reads the columns it overwrites (the ordering the tensor pipe gives MMAs of one thread).
 template <int D>
 __global__ void __launch_bounds__(BwdKVCfg<D>::THREADS, 1)
 swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -201,9 +201,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto qd_empty = [&](int s) { return bar0 + 8u * (4 + C::NSTAGE + s); };
     const uint32_t bb = bar0 + 8u * (4 + 2 * C::NSTAGE);
     const uint32_t s_full = bb, s_read = bb + 8, dp_full = bb + 16, dp_read = bb + 24, p_full = bb + 32,
-                   ds_full = bb + 40, dv_done = bb + 48, dk_done = bb + 56, mma_done = bb + 64,
-                   acc_full = bb + 72, acc_free = bb + 80;
-    const uint32_t item_full0 = bb + 88, item_empty0 = item_full0 + 8u * kItemRing;
+                   ds_full = bb + 40, mma_done = bb + 48, acc_full = bb + 56, acc_free = bb + 64;
+    const uint32_t item_full0 = bb + 72, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
     volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
@@ -226,8 +225,6 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(dp_read, 128);
         mbar_init(p_full, 256);
         mbar_init(ds_full, 256);
-        mbar_init(dv_done, 1);
-        mbar_init(dk_done, 1);
         mbar_init(mma_done, 1);
         mbar_init(acc_full, 1);
         mbar_init(acc_free, 256);
@@ -326,9 +323,9 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             auto wait = [&](uint32_t bar, int phase) {
                 return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
             };
-            // S^T(m) overwrites P^T(m-1): dV(m-1) must have completed.
+            // S^T(m) overwrites P^T(m-1), read by dV(m-1), which this thread issued earlier.
             auto issue_s = [&](int m, bool last) -> bool {
-                if (!wait(qd_full(m % C::NSTAGE), m / C::NSTAGE) || (m > 0 && !wait(dv_done, m - 1))) return false;
+                if (!wait(qd_full(m % C::NSTAGE), m / C::NSTAGE)) return false;
                 tc_fence_after();
                 const uint32_t sQ = stage_q(m);
 #pragma unroll
@@ -340,10 +337,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (last) tc_commit(k_empty);
                 return true;
             };
-            // dP^T(m) overwrites dS^T(m-1): dK(m-1) must have completed.
-            auto issue_dp = [&](int m, bool last) -> bool {
-                if (m > 0 && !wait(dk_done, m - 1)) return false;
-                tc_fence_after();
+            // dP^T(m) overwrites dS^T(m-1), read by dK(m-1), which this thread issued earlier.
+            auto issue_dp = [&](int m, bool last) {
                 const uint32_t sDO = stage_q(m) + C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -353,14 +348,14 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 tc_commit(dp_full);
                 if (last) tc_commit(v_empty);
-                return true;
             };
             for (int ki = 0;; ++ki) {
                 const int item = item_consume_thread(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                      kStatusTimeoutMma, ok);
                 if (!ok || item >= p.n_items) break;
                 const BwdKVItem g = bwd_kv_item(p, item);
-                ok = wait(k_full, ki) && issue_s(n, g.nsteps == 1) && wait(v_full, ki) && issue_dp(n, g.nsteps == 1);
+                ok = wait(k_full, ki) && issue_s(n, g.nsteps == 1) && wait(v_full, ki);
+                if (ok) issue_dp(n, g.nsteps == 1);
                 for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
                     const uint32_t sQ = stage_q(n), sDO = sQ + C::TILE;
                     const bool more = l + 1 < g.nsteps;
@@ -371,7 +366,6 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int kk = 0; kk < C::BM / 16; ++kk)
                         mma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
                                (l > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(dv_done);
                     if (more && !(ok = issue_s(n + 1, l + 2 == g.nsteps))) break;
                     // dK += dS^T Q
                     if (!(ok = wait(ds_full, n))) break;
@@ -380,9 +374,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int kk = 0; kk < C::BM / 16; ++kk)
                         mma_ts(tDK, tDP + kk * 8, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
                                (l > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(dk_done);
                     tc_commit(qd_empty(n % C::NSTAGE));   // Q_n, dO_n, lse and Delta of step n are read
-                    if (more && !(ok = issue_dp(n + 1, l + 2 == g.nsteps))) break;
+                    if (more) issue_dp(n + 1, l + 2 == g.nsteps);
                 }
                 if (!ok) break;
                 tc_commit(acc_full);   // dV, dK of this item are final
@@ -570,9 +563,9 @@ struct BwdQCfg {
     static constexpr int OFF_V = OFF_K + NK * TILE;
     static constexpr int OFF_BAR = OFF_V + NV * TILE;
     // k_full, k_empty per K stage; v_full, v_empty per V stage; q_full, q_empty, do_full, do_empty;
-    // s_full x2, s_read x2, dq_done x2; dp_full, dp_free, ds_full, dq_full, dq_free, mma_done;
+    // s_full x2, s_read x2; dp_full, dp_free, ds_full, dq_full, dq_free, mma_done;
     // item_full, item_empty per ring entry
-    static constexpr int NUM_BAR = 2 * (NK + NV) + 4 + 6 + 6 + 2 * kItemRing;
+    static constexpr int NUM_BAR = 2 * (NK + NV) + 4 + 4 + 6 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
@@ -636,10 +629,9 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t q_full = bb, q_empty = bb + 8, do_full = bb + 16, do_empty = bb + 24;
     auto s_full = [&](int buf) { return bb + 32u + 8u * buf; };
     auto s_read = [&](int buf) { return bb + 48u + 8u * buf; };
-    auto dq_done = [&](int buf) { return bb + 64u + 8u * buf; };
-    const uint32_t dp_full = bb + 80, dp_free = bb + 88, ds_full = bb + 96, dq_full = bb + 104,
-                   dq_free = bb + 112, mma_done = bb + 120;
-    const uint32_t item_full0 = bb + 128, item_empty0 = item_full0 + 8u * kItemRing;
+    const uint32_t dp_full = bb + 64, dp_free = bb + 72, ds_full = bb + 80, dq_full = bb + 88,
+                   dq_free = bb + 96, mma_done = bb + 104;
+    const uint32_t item_full0 = bb + 112, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
     volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
@@ -663,7 +655,6 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full(b), 1);
             mbar_init(s_read(b), 128);
-            mbar_init(dq_done(b), 1);
         }
         mbar_init(dp_full, 1);
         mbar_init(dp_free, 256);
@@ -753,9 +744,9 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             auto wait = [&](uint32_t bar, int phase) {
                 return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
             };
-            // S(m) goes to buffer m%2, which held dS(m-2) for dQ(m-2).
+            // S(m) goes to buffer m%2, which held dS(m-2) for dQ(m-2): issued earlier by this thread.
             auto issue_s = [&](int m, bool last) -> bool {
-                if (!wait(k_full(m), m / C::NK) || (m >= 2 && !wait(dq_done(m & 1), (m - 2) >> 1))) return false;
+                if (!wait(k_full(m), m / C::NK)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -799,7 +790,6 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int kk = 0; kk < C::BN / 16; ++kk)
                         mma_ts(tDQ, tSb(n & 1) + kk * 8, sdesc_sw128(sK(n) + kk * 2048, C::BOX, 1024), C::IDESC_DQ,
                                (l > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(dq_done(n & 1));
                     tc_commit(k_empty(n));   // K_j: read by S(n) and dQ(n)
                 }
                 if (!ok) break;

@@ -244,15 +244,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                            (!first || kk > 0) ? 1u : 0u);
                 tc_commit(o_full(t));
             };
-            // S_t overwrites the columns the last PV_t read P from: wait for that PV first.
-            auto s_ready = [&](int t) -> bool {
-                const int n = t ? npv1 : npv0;
-                if (n == 0) return true;
-                if (!mbar_wait(o_full(t), uint32_t((n - 1) & 1), abort_flag, p.wait_limit, kStatusTimeoutMma))
-                    return false;
-                tc_fence_after();
-                return true;
-            };
+            // S_t overwrites the columns the last PV_t read P from; both are issued by this thread,
+            // and the MMAs of one thread execute in issue order, so S_t needs no wait for PV_t.
             for (;; ++qi) {
                 const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                      kStatusTimeoutMma, ok);
@@ -271,14 +264,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ++it;
                 if (!ok) break;
                 tc_fence_after();
-                if (act(0, g.jbeg)) {
-                    if (!(ok = s_ready(0))) break;
-                    issue_s(0, sk);
-                }
-                if (act(1, g.jbeg)) {
-                    if (!(ok = s_ready(1))) break;
-                    issue_s(1, sk);
-                }
+                if (act(0, g.jbeg)) issue_s(0, sk);
+                if (act(1, g.jbeg)) issue_s(1, sk);
                 for (int j = g.jbeg; j <= g.jend && ok; ++j) {
                     const int sv = it % C::NSTAGE;
                     ok = mbar_wait(kv_full(sv), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
@@ -315,10 +302,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             first = false;
                             ++npv;
                         }
-                        if (more && act(t, j + 1)) {
-                            if (!(ok = s_ready(t))) break;
-                            issue_s(t, sk_next);
-                        }
+                        if (more && act(t, j + 1)) issue_s(t, sk_next);
                     }
                     // K_j (read by the S MMAs issued one step earlier) and V_j are free once the
                     // MMAs issued so far complete.
