@@ -131,16 +131,16 @@ struct BwdKVCfg {
     static constexpr int OFF_QD = 2 * TILE;        // stage s: Q at OFF_QD + s*2*TILE, dO after it
     static constexpr int OFF_LSE = OFF_QD + NSTAGE * 2 * TILE;   // per stage: 128 floats lse*log2e, 128 Delta
     static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
-    // k_full, k_empty, v_full, v_empty, qd_full x NSTAGE, qd_empty x NSTAGE, s_full, s_read, dp_full,
-    // dp_read, p_full, ds_full, mma_done, acc_full, acc_free; item_full, item_empty per ring entry
-    static constexpr int NUM_BAR = 4 + 2 * NSTAGE + 9 + 2 * kItemRing;
+    // k_full, k_empty, v_full, v_empty, qd_full x NSTAGE, qd_empty x NSTAGE, s_full, s_free, dp_full,
+    // p_full, ds_full, mma_done, acc_full, acc_free; item_full, item_empty per ring entry
+    static constexpr int NUM_BAR = 4 + 2 * NSTAGE + 8 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
     // the kernel checks at run time that the aligned layout fits what it was given.
     static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
     static constexpr int THREADS = 320;
-    static constexpr uint32_t TMEM_COLS = 512;     // S^T (then P^T) | dP^T (then dS^T) | dV | dK
+    static constexpr uint32_t TMEM_COLS = 512;     // S^T | dP^T (then packed P^T, dS^T) | dV | dK
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BM, 0, 0);       // K-major A, K-major B
     static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);      // K-major A, MN-major B
     static_assert(SMEM_USED <= 232448, "shared memory");
@@ -169,15 +169,17 @@ __device__ __forceinline__ BwdKVItem bwd_kv_item(const BwdParams& p, int item) {
 
 // Per step n (one query tile of the item):
 //   S^T = K Q^T -> TMEM S,   dP^T = V dO^T -> TMEM dP
-//   P^T = exp2(S^T scale log2e - lse2), masked; bf16 into TMEM S columns 0..63
-//   dV += P^T dO             (A operand from TMEM)
-//   dS^T = P^T (dP^T - Delta); bf16 into TMEM dP columns 0..63
-//   dK += dS^T Q             (A operand from TMEM)
-// With both products' left operands in TMEM only Q, dO, K and V are read from shared memory,
-// which keeps the tensor pipe within the SM's shared-memory bandwidth.  MMA order
-// dV(n) | S(n+1) | dK(n) | dP(n+1): S^T(n+1) overwrites P^T(n) and dP^T(n+1) overwrites dS^T(n),
-// and the MMAs one thread issues execute in issue order, so neither waits for the MMA that
-// reads the columns it overwrites (the ordering the tensor pipe gives MMAs of one thread).
+//   P^T = exp2(S^T scale log2e - lse2), masked     (row warps, from registers)
+//   dS^T = P^T (dP^T - Delta)
+//   both packed to bf16 over the dP^T columns each warpgroup has loaded itself: warps 0..3
+//   (query columns 0..63) put P^T in TMEM columns 0..31 and dS^T in 32..63 of the dP region,
+//   warps 4..7 (query columns 64..127) in 64..95 and 96..127
+//   dV += P^T dO,   dK += dS^T Q   (A operands from TMEM)
+// The S columns hold S^T only, so S^T(n+1) is issued as soon as the row warps have loaded
+// S^T(n), a step ahead of its use; MMA order S(n+1) | dV(n) | dK(n) | dP(n+1).  dP^T(n+1)
+// overwrites the packed operands of dV(n) and dK(n): the MMAs one thread issues execute in
+// issue order, so it needs no wait for them.  With the left operands of dV and dK in TMEM,
+// only Q, dO, K and V are read from shared memory, within the SM's shared-memory bandwidth.
 template <int D>
 __global__ void __launch_bounds__(BwdKVCfg<D>::THREADS, 1)
 swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -200,9 +202,9 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto qd_full = [&](int s) { return bar0 + 8u * (4 + s); };
     auto qd_empty = [&](int s) { return bar0 + 8u * (4 + C::NSTAGE + s); };
     const uint32_t bb = bar0 + 8u * (4 + 2 * C::NSTAGE);
-    const uint32_t s_full = bb, s_read = bb + 8, dp_full = bb + 16, dp_read = bb + 24, p_full = bb + 32,
-                   ds_full = bb + 40, mma_done = bb + 48, acc_full = bb + 56, acc_free = bb + 64;
-    const uint32_t item_full0 = bb + 72, item_empty0 = item_full0 + 8u * kItemRing;
+    const uint32_t s_full = bb, s_free = bb + 8, dp_full = bb + 16, p_full = bb + 24, ds_full = bb + 32,
+                   mma_done = bb + 40, acc_full = bb + 48, acc_free = bb + 56;
+    const uint32_t item_full0 = bb + 64, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
     volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
@@ -220,9 +222,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(qd_empty(s), 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_read, 128);
+        mbar_init(s_free, 256);
         mbar_init(dp_full, 1);
-        mbar_init(dp_read, 128);
         mbar_init(p_full, 256);
         mbar_init(ds_full, 256);
         mbar_init(mma_done, 1);
@@ -323,9 +324,9 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             auto wait = [&](uint32_t bar, int phase) {
                 return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
             };
-            // S^T(m) overwrites P^T(m-1), read by dV(m-1), which this thread issued earlier.
+            // S^T(m) overwrites S^T(m-1), which the row warps have loaded once s_free(m-1) completes.
             auto issue_s = [&](int m, bool last) -> bool {
-                if (!wait(qd_full(m % C::NSTAGE), m / C::NSTAGE)) return false;
+                if (!wait(qd_full(m % C::NSTAGE), m / C::NSTAGE) || (m > 0 && !wait(s_free, m - 1))) return false;
                 tc_fence_after();
                 const uint32_t sQ = stage_q(m);
 #pragma unroll
@@ -337,8 +338,10 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (last) tc_commit(k_empty);
                 return true;
             };
-            // dP^T(m) overwrites dS^T(m-1), read by dK(m-1), which this thread issued earlier.
+            // dP^T(m) overwrites the packed operands of dV(m-1) and dK(m-1), issued earlier by this
+            // thread after the row warps had loaded dP^T(m-1).
             auto issue_dp = [&](int m, bool last) {
+                tc_fence_after();
                 const uint32_t sDO = stage_q(m) + C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -359,21 +362,21 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
                     const uint32_t sQ = stage_q(n), sDO = sQ + C::TILE;
                     const bool more = l + 1 < g.nsteps;
+                    if (more && !(ok = issue_s(n + 1, l + 2 == g.nsteps))) break;
                     // dV += P^T dO  (the previous item's epilogue must have read dV / dK)
                     if (!(ok = wait(p_full, n)) || (l == 0 && ki > 0 && !(ok = wait(acc_free, ki - 1)))) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < C::BM / 16; ++kk)
-                        mma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
-                               (l > 0 || kk > 0) ? 1u : 0u);
-                    if (more && !(ok = issue_s(n + 1, l + 2 == g.nsteps))) break;
+                    for (int kk = 0; kk < C::BM / 16; ++kk)   // query rows 16kk.. : P^T column pairs of warpgroup kk/4
+                        mma_ts(tDV, tDP + (kk >> 2) * 64 + (kk & 3) * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024),
+                               C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
                     // dK += dS^T Q
                     if (!(ok = wait(ds_full, n))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < C::BM / 16; ++kk)
-                        mma_ts(tDK, tDP + kk * 8, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), C::IDESC_ACC,
-                               (l > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts(tDK, tDP + (kk >> 2) * 64 + 32 + (kk & 3) * 8, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024),
+                               C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(qd_empty(n % C::NSTAGE));   // Q_n, dO_n, lse and Delta of step n are read
                     if (more) issue_dp(n + 1, l + 2 == g.nsteps);
                 }
@@ -391,8 +394,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const float sl2 = p.scale_log2;
         // Epilogue of the pki-th item (index pitem): warps 0..3 write this row's dV,
-        // warps 4..7 scale * dK.  It runs after P^T of the next item's first step, so the
-        // next item's S^T / P^T overlap the last dK of this one.
+        // warps 4..7 scale * dK.  It runs at the start of the next item's first step, while
+        // that step's S^T and dP^T MMAs (issued earlier) execute.
         auto epilogue = [&](int pki, int pitem) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(acc_full, uint32_t(pki & 1), abort_flag, p.wait_limit,
                                                    kStatusTimeoutEpilogue)))
@@ -405,15 +408,21 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t src = (rh == 0 ? tDV : tDK) + lane_off;
             const float mul = rh == 0 ? 1.f : p.scale;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {   // 32 columns at a time: P^T of the next step is live
-                uint32_t a[32];
-                tmem_ld32(src + c * 32, a);
-                tmem_ld_wait(a);
-                if (c == D / 32 - 1) {
+#pragma unroll
+            for (int c = 0; c < D / 32; c += 2) {   // 64 columns per wait
+                uint32_t a0[32], a1[32];
+                tmem_ld32(src + c * 32, a0);
+                tmem_ld32(src + c * 32 + 32, a1);
+                tmem_ld_wait(a0);
+                tmem_ld_wait(a1);
+                if (c + 2 == D / 32) {
                     tc_fence_before();
                     mbar_arrive(acc_free);
                 }
-                if (dst) store_row32_bf16(dst + c * 32, a, mul);
+                if (dst) {
+                    store_row32_bf16(dst + c * 32, a0, mul);
+                    store_row32_bf16(dst + c * 32 + 32, a1, mul);
+                }
             }
             return true;
         };
@@ -431,6 +440,11 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t par = uint32_t(n & 1);
                 const long long q0 = (long long)(g.ilo + l) * C::BM;
                 const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024 + rh * 256;   // this half's 64 lse2 values
+                // The previous item's dV / dK leave TMEM before this item's first dV.
+                if (l == 0 && prev_ki >= 0) {
+                    if (!(ok = epilogue(prev_ki, prev_item))) break;
+                    prev_ki = -1;
+                }
                 ok = __all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
@@ -441,6 +455,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tmem_ld32(tS + lane_off + rh * 64 + 32, r1);
                     tmem_ld_wait(r0);
                     tmem_ld_wait(r1);
+                    tc_fence_before();
+                    mbar_arrive(s_free);   // S^T(n+1) may be written
 #pragma unroll
                     for (int gq = 0; gq < 8; ++gq) {
                         const float4 a = lds_f32x4(sL + gq * 16);
@@ -455,12 +471,6 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         pr[32 + 4 * gq + 3] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 3]), sl2, -b.w));
                     }
                 }
-                // Packed P^T of query columns 64..127 goes to TMEM columns 32..63, which hold S^T of
-                // query columns 32..63 that warps 0..3 read: those warps say when they have.
-                if (rh == 0) {
-                    tc_fence_before();
-                    mbar_arrive(s_read);
-                }
                 // Tiles that cut the diagonal, the window's far edge or T: keep query columns clo..chi
                 // of this key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
                 const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
@@ -472,60 +482,54 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                     for (int col = 0; col < 64; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
                 }
-                if (rh == 1) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(s_read, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
-                    if (!ok) break;
-                    tc_fence_after();
-                }
-                {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
-                    tmem_st32(tS + lane_off + rh * 32, pk);
-                }
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(p_full);
-                if (l == 0 && prev_ki >= 0) {
-                    if (!(ok = epilogue(prev_ki, prev_item))) break;
-                    prev_ki = -1;
-                }
-                // dS^T = P^T (dP^T - Delta)
                 ok = __all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t w[32];
+                // This warpgroup's dP^T columns: the first 32 take packed P^T, the last 32 packed dS^T,
+                // each once its dP^T values are in registers.
+                const uint32_t tOwn = tDP + lane_off + rh * 64;
+                uint32_t w0[16];
                 {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(tDP + lane_off + rh * 64, r0);
-                    tmem_ld32(tDP + lane_off + rh * 64 + 32, r1);
-                    tmem_ld_wait(r0);
-                    tmem_ld_wait(r1);
-                    if (rh == 0) {   // packed dS^T of columns 64..127 goes over dP^T columns 32..63
-                        tc_fence_before();
-                        mbar_arrive(dp_read);
+                    uint32_t r[32];
+                    tmem_ld32(tOwn, r);
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pr[hh * 32 + 2 * i], pr[hh * 32 + 2 * i + 1]);
+                        tmem_st16(tOwn + hh * 16, pk);
                     }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(p_full);
+                    // dS^T = P^T (dP^T - Delta), query columns 0..31 of this half
 #pragma unroll
                     for (int gq = 0; gq < 8; ++gq) {
                         const float4 a = lds_f32x4(sL + 512 + gq * 16);
-                        const float4 b = lds_f32x4(sL + 512 + 128 + gq * 16);
                         const int c = 4 * gq;
-                        w[2 * gq] = pack_bf16x2(pr[c] * (__uint_as_float(r0[c]) - a.x),
-                                                pr[c + 1] * (__uint_as_float(r0[c + 1]) - a.y));
-                        w[2 * gq + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(r0[c + 2]) - a.z),
-                                                    pr[c + 3] * (__uint_as_float(r0[c + 3]) - a.w));
-                        w[16 + 2 * gq] = pack_bf16x2(pr[32 + c] * (__uint_as_float(r1[c]) - b.x),
-                                                     pr[33 + c] * (__uint_as_float(r1[c + 1]) - b.y));
-                        w[17 + 2 * gq] = pack_bf16x2(pr[34 + c] * (__uint_as_float(r1[c + 2]) - b.z),
-                                                     pr[35 + c] * (__uint_as_float(r1[c + 3]) - b.w));
+                        w0[2 * gq] = pack_bf16x2(pr[c] * (__uint_as_float(r[c]) - a.x),
+                                                 pr[c + 1] * (__uint_as_float(r[c + 1]) - a.y));
+                        w0[2 * gq + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(r[c + 2]) - a.z),
+                                                     pr[c + 3] * (__uint_as_float(r[c + 3]) - a.w));
                     }
                 }
-                if (rh == 1) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(dp_read, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
-                    if (!ok) break;
-                    tc_fence_after();
+                {
+                    uint32_t r[32], w1[16];   // query columns 32..63 of this half
+                    tmem_ld32(tOwn + 32, r);
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 a = lds_f32x4(sL + 512 + 128 + gq * 16);
+                        const int c = 4 * gq;
+                        w1[2 * gq] = pack_bf16x2(pr[32 + c] * (__uint_as_float(r[c]) - a.x),
+                                                 pr[33 + c] * (__uint_as_float(r[c + 1]) - a.y));
+                        w1[2 * gq + 1] = pack_bf16x2(pr[34 + c] * (__uint_as_float(r[c + 2]) - a.z),
+                                                     pr[35 + c] * (__uint_as_float(r[c + 3]) - a.w));
+                    }
+                    tmem_st16(tOwn + 32, w0);
+                    tmem_st16(tOwn + 48, w1);
                 }
-                tmem_st32(tDP + lane_off + rh * 32, w);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(ds_full);
