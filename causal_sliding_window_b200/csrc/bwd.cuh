@@ -125,15 +125,20 @@ struct BwdKVCfg {
     static constexpr int TILE = 128 * D * 2;
     static constexpr int BOX = 128 * 64 * 2;
     static constexpr int NBOX = D / 64;
-    static constexpr int NSTAGE = 2;               // Q_n / dO_n ring
+    // Q_n ring one deeper than the dO_n ring: S^T(n+1) is issued a step ahead of its use, while
+    // the Q and dO slots of step n are freed only once dK(n) has been issued.
+    static constexpr int NQ = D == 128 ? 3 : 4;
+    static constexpr int NDO = D == 128 ? 2 : 3;   // dO_n with step n's lse*log2e and Delta rows
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = TILE;
-    static constexpr int OFF_QD = 2 * TILE;        // stage s: Q at OFF_QD + s*2*TILE, dO after it
-    static constexpr int OFF_LSE = OFF_QD + NSTAGE * 2 * TILE;   // per stage: 128 floats lse*log2e, 128 Delta
-    static constexpr int OFF_BAR = OFF_LSE + NSTAGE * 2 * 128 * 4;
-    // k_full, k_empty, v_full, v_empty, qd_full x NSTAGE, qd_empty x NSTAGE, s_full, s_free, dp_full,
-    // p_full, ds_full, mma_done, acc_full, acc_free; item_full, item_empty per ring entry
-    static constexpr int NUM_BAR = 4 + 2 * NSTAGE + 8 + 2 * kItemRing;
+    static constexpr int OFF_Q = 2 * TILE;
+    static constexpr int OFF_DO = OFF_Q + NQ * TILE;
+    static constexpr int OFF_LSE = OFF_DO + NDO * TILE;   // per dO stage: 128 floats lse*log2e, 128 Delta
+    static constexpr int OFF_BAR = OFF_LSE + NDO * 2 * 128 * 4;
+    // k_full, k_empty, v_full, v_empty, q_full x NQ, q_empty x NQ, do_full x NDO, do_empty x NDO,
+    // s_full, s_free, dp_full, p_full, ds_full, mma_done, acc_full, acc_free; item_full, item_empty
+    // per ring entry
+    static constexpr int NUM_BAR = 4 + 2 * NQ + 2 * NDO + 8 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
@@ -195,13 +200,18 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         return;
     }
 
-    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sQD = base + C::OFF_QD;
-    const uint32_t sLSE = base + C::OFF_LSE;   // stage s: lse2 at sLSE + s*1024, Delta 512 bytes later
+    const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+    auto sQ = [&](int m) { return base + C::OFF_Q + uint32_t(m % C::NQ) * C::TILE; };     // Q of step m
+    auto sDO = [&](int m) { return base + C::OFF_DO + uint32_t(m % C::NDO) * C::TILE; };  // dO of step m
+    // lse2 of step m at sLSE(m), Delta 512 bytes later
+    auto sLSE = [&](int m) { return base + C::OFF_LSE + uint32_t(m % C::NDO) * 1024u; };
     const uint32_t bar0 = base + C::OFF_BAR;
     const uint32_t k_full = bar0, k_empty = bar0 + 8, v_full = bar0 + 16, v_empty = bar0 + 24;
-    auto qd_full = [&](int s) { return bar0 + 8u * (4 + s); };
-    auto qd_empty = [&](int s) { return bar0 + 8u * (4 + C::NSTAGE + s); };
-    const uint32_t bb = bar0 + 8u * (4 + 2 * C::NSTAGE);
+    auto q_full = [&](int m) { return bar0 + 8u * (4 + m % C::NQ); };
+    auto q_empty = [&](int m) { return bar0 + 8u * (4 + C::NQ + m % C::NQ); };
+    auto do_full = [&](int m) { return bar0 + 8u * (4 + 2 * C::NQ + m % C::NDO); };
+    auto do_empty = [&](int m) { return bar0 + 8u * (4 + 2 * C::NQ + C::NDO + m % C::NDO); };
+    const uint32_t bb = bar0 + 8u * (4 + 2 * C::NQ + 2 * C::NDO);
     const uint32_t s_full = bb, s_free = bb + 8, dp_full = bb + 16, p_full = bb + 24, ds_full = bb + 32,
                    mma_done = bb + 40, acc_full = bb + 48, acc_free = bb + 56;
     const uint32_t item_full0 = bb + 64, item_empty0 = item_full0 + 8u * kItemRing;
@@ -217,9 +227,13 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(k_empty, 1);
         mbar_init(v_full, 1);
         mbar_init(v_empty, 1);
-        for (int s = 0; s < C::NSTAGE; ++s) {
-            mbar_init(qd_full(s), 1);
-            mbar_init(qd_empty(s), 1);
+        for (int s = 0; s < C::NQ; ++s) {
+            mbar_init(q_full(s), 1);
+            mbar_init(q_empty(s), 1);
+        }
+        for (int s = 0; s < C::NDO; ++s) {
+            mbar_init(do_full(s), 1);
+            mbar_init(do_empty(s), 1);
         }
         mbar_init(s_full, 1);
         mbar_init(s_free, 256);
@@ -249,14 +263,14 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
-        // Per item: K, the first Q/dO stage, V, then the other stages, so that S of the
-        // item's first step waits for K and one stage only.
+        // Per item: K, Q_first, V, dO_first, then Q and dO per step, so that S of the item's
+        // first step waits for K and one Q tile only.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            int n = 0, nk = 0, nv = 0;   // stages, K tiles and V tiles issued so far
+            int n = 0, nq = 0, nk = 0, nv = 0;   // steps (dO tiles), Q, K and V tiles issued so far
             bool ok = true;
             for (int ki = 0;; ++ki) {
                 const int item =
@@ -279,21 +293,14 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             tma_load_4d(sK + x * C::BOX, &tm_k, k_full, x * 64, g.h, int(g.k0), g.b);
                         ++nk;
                     }
-                    const int s = n % C::NSTAGE;
-                    if (!(ok = mbar_wait(qd_empty(s), ((n / C::NSTAGE) & 1) ^ 1u, abort_flag, p.wait_limit,
+                    const int qrow = (g.ilo + l) * C::BM;
+                    if (!(ok = mbar_wait(q_empty(n), ((n / C::NQ) & 1) ^ 1u, abort_flag, p.wait_limit,
                                          kStatusTimeoutProducer)))
                         break;
-                    const int qrow = (g.ilo + l) * C::BM;
-                    mbar_arrive_expect_tx(qd_full(s), 2 * C::TILE + 1024);
-                    const uint32_t dst = sQD + s * 2 * C::TILE;
-                    for (int x = 0; x < C::NBOX; ++x) {
-                        tma_load_4d(dst + x * C::BOX, &tm_q, qd_full(s), x * 64, g.h, qrow, g.b);
-                        tma_load_4d(dst + C::TILE + x * C::BOX, &tm_do, qd_full(s), x * 64, g.h, qrow, g.b);
-                    }
-                    const size_t row = size_t(g.bh) * p.Tp + size_t(qrow);
-                    bulk_load(sLSE + s * 1024, p.lse2 + row, 512, qd_full(s));
-                    bulk_load(sLSE + s * 1024 + 512, p.delta + row, 512, qd_full(s));
-                    ++n;
+                    mbar_arrive_expect_tx(q_full(n), C::TILE);
+                    for (int x = 0; x < C::NBOX; ++x)
+                        tma_load_4d(sQ(n) + x * C::BOX, &tm_q, q_full(n), x * 64, g.h, qrow, g.b);
+                    ++nq;
                     if (l == 0) {   // V of the previous item is free once its last dP completed
                         if (ki > 0 && !(ok = mbar_wait(v_empty, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit,
                                                        kStatusTimeoutProducer)))
@@ -303,15 +310,25 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             tma_load_4d(sV + x * C::BOX, &tm_v, v_full, x * 64, g.h, int(g.k0), g.b);
                         ++nv;
                     }
+                    if (!(ok = mbar_wait(do_empty(n), ((n / C::NDO) & 1) ^ 1u, abort_flag, p.wait_limit,
+                                         kStatusTimeoutProducer)))
+                        break;
+                    mbar_arrive_expect_tx(do_full(n), C::TILE + 1024);
+                    for (int x = 0; x < C::NBOX; ++x)
+                        tma_load_4d(sDO(n) + x * C::BOX, &tm_do, do_full(n), x * 64, g.h, qrow, g.b);
+                    const size_t row = size_t(g.bh) * p.Tp + size_t(qrow);
+                    bulk_load(sLSE(n), p.lse2 + row, 512, do_full(n));
+                    bulk_load(sLSE(n) + 512, p.delta + row, 512, do_full(n));
+                    ++n;
                 }
                 if (!ok) break;
             }
             work_slot_finish(p.work_slot);
             // Drain: no copy of this CTA may still be landing when it exits.
-            for (int s = 0; s < C::NSTAGE && s < n; ++s) {
-                const int fills = (n - s + C::NSTAGE - 1) / C::NSTAGE;
-                mbar_drain(qd_full(s), uint32_t((fills - 1) & 1), p.wait_limit);
-            }
+            for (int s = 0; s < C::NQ && s < nq; ++s)
+                mbar_drain(q_full(s), uint32_t(((nq - s + C::NQ - 1) / C::NQ - 1) & 1), p.wait_limit);
+            for (int s = 0; s < C::NDO && s < n; ++s)
+                mbar_drain(do_full(s), uint32_t(((n - s + C::NDO - 1) / C::NDO - 1) & 1), p.wait_limit);
             if (nk > 0) mbar_drain(k_full, uint32_t((nk - 1) & 1), p.wait_limit);
             if (nv > 0) mbar_drain(v_full, uint32_t((nv - 1) & 1), p.wait_limit);
         }
@@ -320,19 +337,18 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (lane == 0) {
             bool ok = true;
             int n = 0;
-            auto stage_q = [&](int m) { return sQD + (m % C::NSTAGE) * 2 * C::TILE; };
             auto wait = [&](uint32_t bar, int phase) {
                 return mbar_wait(bar, uint32_t(phase & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
             };
             // S^T(m) overwrites S^T(m-1), which the row warps have loaded once s_free(m-1) completes.
             auto issue_s = [&](int m, bool last) -> bool {
-                if (!wait(qd_full(m % C::NSTAGE), m / C::NSTAGE) || (m > 0 && !wait(s_free, m - 1))) return false;
+                if (!wait(q_full(m), m / C::NQ) || (m > 0 && !wait(s_free, m - 1))) return false;
                 tc_fence_after();
-                const uint32_t sQ = stage_q(m);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), C::IDESC_S, kk > 0);
+                    mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ(m) + off, 16, 1024), C::IDESC_S,
+                           kk > 0);
                 }
                 tc_commit(s_full);
                 if (last) tc_commit(k_empty);
@@ -340,27 +356,26 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             };
             // dP^T(m) overwrites the packed operands of dV(m-1) and dK(m-1), issued earlier by this
             // thread after the row warps had loaded dP^T(m-1).
-            auto issue_dp = [&](int m, bool last) {
+            auto issue_dp = [&](int m, bool last) -> bool {
+                if (!wait(do_full(m), m / C::NDO)) return false;
                 tc_fence_after();
-                const uint32_t sDO = stage_q(m) + C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), C::IDESC_S,
+                    mma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO(m) + off, 16, 1024), C::IDESC_S,
                            kk > 0);
                 }
                 tc_commit(dp_full);
                 if (last) tc_commit(v_empty);
+                return true;
             };
             for (int ki = 0;; ++ki) {
                 const int item = item_consume_thread(ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                      kStatusTimeoutMma, ok);
                 if (!ok || item >= p.n_items) break;
                 const BwdKVItem g = bwd_kv_item(p, item);
-                ok = wait(k_full, ki) && issue_s(n, g.nsteps == 1) && wait(v_full, ki);
-                if (ok) issue_dp(n, g.nsteps == 1);
+                ok = wait(k_full, ki) && issue_s(n, g.nsteps == 1) && wait(v_full, ki) && issue_dp(n, g.nsteps == 1);
                 for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
-                    const uint32_t sQ = stage_q(n), sDO = sQ + C::TILE;
                     const bool more = l + 1 < g.nsteps;
                     if (more && !(ok = issue_s(n + 1, l + 2 == g.nsteps))) break;
                     // dV += P^T dO  (the previous item's epilogue must have read dV / dK)
@@ -368,17 +383,18 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < C::BM / 16; ++kk)   // query rows 16kk.. : P^T column pairs of warpgroup kk/4
-                        mma_ts(tDV, tDP + (kk >> 2) * 64 + (kk & 3) * 8, sdesc_sw128(sDO + kk * 2048, C::BOX, 1024),
+                        mma_ts(tDV, tDP + (kk >> 2) * 64 + (kk & 3) * 8, sdesc_sw128(sDO(n) + kk * 2048, C::BOX, 1024),
                                C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
                     // dK += dS^T Q
                     if (!(ok = wait(ds_full, n))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < C::BM / 16; ++kk)
-                        mma_ts(tDK, tDP + (kk >> 2) * 64 + 32 + (kk & 3) * 8, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024),
+                        mma_ts(tDK, tDP + (kk >> 2) * 64 + 32 + (kk & 3) * 8, sdesc_sw128(sQ(n) + kk * 2048, C::BOX, 1024),
                                C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(qd_empty(n % C::NSTAGE));   // Q_n, dO_n, lse and Delta of step n are read
-                    if (more) issue_dp(n + 1, l + 2 == g.nsteps);
+                    tc_commit(q_empty(n));    // Q_n is read
+                    tc_commit(do_empty(n));   // dO_n, lse and Delta of step n are read
+                    if (more && !(ok = issue_dp(n + 1, l + 2 == g.nsteps))) break;
                 }
                 if (!ok) break;
                 tc_commit(acc_full);   // dV, dK of this item are final
@@ -439,13 +455,17 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
                 const uint32_t par = uint32_t(n & 1);
                 const long long q0 = (long long)(g.ilo + l) * C::BM;
-                const uint32_t sL = sLSE + (n % C::NSTAGE) * 1024 + rh * 256;   // this half's 64 lse2 values
+                const uint32_t sL = sLSE(n) + rh * 256;   // this half's 64 lse2 values
                 // The previous item's dV / dK leave TMEM before this item's first dV.
                 if (l == 0 && prev_ki >= 0) {
                     if (!(ok = epilogue(prev_ki, prev_item))) break;
                     prev_ki = -1;
                 }
-                ok = __all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+                // S^T(n) implies Q_n has landed, not the dO_n stage that carries lse and Delta.
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(s_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax) &&
+                                    mbar_wait(do_full(n), uint32_t((n / C::NDO) & 1), abort_flag, p.wait_limit,
+                                              kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
                 float pr[64];
