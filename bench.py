@@ -85,6 +85,39 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+PROFILE_FOR_KERNEL = {
+    "swa_bwd_dkdv_kernel<128>": "swa_bwd_dkdv_kernel_d24shape_b8.md",
+    "swa_bwd_dq_kernel<128>": "swa_bwd_dq_kernel_d24shape_b8.md",
+    "swa_fwd_kernel<128>": "swa_fwd_kernel_d24shape_b8.md",
+    "swa_decode_kernel<128>": "swa_decode_kernel_decode_workload.md",
+}
+
+
+def measured_traffic(kernel, windows, batch):
+    """DRAM bytes per launch (read + write) of `kernel` from its committed ncu summary, scaled from
+    the captured batch to `batch` and averaged over the step's launches (one per window); None when
+    there is no summary or the kernel's sources changed since the capture (fingerprint mismatch)."""
+    import hashlib
+    import re
+
+    name = PROFILE_FOR_KERNEL.get(kernel)
+    path = os.path.join(ROOT, "profiles", name) if name else None
+    if not path or not os.path.exists(path):
+        return None
+    m = re.search(r"^traffic_bytes: (.*); batch (\d+); source_sha256 ([0-9a-f]{64}) \((.*)\)$",
+                  open(path).read(), flags=re.M)
+    if not m:
+        return None
+    per_w = {int(w): int(b) for w, b in re.findall(r"W=(\d+) (\d+)", m.group(1))}
+    h = hashlib.sha256()
+    for f in m.group(4).split(" + "):
+        with open(os.path.join(ROOT, "causal_sliding_window_b200", "csrc", f.strip()), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != m.group(3) or any(w not in per_w for w in windows):
+        return None
+    return sum(per_w[w] for w in windows) / len(windows) * batch / int(m.group(2))
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling of one GPU while the timed region runs."""
 
@@ -435,7 +468,9 @@ def main():
             roof = {"kernel": "swa_bwd_dkdv_kernel<128>", "bound": "tensor", "achieved": dkdv_tf, "peak": peak_t,
                     "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = None
+        roof["traffic"] = (measured_traffic(roof["kernel"], dwins, dB) if roof["kernel"].startswith("swa_decode")
+                           else measured_traffic(roof["kernel"], windows, B))
+        roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
         roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['unit'] == 'TFLOP/s' else 'copy'})"
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
