@@ -1,8 +1,10 @@
 """ctypes wrapper around the C oracle (test infrastructure; see package docstring).
 
 Inputs are numpy arrays holding either bf16 bit patterns (dtype uint16) or
-float64 values; outputs are float64. Shapes: q/k/v/dO ``[B, T, H, D]``, lse
-``[B, H, T]``; decode q ``[B, H, D]``, caches ``[B, cap, H, D]``.
+float64 values; outputs are float64. Shapes: q/dO ``[B, T, H, D]``, k/v
+``[B, T, Hk, D]`` with Hk dividing H (query head h reads K/V head h // (H // Hk);
+Hk = H is plain multi-head attention), lse ``[B, H, T]``; decode q ``[B, H, D]``,
+caches ``[B, cap, Hk, D]``.
 """
 from __future__ import annotations
 
@@ -37,12 +39,12 @@ def _load():
             lib = ctypes.CDLL(build_oracle())
             vp, L, d, dp, lp, ip = (ctypes.c_void_p, ctypes.c_long, ctypes.c_double,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p)
-            lib.swa_oracle_fwd.argtypes = [vp, vp, vp, ctypes.c_int, L, L, L, L, L, d, dp, dp]
-            lib.swa_oracle_fwd_rows.argtypes = [vp, vp, vp, ctypes.c_int, L, L, L, L, L, d, L, lp, dp, dp]
-            lib.swa_oracle_bwd.argtypes = [vp, vp, vp, vp, ctypes.c_int, L, L, L, L, L, d, dp, dp, dp]
-            lib.swa_oracle_dq_rows.argtypes = [vp, vp, vp, vp, ctypes.c_int, L, L, L, L, L, d, L, lp, dp]
-            lib.swa_oracle_dkv_rows.argtypes = [vp, vp, vp, vp, ctypes.c_int, L, L, L, L, L, d, L, lp, dp, dp]
-            lib.swa_oracle_decode.argtypes = [vp, vp, vp, ctypes.c_int, ip, L, L, L, L, L, d, dp, dp]
+            lib.swa_oracle_fwd.argtypes = [vp, vp, vp, ctypes.c_int, L, L, L, L, L, L, d, dp, dp]
+            lib.swa_oracle_fwd_rows.argtypes = [vp, vp, vp, ctypes.c_int, L, L, L, L, L, L, d, L, lp, dp, dp]
+            lib.swa_oracle_bwd.argtypes = [vp, vp, vp, vp, ctypes.c_int, L, L, L, L, L, L, d, dp, dp, dp]
+            lib.swa_oracle_dq_rows.argtypes = [vp, vp, vp, vp, ctypes.c_int, L, L, L, L, L, L, d, L, lp, dp]
+            lib.swa_oracle_dkv_rows.argtypes = [vp, vp, vp, vp, ctypes.c_int, L, L, L, L, L, L, d, L, lp, dp, dp]
+            lib.swa_oracle_decode.argtypes = [vp, vp, vp, ctypes.c_int, ip, L, L, L, L, L, L, d, dp, dp]
             for f in ("swa_oracle_fwd", "swa_oracle_fwd_rows", "swa_oracle_bwd", "swa_oracle_dq_rows",
                       "swa_oracle_dkv_rows", "swa_oracle_decode"):
                 getattr(lib, f).restype = None
@@ -75,14 +77,23 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _kv_heads(H: int, kv) -> int:
+    """K/V head count of a K or V array (axis 2), which must divide the query head count H."""
+    Hk = kv.shape[2]
+    if Hk < 1 or H % Hk != 0:
+        raise ValueError(f"K/V heads ({Hk}) must divide query heads ({H})")
+    return Hk
+
+
 def oracle_fwd(q, k, v, W: int, scale: float | None = None):
     """Full forward. Returns (o [B,T,H,D] f64, lse [B,H,T] f64)."""
     (q, k, v), bf = _prep(q, k, v)
     B, T, H, D = q.shape
+    Hk = _kv_heads(H, k)
     scale = 1.0 / np.sqrt(D) if scale is None else scale
     o = np.empty((B, T, H, D), np.float64)
     lse = np.empty((B, H, T), np.float64)
-    _load().swa_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), bf, B, T, H, D, int(W), float(scale), _ptr(o), _ptr(lse))
+    _load().swa_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), bf, B, T, H, Hk, D, int(W), float(scale), _ptr(o), _ptr(lse))
     return o, lse
 
 
@@ -95,20 +106,21 @@ def oracle_fwd_rows(q, k, v, W: int, rows, scale: float | None = None):
     n = idx.shape[0]
     o = np.empty((n, D), np.float64)
     lse = np.empty((n,), np.float64)
-    _load().swa_oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), bf, B, T, H, D, int(W), float(scale),
+    _load().swa_oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), bf, B, T, H, _kv_heads(H, k), D, int(W), float(scale),
                                 n, _ptr(idx), _ptr(o), _ptr(lse))
     return o, lse
 
 
 def oracle_bwd(q, k, v, do, W: int, scale: float | None = None):
-    """Full backward. Returns (dq, dk, dv), each [B,T,H,D] f64."""
+    """Full backward. Returns (dq [B,T,H,D], dk [B,T,Hk,D], dv [B,T,Hk,D]) f64."""
     (q, k, v, do), bf = _prep(q, k, v, do)
     B, T, H, D = q.shape
+    Hk = _kv_heads(H, k)
     scale = 1.0 / np.sqrt(D) if scale is None else scale
     dq = np.empty((B, T, H, D), np.float64)
-    dk = np.empty_like(dq)
-    dv = np.empty_like(dq)
-    _load().swa_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), bf, B, T, H, D, int(W), float(scale),
+    dk = np.empty((B, T, Hk, D), np.float64)
+    dv = np.empty_like(dk)
+    _load().swa_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), bf, B, T, H, Hk, D, int(W), float(scale),
                            _ptr(dq), _ptr(dk), _ptr(dv))
     return dq, dk, dv
 
@@ -120,28 +132,32 @@ def oracle_dq_rows(q, k, v, do, W: int, rows, scale: float | None = None):
     scale = 1.0 / np.sqrt(D) if scale is None else scale
     idx = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     dq = np.empty((idx.shape[0], D), np.float64)
-    _load().swa_oracle_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), bf, B, T, H, D, int(W), float(scale),
+    _load().swa_oracle_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), bf, B, T, H, _kv_heads(H, k), D, int(W),
+                               float(scale),
                                idx.shape[0], _ptr(idx), _ptr(dq))
     return dq
 
 
 def oracle_dkv_rows(q, k, v, do, W: int, rows, scale: float | None = None):
-    """dK, dV on selected key rows (b, h, j). Returns (dk [n,D], dv [n,D]) f64."""
+    """dK, dV on selected key rows (b, hk, j), hk a K/V head. Returns (dk [n,D], dv [n,D]) f64."""
     (q, k, v, do), bf = _prep(q, k, v, do)
     B, T, H, D = q.shape
     scale = 1.0 / np.sqrt(D) if scale is None else scale
     idx = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     dk = np.empty((idx.shape[0], D), np.float64)
     dv = np.empty_like(dk)
-    _load().swa_oracle_dkv_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), bf, B, T, H, D, int(W), float(scale),
+    _load().swa_oracle_dkv_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), bf, B, T, H, _kv_heads(H, k), D, int(W),
+                                float(scale),
                                 idx.shape[0], _ptr(idx), _ptr(dk), _ptr(dv))
     return dk, dv
 
 
 def oracle_decode(q, k_cache, v_cache, cache_len, W: int, scale: float | None = None):
-    """Decode. q [B,H,D], caches [B,cap,H,D], cache_len [B] int. Returns (o [B,H,D], lse [B,H]) f64."""
+    """Decode. q [B,H,D], caches [B,cap,Hk,D], cache_len [B] int. Returns (o [B,H,D], lse [B,H]) f64."""
     (q, k_cache, v_cache), bf = _prep(q, k_cache, v_cache)
-    B, cap, H, D = k_cache.shape
+    B, H, D = q.shape
+    cap = k_cache.shape[1]
+    Hk = _kv_heads(H, k_cache)
     scale = 1.0 / np.sqrt(D) if scale is None else scale
     cl = np.ascontiguousarray(np.asarray(cache_len, dtype=np.int32))
     if cl.shape != (B,) or cl.min(initial=1) < 1 or cl.max(initial=1) > cap:
@@ -149,5 +165,5 @@ def oracle_decode(q, k_cache, v_cache, cache_len, W: int, scale: float | None = 
     o = np.empty((B, H, D), np.float64)
     lse = np.empty((B, H), np.float64)
     _load().swa_oracle_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), bf, cl.ctypes.data_as(ctypes.c_void_p),
-                              B, cap, H, D, int(W), float(scale), _ptr(o), _ptr(lse))
+                              B, cap, H, Hk, D, int(W), float(scale), _ptr(o), _ptr(lse))
     return o, lse

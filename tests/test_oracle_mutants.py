@@ -23,10 +23,13 @@ MUTANTS = {
     "window_edge_off_by_one": ("long lo = i - W + 1;", "long lo = i - W;"),
     "dq_scale_dropped": ("dq[at4(T, H, D, b, i, h, d)] += scale * ds *", "dq[at4(T, H, D, b, i, h, d)] += ds *"),
     "delta_sign_flipped": ("double ds = pij * (dp - delta);", "double ds = pij * (dp + delta);"),
-    "dk_uses_k_not_q": ("dk[at4(T, H, D, b, j, h, d)] += scale * ds * ld(q,",
-                        "dk[at4(T, H, D, b, j, h, d)] += scale * ds * ld(k,"),
-    "dv_uses_key_row_of_dO": ("dv[at4(T, H, D, b, j, h, d)] += pij * ld(dout, in_bf16, at4(T, H, D, b, i, h, d));",
-                              "dv[at4(T, H, D, b, j, h, d)] += pij * ld(dout, in_bf16, at4(T, H, D, b, j, h, d));"),
+    "dk_uses_k_not_q": ("dk[at4(T, Hk, D, b, j, hk, d)] += scale * ds * ld(q,",
+                        "dk[at4(T, Hk, D, b, j, hk, d)] += scale * ds * ld(k,"),
+    "dv_uses_key_row_of_dO": ("dv[at4(T, Hk, D, b, j, hk, d)] += pij * ld(dout, in_bf16, at4(T, H, D, b, i, h, d));",
+                              "dv[at4(T, Hk, D, b, j, hk, d)] += pij * ld(dout, in_bf16, at4(T, H, D, b, j, h, d));"),
+    "kv_head_map_modulo": ("long hk = h / (H / Hk);", "long hk = h % Hk;"),
+    "kv_group_sums_one_head": ("for (long h = hk * G; h < (hk + 1) * G; ++h) {\n                for (long i = 0;",
+                               "for (long h = hk * G; h < hk * G + 1; ++h) {\n                for (long i = 0;"),
     "lse_log2": ("*lse_i = m + log(l);", "*lse_i = m + log2(l);"),
     "softmax_not_normalised": ("for (long c = 0; c < n; ++c) p[c] /= l;", ""),
     "decode_window_short_by_one": ("long lo = L - W;", "long lo = L - W + 1;"),
@@ -51,6 +54,15 @@ def _pins_pass() -> bool:
         for got, name in ((o, "o"), (lse, "lse"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
             if not np.allclose(got, ref[name], rtol=0, atol=1e-10):
                 return False
+    # grouped K/V heads: 4 query heads on 2 K/V heads
+    x = inputs.attention_inputs(1, 30, 4, 8, seed=61)
+    k2, v2 = (np.ascontiguousarray(x[n][:, :, :2]) for n in ("k", "v"))
+    o, lse = so.oracle_fwd(x["q"], k2, v2, 7)
+    dq, dk, dv = so.oracle_bwd(x["q"], k2, v2, x["do"], 7)
+    ref = torch_reference(f64(x["q"]), f64(k2), f64(v2), 7, x["scale"], do=f64(x["do"]))
+    for got, name in ((o, "o"), (lse, "lse"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if not np.allclose(got, ref[name], rtol=0, atol=1e-10):
+            return False
     import torch
 
     x = inputs.decode_inputs(3, 30, 2, 16, seed=4, cache_len=np.array([1, 17, 30]))

@@ -24,12 +24,16 @@ def band_mask(T, W):
 
 
 def torch_reference(q, k, v, W, scale, do=None):
-    """PyTorch fp64 SDPA with an explicit boolean band mask; q.. are [B,T,H,D] float64 numpy."""
+    """PyTorch fp64 SDPA with an explicit boolean band mask; q is [B,T,H,D], k, v [B,T,Hk,D] float64
+    numpy.  With Hk < H each K/V head is repeated for its H/Hk consecutive query heads inside
+    autograd, so the K/V gradients come out summed over each group."""
     tq, tk, tv = (torch.tensor(x).permute(0, 2, 1, 3).contiguous().requires_grad_(do is not None)
                   for x in (q, k, v))
+    G = q.shape[2] // k.shape[2]
+    ek, ev = (t.repeat_interleave(G, dim=1) for t in (tk, tv))
     mask = torch.tensor(band_mask(q.shape[1], W))
-    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
-    scores = (tq @ tk.transpose(-1, -2)) * scale
+    o = torch.nn.functional.scaled_dot_product_attention(tq, ek, ev, attn_mask=mask, scale=scale)
+    scores = (tq @ ek.transpose(-1, -2)) * scale
     lse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1)
     out = {"o": o.detach().permute(0, 2, 1, 3).numpy(), "lse": lse.detach().numpy()}
     if do is not None:
@@ -248,3 +252,80 @@ def test_input_generator_is_deterministic_and_normal():
     np.testing.assert_allclose(rms, 1.5, rtol=5e-3)
     lens = inputs.uniform_int(3, "cache_len", 10000, 1, 2048)
     assert lens.min() >= 1 and lens.max() <= 2048 and abs(lens.mean() - 1024.5) < 30
+
+
+GQA_CASES = [
+    # (B, T, H, Hk, D, W): grouped K/V heads (the GPT config's n_kv_head)
+    (1, 40, 4, 2, 16, 9),
+    (2, 33, 6, 1, 8, 10 ** 9),   # one K/V head for all query heads
+    (1, 70, 8, 4, 16, 25),
+]
+
+
+def gqa_inputs(B, T, H, Hk, D, seed):
+    """Attention inputs whose K / V keep only their first Hk heads."""
+    x = inputs.attention_inputs(B, T, H, D, seed=seed)
+    x["k"] = np.ascontiguousarray(x["k"][:, :, :Hk])
+    x["v"] = np.ascontiguousarray(x["v"][:, :, :Hk])
+    return x
+
+
+@pytest.mark.parametrize("B,T,H,Hk,D,W", GQA_CASES)
+def test_grouped_kv_heads_match_torch(B, T, H, Hk, D, W):
+    x = gqa_inputs(B, T, H, Hk, D, seed=300 + T)
+    o, lse = oracle_fwd(x["q"], x["k"], x["v"], W)
+    dq, dk, dv = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    ref = torch_reference(f64(x["q"]), f64(x["k"]), f64(x["v"]), W, x["scale"], do=f64(x["do"]))
+    assert dk.shape == (B, T, Hk, D) and dv.shape == (B, T, Hk, D)
+    for got, name in ((o, "o"), (lse, "lse"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        np.testing.assert_allclose(got, ref[name], rtol=0, atol=1e-11, err_msg=name)
+
+
+def test_grouped_kv_heads_reduce_to_repeated_heads():
+    """Grouped K/V equals multi-head attention on K/V repeated per group; dK/dV of a K/V head is the
+    sum of the repeated heads' gradients."""
+    B, T, H, Hk, D, W = 1, 48, 6, 2, 16, 13
+    x = gqa_inputs(B, T, H, Hk, D, seed=91)
+    kr, vr = (np.ascontiguousarray(np.repeat(x[n], H // Hk, axis=2)) for n in ("k", "v"))
+    o_g, lse_g = oracle_fwd(x["q"], x["k"], x["v"], W)
+    o_m, lse_m = oracle_fwd(x["q"], kr, vr, W)
+    np.testing.assert_array_equal(o_g, o_m)
+    np.testing.assert_array_equal(lse_g, lse_m)
+    dq_g, dk_g, dv_g = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    dq_m, dk_m, dv_m = oracle_bwd(x["q"], kr, vr, x["do"], W)
+    np.testing.assert_array_equal(dq_g, dq_m)
+    np.testing.assert_allclose(dk_g, dk_m.reshape(B, T, Hk, H // Hk, D).sum(axis=3), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv_g, dv_m.reshape(B, T, Hk, H // Hk, D).sum(axis=3), rtol=0, atol=1e-12)
+
+
+def test_grouped_kv_rows_and_decode():
+    B, T, H, Hk, D, W = 2, 45, 4, 2, 16, 11
+    x = gqa_inputs(B, T, H, Hk, D, seed=17)
+    o, lse = oracle_fwd(x["q"], x["k"], x["v"], W)
+    dq, dk, dv = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    rows = np.array([[0, 0, 0], [1, 3, 44], [0, 1, 10], [1, 2, 11]])
+    o_r, lse_r = oracle_fwd_rows(x["q"], x["k"], x["v"], W, rows)
+    np.testing.assert_allclose(o_r, o[rows[:, 0], rows[:, 2], rows[:, 1]], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse_r, lse[rows[:, 0], rows[:, 1], rows[:, 2]], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(oracle_dq_rows(x["q"], x["k"], x["v"], x["do"], W, rows),
+                               dq[rows[:, 0], rows[:, 2], rows[:, 1]], rtol=0, atol=1e-12)
+    krows = np.array([[0, 0, 0], [1, 1, 44], [0, 1, 20], [1, 0, 33]])   # (b, K/V head, key)
+    dk_r, dv_r = oracle_dkv_rows(x["q"], x["k"], x["v"], x["do"], W, krows)
+    np.testing.assert_allclose(dk_r, dk[krows[:, 0], krows[:, 2], krows[:, 1]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv_r, dv[krows[:, 0], krows[:, 2], krows[:, 1]], rtol=0, atol=1e-12)
+    # decode of the last row equals forward row L-1 for every query head of each group
+    cache_len = np.array([T, 20])
+    q_dec = np.ascontiguousarray(np.stack([x["q"][b, cache_len[b] - 1] for b in range(B)]))
+    od, ld_ = oracle_decode(q_dec, x["k"], x["v"], cache_len, W)
+    for b in range(B):
+        L = int(cache_len[b])
+        sub_o, sub_lse = oracle_fwd(x["q"][b:b + 1, :L], x["k"][b:b + 1, :L], x["v"][b:b + 1, :L], W)
+        np.testing.assert_allclose(od[b], sub_o[0, L - 1], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(ld_[b], sub_lse[0, :, L - 1], rtol=0, atol=1e-13)
+
+
+def test_grouped_kv_heads_must_divide():
+    x = inputs.attention_inputs(1, 8, 3, 8, seed=1)
+    with pytest.raises(ValueError):
+        oracle_fwd(x["q"], x["k"][:, :, :2].copy(), x["v"][:, :, :2].copy(), 4)
+
