@@ -40,11 +40,12 @@ struct BwdParams {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     int B, T, H;
+    int G;                // query heads per K/V head (k, v, dk, dv have H / G heads)
     long long W;
     float scale;
     float scale_log2;
     int n_blk;            // ceil(T / 128)
-    int n_items;          // n_blk * B * H
+    int n_items;          // items of this launch: n_blk * B * H (dQ) or n_blk * B * H / G (dK/dV)
     int work_slot;        // index into g_work_slots for this launch
     int Tp;               // T rounded up to 128
     long long wait_limit;
@@ -153,23 +154,34 @@ struct BwdKVCfg {
 
 // Item of the key-stationary kernel: key block kblk of head (b, h); head-major, lowest key
 // blocks (the most query tiles under causal masking) first.
+// With grouped K/V heads an item is a key tile of one K/V head, and its steps walk the band's
+// query tiles for each query head of the group in turn (dK, dV sum over the group).
 struct BwdKVItem {
-    int b, h, bh;
+    int b, h;             // batch, K/V head
     long long k0;         // first key row
-    int ilo, nsteps;      // first query tile and number of query tiles in the band
+    int ilo, nband;       // first query tile and number of query tiles in the band
+    int nsteps;           // nband * G
 };
 
 __device__ __forceinline__ BwdKVItem bwd_kv_item(const BwdParams& p, int item) {
     BwdKVItem it;
     const int kblk = item % p.n_blk;
-    it.bh = item / p.n_blk;
-    it.b = it.bh / p.H;
-    it.h = it.bh % p.H;
+    const int bhk = item / p.n_blk;
+    const int Hk = p.H / p.G;
+    it.b = bhk / Hk;
+    it.h = bhk % Hk;
     it.k0 = (long long)kblk * 128;
     it.ilo = kblk;
     const int ihi = int(imin_ll(p.T - 1, it.k0 + 127 + p.W - 1) / 128);
-    it.nsteps = ihi - it.ilo + 1;
+    it.nband = ihi - it.ilo + 1;
+    it.nsteps = it.nband * p.G;
     return it;
+}
+
+// Query head and query tile of step l of a key-stationary item.
+__device__ __forceinline__ void bwd_kv_step(const BwdParams& p, const BwdKVItem& g, int l, int& qh, int& qt) {
+    qh = g.h * p.G + l / g.nband;
+    qt = g.ilo + l % g.nband;
 }
 
 // Per step n (one query tile of the item):
@@ -293,13 +305,15 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             tma_load_4d(sK + x * C::BOX, &tm_k, k_full, x * 64, g.h, int(g.k0), g.b);
                         ++nk;
                     }
-                    const int qrow = (g.ilo + l) * C::BM;
+                    int qh, qt;
+                    bwd_kv_step(p, g, l, qh, qt);
+                    const int qrow = qt * C::BM;
                     if (!(ok = mbar_wait(q_empty(n), ((n / C::NQ) & 1) ^ 1u, abort_flag, p.wait_limit,
                                          kStatusTimeoutProducer)))
                         break;
                     mbar_arrive_expect_tx(q_full(n), C::TILE);
                     for (int x = 0; x < C::NBOX; ++x)
-                        tma_load_4d(sQ(n) + x * C::BOX, &tm_q, q_full(n), x * 64, g.h, qrow, g.b);
+                        tma_load_4d(sQ(n) + x * C::BOX, &tm_q, q_full(n), x * 64, qh, qrow, g.b);
                     ++nq;
                     if (l == 0) {   // V of the previous item is free once its last dP completed
                         if (ki > 0 && !(ok = mbar_wait(v_empty, uint32_t((ki - 1) & 1), abort_flag, p.wait_limit,
@@ -315,8 +329,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         break;
                     mbar_arrive_expect_tx(do_full(n), C::TILE + 1024);
                     for (int x = 0; x < C::NBOX; ++x)
-                        tma_load_4d(sDO(n) + x * C::BOX, &tm_do, do_full(n), x * 64, g.h, qrow, g.b);
-                    const size_t row = size_t(g.bh) * p.Tp + size_t(qrow);
+                        tma_load_4d(sDO(n) + x * C::BOX, &tm_do, do_full(n), x * 64, qh, qrow, g.b);
+                    const size_t row = (size_t(g.b) * p.H + size_t(qh)) * p.Tp + size_t(qrow);
                     bulk_load(sLSE(n), p.lse2 + row, 512, do_full(n));
                     bulk_load(sLSE(n) + 512, p.delta + row, 512, do_full(n));
                     ++n;
@@ -420,7 +434,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const BwdKVItem pg = bwd_kv_item(p, pitem);
             const long long pkv = pg.k0 + row;
             __nv_bfloat16* dst =
-                pkv < T ? (rh == 0 ? p.dv : p.dk) + ((size_t(pg.b) * T + size_t(pkv)) * p.H + pg.h) * D : nullptr;
+                pkv < T ? (rh == 0 ? p.dv : p.dk) + ((size_t(pg.b) * T + size_t(pkv)) * (p.H / p.G) + pg.h) * D
+                        : nullptr;
             const uint32_t src = (rh == 0 ? tDV : tDK) + lane_off;
             const float mul = rh == 0 ? 1.f : p.scale;
 #pragma unroll
@@ -454,7 +469,9 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const long long kv = k0 + row;
             for (int l = 0; l < g.nsteps && ok; ++l, ++n) {
                 const uint32_t par = uint32_t(n & 1);
-                const long long q0 = (long long)(g.ilo + l) * C::BM;
+                int qh, qt;
+                bwd_kv_step(p, g, l, qh, qt);
+                const long long q0 = (long long)qt * C::BM;
                 const uint32_t sL = sLSE(n) + rh * 256;   // this half's 64 lse2 values
                 // The previous item's dV / dK leave TMEM before this item's first dV.
                 if (l == 0 && prev_ki >= 0) {
@@ -603,7 +620,7 @@ struct BwdQCfg {
 // Item of the query-stationary kernel: query tile qt of head (b, h); head-major, latest
 // query tiles (the most key tiles under causal masking) first.
 struct BwdQItem {
-    int b, h, bh;
+    int b, h, bh, hk;     // batch, query head, b*H + h, K/V head
     long long q0;         // first query row
     int jlo, jhi;         // key tiles of the band
 };
@@ -614,6 +631,7 @@ __device__ __forceinline__ BwdQItem bwd_q_item(const BwdParams& p, int item) {
     it.bh = item / p.n_blk;
     it.b = it.bh / p.H;
     it.h = it.bh % p.H;
+    it.hk = it.h / p.G;
     it.q0 = (long long)qt * 128;
     it.jlo = int(imax_ll(0, it.q0 - p.W + 1) / 128);
     it.jhi = qt;
@@ -738,7 +756,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     if (!(ok = wait_p(k_empty(n), n / C::NK + 1))) break;   // first pass: the phase before 0
                     mbar_arrive_expect_tx(k_full(n), C::TILE);
-                    for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sK(n) + x * C::BOX, &tm_k, k_full(n), x * 64, g.h, j * C::BN, g.b);
+                    for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sK(n) + x * C::BOX, &tm_k, k_full(n), x * 64, g.hk, j * C::BN, g.b);
                     ++nk;
                     if (j == g.jlo) {
                         if (qi > 0 && !(ok = wait_p(do_empty, qi - 1))) break;
@@ -748,7 +766,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     if (!(ok = wait_p(v_empty(n), n / C::NV + 1))) break;
                     mbar_arrive_expect_tx(v_full(n), C::TILE);
-                    for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sV(n) + x * C::BOX, &tm_v, v_full(n), x * 64, g.h, j * C::BN, g.b);
+                    for (int x = 0; x < C::NBOX; ++x) tma_load_4d(sV(n) + x * C::BOX, &tm_v, v_full(n), x * 64, g.hk, j * C::BN, g.b);
                     ++nv;
                 }
                 if (!ok) break;

@@ -29,7 +29,7 @@ constexpr int kDecodeUnroll = 4;   // slots per batch (two batches in flight per
 
 struct DecParams {
     const __nv_bfloat16* q;        // [B,H,D]
-    const __nv_bfloat16* kc;       // [B,cap,H,D]
+    const __nv_bfloat16* kc;       // [B,cap,Hk,D], Hk = H / kv_group
     const __nv_bfloat16* vc;
     const int32_t* cache_len;      // [B]
     __nv_bfloat16* o;              // [B,H,D]
@@ -38,6 +38,7 @@ struct DecParams {
     float* part_ml;                // [B, nsplit_max, H, 2]
     float* part_o;                 // [B, nsplit_max, H, D]
     int B, cap, H;
+    int kv_group;                  // query heads per K/V head: query head h reads cache head h / kv_group
     long long W;
     float scale_log2;
     int nsplit;                    // splits launched per sequence
@@ -89,9 +90,10 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
-    const size_t row_elems = size_t(H) * D;
-    const __nv_bfloat16* kb = p.kc + size_t(b) * p.cap * row_elems + size_t(h) * D + c * 8;
-    const __nv_bfloat16* vb = p.vc + size_t(b) * p.cap * row_elems + size_t(h) * D + c * 8;
+    const size_t row_elems = size_t(H / p.kv_group) * D;   // one cache slot: all K/V heads
+    const int hk = h / p.kv_group;
+    const __nv_bfloat16* kb = p.kc + size_t(b) * p.cap * row_elems + size_t(hk) * D + c * 8;
+    const __nv_bfloat16* vb = p.vc + size_t(b) * p.cap * row_elems + size_t(hk) * D + c * 8;
 
     // Two batches of kDecodeUnroll slots are in flight: the next batch's loads are issued
     // before the current batch is consumed.

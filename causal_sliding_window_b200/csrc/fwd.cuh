@@ -61,6 +61,7 @@ struct FwdParams {
     __nv_bfloat16* o;
     float* lse;
     int B, T, H;
+    int G;                // query heads per K/V head (K, V have H / G heads)
     long long W;
     float scale_log2;     // softmax scale * log2(e)
     int n_qblk;           // ceil(T / 256)
@@ -71,7 +72,7 @@ struct FwdParams {
 
 // Geometry of one work item: query block qblk of head (b, h).
 struct FwdItem {
-    int b, h;
+    int b, h, hk;         // batch, query head, K/V head
     long long q0;         // first query row of tile 0 (tile 1 starts 128 rows later)
     bool valid1;          // tile 1 has rows below T
     int jlo0, jhi0, jlo1, jhi1, jbeg, jend;
@@ -86,6 +87,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
     const int qblk = p.n_qblk - 1 - item % p.n_qblk;
     it.b = bh / p.H;
     it.h = bh % p.H;
+    it.hk = it.h / p.G;
     it.q0 = (long long)qblk * 256;
     it.valid1 = it.q0 + 128 < p.T;
     it.jlo0 = int(imax_ll(0, it.q0 - p.W + 1) / 128);
@@ -202,7 +204,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         mbar_arrive_expect_tx(kv_full(s), C::TILE);
                         const CUtensorMap* m = kv ? &tm_v : &tm_k;
                         for (int x = 0; x < C::NBOX; ++x)
-                            tma_load_4d(sKV + s * C::TILE + x * C::BOX, m, kv_full(s), x * 64, g.h, j * C::BN, g.b);
+                            tma_load_4d(sKV + s * C::TILE + x * C::BOX, m, kv_full(s), x * 64, g.hk, j * C::BN, g.b);
                     }
                 }
             }

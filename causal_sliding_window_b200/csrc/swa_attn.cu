@@ -93,6 +93,9 @@ bool valid_common(int B, int T, int H, int D, int W, float scale) {
     return true;
 }
 
+// Grouped K/V heads: Hkv >= 1 and divides H.
+bool valid_kv_heads(int H, int Hkv) { return Hkv >= 1 && H >= 1 && H % Hkv == 0; }
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Optional events recorded between the three launches of attn_bwd (see
@@ -154,19 +157,20 @@ void* noalloc_scratch() {
 
 extern "C" {
 
-int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B, int T,
-             int H, int D, int W, float scale, void* stream) {
+int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B,
+                 int T, int H, int Hkv, int D, int W, float scale, void* stream) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_INVALID_ARG;
-    if (!valid_common(B, T, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     const int n_qblk = (T + 255) / 256;
     const long long n_items = (long long)n_qblk * B * H;
     if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
     CUtensorMap mq, mk, mv;
-    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, H, D) || !make_bthd_map(&mv, v, B, T, H, D))
+    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, Hkv, D) ||
+        !make_bthd_map(&mv, v, B, T, Hkv, D))
         return ATTN_ERR_LAUNCH;
     FwdParams p;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
@@ -174,6 +178,7 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     p.B = B;
     p.T = T;
     p.H = H;
+    p.G = H / Hkv;
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_qblk = n_qblk;
@@ -191,6 +196,11 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     return launch_status();
 }
 
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B, int T,
+             int H, int D, int W, float scale, void* stream) {
+    return attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, W, scale, stream);
+}
+
 // Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128).
 size_t attn_bwd_workspace_bytes(int B, int T, int H, int D) {
     if (B < 1 || T < 1 || H < 1 || D < 1) return 0;
@@ -198,15 +208,15 @@ size_t attn_bwd_workspace_bytes(int B, int T, int H, int D) {
     return 2 * align256(size_t(B) * H * Tp * 4);
 }
 
-int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
-             const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace, size_t ws_bytes,
-             int B, int T, int H, int D, int W, float scale, void* stream) {
+int attn_bwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
+                 const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace,
+                 size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, void* stream) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
     for (const void* ptr : ptrs)
         if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
-    if (!valid_common(B, T, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_bwd_workspace_bytes(B, T, H, D)) return ATTN_ERR_WORKSPACE;
     const int n_blk = (T + 127) / 128;
@@ -214,8 +224,8 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
     CUtensorMap mq, mk, mv, mdo;
-    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, H, D) ||
-        !make_bthd_map(&mv, v, B, T, H, D) || !make_bthd_map(&mdo, dout, B, T, H, D))
+    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, Hkv, D) ||
+        !make_bthd_map(&mv, v, B, T, Hkv, D) || !make_bthd_map(&mdo, dout, B, T, H, D))
         return ATTN_ERR_LAUNCH;
     const int Tp = (T + 127) / 128 * 128;
     const size_t row_bytes = align256(size_t(B) * H * Tp * 4);
@@ -241,6 +251,7 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     p.B = B;
     p.T = T;
     p.H = H;
+    p.G = H / Hkv;
     p.W = W;
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
@@ -248,17 +259,22 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     p.n_items = int(n_items);
     p.Tp = Tp;
     p.wait_limit = kDefaultWaitLimit;
-    // dK, dV (key-stationary), then dQ (query-stationary); each launch draws from its own counter.
+    // dK, dV (key-stationary, one item per key tile of a K/V head), then dQ (query-stationary, one
+    // item per query tile of a query head); each launch draws from its own counter.
+    const long long n_items_kv = (long long)n_blk * B * Hkv;
+    const long long grid_kv = n_items_kv < sm_count() ? n_items_kv : sm_count();
+    p.n_items = int(n_items_kv);
     p.work_slot = next_work_slot();
     if (D == 128) {
         if (!ensure_smem((const void*)swa_bwd_dkdv_kernel<128>, BwdKVCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_dkdv_kernel<128><<<unsigned(grid), BwdKVCfg<128>::THREADS, BwdKVCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
+        swa_bwd_dkdv_kernel<128><<<unsigned(grid_kv), BwdKVCfg<128>::THREADS, BwdKVCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
     } else {
         if (!ensure_smem((const void*)swa_bwd_dkdv_kernel<64>, BwdKVCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_dkdv_kernel<64><<<unsigned(grid), BwdKVCfg<64>::THREADS, BwdKVCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
+        swa_bwd_dkdv_kernel<64><<<unsigned(grid_kv), BwdKVCfg<64>::THREADS, BwdKVCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
     }
     if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
     if (g_ev_after_main) cudaEventRecord(g_ev_after_main, s);
+    p.n_items = int(n_items);
     p.work_slot = next_work_slot();
     if (D == 128) {
         if (!ensure_smem((const void*)swa_bwd_dq_kernel<128>, BwdQCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
@@ -270,6 +286,12 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     return launch_status();
 }
 
+int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
+             const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace, size_t ws_bytes,
+             int B, int T, int H, int D, int W, float scale, void* stream) {
+    return attn_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, H, D, W, scale, stream);
+}
+
 size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
     if (B < 1 || cap < 1 || H < 1 || (D != 64 && D != 128)) return 0;
     const size_t nsm = size_t((cap + kDecodeChunk - 1) / kDecodeChunk);
@@ -278,15 +300,15 @@ size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
            align256(size_t(B) * nsm * H * D * 4);
 }
 
-int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache, const int32_t* cache_len,
-                attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B, int cap, int H, int D, int W,
-                float scale, void* stream) {
+int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                    const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                    int cap, int H, int Hkv, int D, int W, float scale, void* stream) {
     if (!q || !k_cache || !v_cache || !cache_len || !o || !workspace) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
-    if (!valid_common(B, cap, H, D, W, scale)) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, cap, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_decode_workspace_bytes(B, cap, H, D)) return ATTN_ERR_WORKSPACE;
@@ -310,6 +332,7 @@ int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v
     p.B = B;
     p.cap = cap;
     p.H = H;
+    p.kv_group = H / Hkv;
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.nsplit = (span + kDecodeChunk - 1) / kDecodeChunk;
@@ -322,6 +345,13 @@ int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v
     else
         swa_decode_kernel<64><<<grid, threads, 0, s>>>(p);
     return launch_status();
+}
+
+int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache, const int32_t* cache_len,
+                attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B, int cap, int H, int D, int W,
+                float scale, void* stream) {
+    return attn_decode_gqa(q, k_cache, v_cache, cache_len, o, lse, workspace, ws_bytes, B, cap, H, H, D, W, scale,
+                           stream);
 }
 
 int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,

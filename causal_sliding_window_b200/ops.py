@@ -9,6 +9,8 @@ Low-level calls (caller provides every buffer, torch tensors on one CUDA device)
   attn_fwd(q, k, v, o, lse, W, scale=None, stream=None)
   attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, W, scale=None, stream=None)
   attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W, scale=None, stream=None)
+K and V (and dK, dV, the caches) may have fewer heads than Q (grouped K/V heads, Hkv dividing H);
+the calls then go to the C entry points' _gqa forms.
 Convenience wrappers that allocate outputs: forward, backward, decode.
 """
 from __future__ import annotations
@@ -41,6 +43,12 @@ _lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
 _lib.attn_decode_workspace_bytes.restype = _sz
 _lib.attn_decode.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode.restype = _i
+_lib.attn_fwd_gqa.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_fwd_gqa.restype = _i
+_lib.attn_bwd_gqa.argtypes = [_p] * 10 + [_sz, _i, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_bwd_gqa.restype = _i
+_lib.attn_decode_gqa.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_decode_gqa.restype = _i
 _lib.attn_decode_noalloc.argtypes = [_p] * 6 + [_i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode_noalloc.restype = _i
 _lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
@@ -52,8 +60,8 @@ _lib.attn_selftest_wait_timeout.restype = _i
 _lib.attn_status_string.argtypes = [_i]
 _lib.attn_status_string.restype = ctypes.c_char_p
 
-EXPORTED = ["attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_decode_workspace_bytes", "attn_decode",
-            "attn_decode_noalloc", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
+EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_gqa",
+            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
             "attn_status_string"]
 
 
@@ -88,16 +96,30 @@ def _bthd(*ts):
     return shape
 
 
+def _kv_heads(qshape, *kv):
+    """K/V tensors share one [B, T, Hkv, D] shape, with B, T, D of q and Hkv dividing q's H."""
+    kshape = _bthd(*kv)
+    B, T, H, D = qshape
+    if kshape[0] != B or kshape[1] != T or kshape[3] != D or kshape[2] < 1 or H % kshape[2] != 0:
+        raise ValueError("K/V must be [B, T, Hkv, D] with Hkv dividing the query heads")
+    return kshape[2]
+
+
 def _scale(scale, D):
     return 1.0 / math.sqrt(D) if scale is None else float(scale)
 
 
 def attn_fwd(q, k, v, o, lse, W: int, scale=None, stream=None):
-    B, T, H, D = _bthd(q, k, v, o)
+    B, T, H, D = _bthd(q, o)
+    Hkv = _kv_heads((B, T, H, D), k, v)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 [B, H, T] tensor")
-    _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, H, D, int(W), _scale(scale, D),
-                         _stream(stream)), "attn_fwd")
+    if Hkv == H:
+        _check(_lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, H, D, int(W), _scale(scale, D),
+                             _stream(stream)), "attn_fwd")
+    else:
+        _check(_lib.attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, H, Hkv, D, int(W),
+                                 _scale(scale, D), _stream(stream)), "attn_fwd_gqa")
 
 
 def attn_bwd_workspace_bytes(B: int, T: int, H: int, D: int) -> int:
@@ -105,13 +127,17 @@ def attn_bwd_workspace_bytes(B: int, T: int, H: int, D: int) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, W: int, scale=None, stream=None):
-    B, T, H, D = _bthd(q, k, v, o, dout, dq, dk, dv)
+    B, T, H, D = _bthd(q, o, dout, dq)
+    Hkv = _kv_heads((B, T, H, D), k, v, dk, dv)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T):
         raise ValueError("lse must be float32 [B, H, T]")
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(_lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                         _ptr(workspace), ws_bytes, B, T, H, D, int(W), _scale(scale, D), _stream(stream)),
-           "attn_bwd")
+    ptrs = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace))
+    if Hkv == H:
+        _check(_lib.attn_bwd(*ptrs, ws_bytes, B, T, H, D, int(W), _scale(scale, D), _stream(stream)), "attn_bwd")
+    else:
+        _check(_lib.attn_bwd_gqa(*ptrs, ws_bytes, B, T, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)),
+               "attn_bwd_gqa")
 
 
 def attn_decode_workspace_bytes(B: int, cap: int, H: int, D: int) -> int:
@@ -119,15 +145,21 @@ def attn_decode_workspace_bytes(B: int, cap: int, H: int, D: int) -> int:
 
 
 def attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W: int, scale=None, stream=None):
-    B, cap, H, D = _bthd(k_cache, v_cache)
-    if tuple(q.shape) != (B, H, D) or tuple(o.shape) != (B, H, D) or q.dtype != torch.bfloat16:
-        raise ValueError("q and o must be bf16 [B, H, D]")
+    B, cap, Hkv, D = _bthd(k_cache, v_cache)
+    H = q.shape[1] if q.dim() == 3 else -1
+    if (tuple(q.shape) != (B, H, D) or tuple(o.shape) != (B, H, D) or q.dtype != torch.bfloat16
+            or H % Hkv != 0):
+        raise ValueError("q and o must be bf16 [B, H, D] with the caches' head count dividing H")
     if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or not cache_len.is_cuda:
         raise ValueError("cache_len must be an int32 CUDA tensor of shape [B]")
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(_lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), _ptr(o), _ptr(lse),
-                            _ptr(workspace), ws_bytes, B, cap, H, D, int(W), _scale(scale, D), _stream(stream)),
-           "attn_decode")
+    ptrs = (_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), _ptr(o), _ptr(lse), _ptr(workspace))
+    if Hkv == H:
+        _check(_lib.attn_decode(*ptrs, ws_bytes, B, cap, H, D, int(W), _scale(scale, D), _stream(stream)),
+               "attn_decode")
+    else:
+        _check(_lib.attn_decode_gqa(*ptrs, ws_bytes, B, cap, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)),
+               "attn_decode_gqa")
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, cache_len, o, lse, W: int, scale=None, stream=None):
@@ -190,7 +222,8 @@ def decode_workspace(B: int, cap: int, H: int, D: int, device) -> torch.Tensor:
 
 
 def decode(q, k_cache, v_cache, cache_len, W: int, scale=None, stream=None, workspace=None):
-    B, cap, H, D = k_cache.shape
+    B, H, D = q.shape
+    cap = k_cache.shape[1]
     o = torch.empty((B, H, D), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     if workspace is None:

@@ -70,6 +70,16 @@ typedef enum {
 int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
              int B, int T, int H, int D, int W, float scale, void* stream);
 
+/*
+ * Grouped K/V heads (GQA / MQA): the GPT config's n_kv_head (apidog guide,
+ * section 1, "GPT model").  k and v are [B, T, Hkv, D] with Hkv >= 1 dividing H;
+ * query head h reads K/V head h / (H / Hkv), so H / Hkv consecutive query heads
+ * share one K/V head.  Everything else as attn_fwd; attn_fwd is this call with
+ * Hkv = H.  Hkv that does not divide H returns ATTN_ERR_INVALID_ARG.
+ */
+int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
+                 int B, int T, int H, int Hkv, int D, int W, float scale, void* stream);
+
 /* Bytes of workspace attn_bwd needs: fp32 rows of lse*log2(e) and Delta, [B*H, T rounded up
  * to 128] each (256-byte padded). */
 size_t attn_bwd_workspace_bytes(int B, int T, int H, int D);
@@ -93,6 +103,17 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
              void* workspace, size_t ws_bytes, int B, int T, int H, int D, int W, float scale,
              void* stream);
 
+/*
+ * Backward with grouped K/V heads: k, v, dk, dv are [B, T, Hkv, D]; dk and dv of a
+ * K/V head are the sums over its H / Hkv query heads.  The workspace is
+ * attn_bwd_workspace_bytes(B, T, H, D) (per query head).  attn_bwd is this call
+ * with Hkv = H.
+ */
+int attn_bwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o,
+                 const float* lse, const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv,
+                 void* workspace, size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W,
+                 float scale, void* stream);
+
 /* Bytes of workspace attn_decode needs for B sequences of capacity cap (any W); 0 for
  * sizes attn_decode rejects (B, cap or H below 1, D not 64 or 128). */
 size_t attn_decode_workspace_bytes(int B, int cap, int H, int D);
@@ -115,6 +136,15 @@ size_t attn_decode_workspace_bytes(int B, int cap, int H, int D);
 int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
                 const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes,
                 int B, int cap, int H, int D, int W, float scale, void* stream);
+
+/*
+ * Decode with grouped K/V heads: k_cache, v_cache are [B, cap, Hkv, D]; query head h
+ * reads cache head h / (H / Hkv).  Workspace as attn_decode (per query head).
+ * attn_decode is this call with Hkv = H.
+ */
+int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                    const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes,
+                    int B, int cap, int H, int Hkv, int D, int W, float scale, void* stream);
 
 /*
  * attn_decode without a caller-provided workspace, for callers that cannot

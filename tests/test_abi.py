@@ -119,3 +119,15 @@ def test_product_path_has_no_oracle_or_fallback():
                 assert "oracle" not in src.replace("oracle_", "").lower() or f == "inputs.py", f
     src = open(ops.__file__).read()
     assert "raise ImportError" in src
+
+
+def test_grouped_kv_heads_argument_checks():
+    # Hkv must be >= 1 and divide H (checked before any launch)
+    assert ops._lib.attn_fwd_gqa(A, A, A, A, A, 1, 16, 6, 4, 128, 4, 0.1, None) == ERR_INVALID
+    assert ops._lib.attn_fwd_gqa(A, A, A, A, A, 1, 16, 6, 0, 128, 4, 0.1, None) == ERR_INVALID
+    ws = ops.attn_bwd_workspace_bytes(1, 16, 6, 128)
+    assert ops._lib.attn_bwd_gqa(A, A, A, A, A, A, A, A, A, A, ws, 1, 16, 6, 5, 128, 4, 0.1, None) == ERR_INVALID
+    dws = ops.attn_decode_workspace_bytes(2, 64, 6, 128)
+    assert ops._lib.attn_decode_gqa(A, A, A, A, A, A, A, dws, 2, 64, 6, 4, 128, 8, 0.1, None) == ERR_INVALID
+    assert ops._lib.attn_fwd_gqa(A, A, A, A, A, 1, 16, 6, 2, 96, 4, 0.1, None) == ERR_UNSUPPORTED
+

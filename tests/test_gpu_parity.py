@@ -227,3 +227,64 @@ def test_bounded_wait_reports_timeout_without_hanging(ops):
     got = run_fwd_bwd(ops, x, 16, with_bwd=False)
     o, _ = oracle_fwd(x["q"], x["k"], x["v"], 16)
     assert rel_l2(got["o"], o) <= O_REL
+
+
+# ---------------------------------------------------------------------------
+# Grouped K/V heads (the GPT config's n_kv_head): K, V, dK, dV and the caches carry Hkv heads.
+# ---------------------------------------------------------------------------
+GQA_SMALL = [
+    # (B, T, H, Hkv, D, W)
+    (1, 333, 4, 2, 128, 100),
+    (2, 300, 6, 1, 64, 10 ** 9),    # one K/V head for all query heads
+    (1, 640, 8, 4, 128, 129),
+    (2, 257, 6, 3, 128, 1),
+]
+
+
+def grouped_inputs(B, T, H, Hkv, D, seed):
+    x = inputs.attention_inputs(B, T, H, D, seed=seed)
+    x["k"] = np.ascontiguousarray(x["k"][:, :, :Hkv])
+    x["v"] = np.ascontiguousarray(x["v"][:, :, :Hkv])
+    return x
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,W", GQA_SMALL)
+def test_grouped_kv_heads_match_oracle(ops, B, T, H, Hkv, D, W):
+    x = grouped_inputs(B, T, H, Hkv, D, seed=500 + T + H)
+    q, k, v, do = (dev_bf16(x[n]) for n in ("q", "k", "v", "do"))
+    o, lse = Guarded((B, T, H, D), torch.bfloat16), Guarded((B, H, T), torch.float32)
+    dq = Guarded((B, T, H, D), torch.bfloat16)
+    dk, dv = Guarded((B, T, Hkv, D), torch.bfloat16), Guarded((B, T, Hkv, D), torch.bfloat16)
+    ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device="cuda")
+    ops.attn_fwd(q, k, v, o.t, lse.t, W)
+    ops.attn_bwd(q, k, v, o.t, lse.t, do, dq.t, dk.t, dv.t, ws, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    for g in (o, lse, dq, dk, dv):
+        assert g.guards_intact(), "write outside an output buffer"
+    ro, rl = oracle_fwd(x["q"], x["k"], x["v"], W)
+    rdq, rdk, rdv = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    go, gl = host_f64(o.t), host_f64(lse.t)
+    assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
+    assert np.max(np.abs(gl - rl)) <= LSE_ABS
+    if W == 1:   # dQ = dK = 0 exactly (each row's only key is its own): bound the rounding residue
+        assert np.max(np.abs(host_f64(dq.t))) <= 1e-4 and np.max(np.abs(host_f64(dk.t))) <= 1e-4
+    else:
+        assert rel_l2(host_f64(dq.t), rdq) <= G_REL and rel_l2(host_f64(dk.t), rdk) <= G_REL
+    assert rel_l2(host_f64(dv.t), rdv) <= G_REL
+
+
+@pytest.mark.parametrize("H,Hkv", [(12, 4), (8, 1)])
+def test_grouped_kv_heads_decode(ops, H, Hkv):
+    B, cap, D, W = 5, 300, 128, 150
+    x = inputs.decode_inputs(B, cap, H, D, seed=H + Hkv, cache_len=np.array([1, 64, 149, 151, 300]))
+    kc = np.ascontiguousarray(x["k_cache"][:, :, :Hkv])
+    vc = np.ascontiguousarray(x["v_cache"][:, :, :Hkv])
+    cl = torch.from_numpy(x["cache_len"]).cuda()
+    o, lse = ops.decode(dev_bf16(x["q"]), dev_bf16(kc), dev_bf16(vc), cl, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    ro, rl = oracle_decode(x["q"], kc, vc, x["cache_len"], W)
+    assert rel_l2(host_f64(o), ro) <= O_REL and np.max(np.abs(host_f64(o) - ro)) <= O_ABS
+    assert np.max(np.abs(host_f64(lse) - rl)) <= LSE_ABS
+
