@@ -60,8 +60,11 @@ struct FwdCfg {
 struct FwdParams {
     __nv_bfloat16* o;
     float* lse;
-    int B, T, H;
+    int B, T, H;          // T: query rows per sequence
     int G;                // query heads per K/V head (K, V have H / G heads)
+    // Chunked prefill (kernel instantiated with kOffset): query row t of sequence b sits at
+    // absolute position q_offset[b] + t, and keys are absolute positions in K / V (a KV cache).
+    const int* q_offset;
     long long W;
     float scale_log2;     // softmax scale * log2(e)
     int n_qblk;           // ceil(T / 256)
@@ -73,6 +76,7 @@ struct FwdParams {
 // Geometry of one work item: query block qblk of head (b, h).
 struct FwdItem {
     int b, h, hk;         // batch, query head, K/V head
+    int L;                // absolute position of query row 0 of this sequence
     long long q0;         // first query row of tile 0 (tile 1 starts 128 rows later)
     bool valid1;          // tile 1 has rows below T
     int jlo0, jhi0, jlo1, jhi1, jbeg, jend;
@@ -81,6 +85,7 @@ struct FwdItem {
 // Items are head-major (all query blocks of one (b, h), then the next head), so the CTAs that
 // run at the same time read the same head's K/V tiles and share them through L2; within a
 // head the heaviest (latest) query blocks come first.
+template <bool kOffset>
 __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
     FwdItem it;
     const int bh = item / p.n_qblk;
@@ -88,18 +93,22 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
     it.b = bh / p.H;
     it.h = bh % p.H;
     it.hk = it.h / p.G;
+    it.L = kOffset ? max(0, p.q_offset[it.b]) : 0;
     it.q0 = (long long)qblk * 256;
     it.valid1 = it.q0 + 128 < p.T;
-    it.jlo0 = int(imax_ll(0, it.q0 - p.W + 1) / 128);
-    it.jhi0 = int(imin_ll(it.q0 + 127, p.T - 1) / 128);
-    it.jlo1 = int(imax_ll(0, it.q0 + 128 - p.W + 1) / 128);
-    it.jhi1 = int(imin_ll(it.q0 + 255, p.T - 1) / 128);
+    // key tiles by absolute position: query row t sees keys (L+t-W, L+t]
+    it.jlo0 = int(imax_ll(0, it.L + it.q0 - p.W + 1) / 128);
+    it.jhi0 = int((it.L + imin_ll(it.q0 + 127, p.T - 1)) / 128);
+    it.jlo1 = int(imax_ll(0, it.L + it.q0 + 128 - p.W + 1) / 128);
+    it.jhi1 = int((it.L + imin_ll(it.q0 + 255, p.T - 1)) / 128);
     it.jbeg = it.jlo0;
     it.jend = it.valid1 ? it.jhi1 : it.jhi0;
     return it;
 }
 
-template <int D>
+// kOffset: chunked prefill (query rows start at q_offset[b]); false for training, where the
+// offset is zero and costs nothing.
+template <int D, bool kOffset = false>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -182,7 +191,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int item =
                     item_produce(p.work_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
-                const FwdItem g = fwd_item(p, item);
+                const FwdItem g = fwd_item<kOffset>(p, item);
                 // A Q buffer is free once the S MMAs of the item that used it completed.
                 const int qb = qi % C::NQBUF;
                 if (qi >= C::NQBUF) {
@@ -252,7 +261,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                      kStatusTimeoutMma, ok);
                 if (!ok || item >= p.n_items) break;
-                const FwdItem g = fwd_item(p, item);
+                const FwdItem g = fwd_item<kOffset>(p, item);
                 auto act = [&](int t, int j) {
                     return t ? (g.valid1 && j >= g.jlo1 && j <= g.jhi1) : (j >= g.jlo0 && j <= g.jhi0);
                 };
@@ -333,10 +342,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int item = item_consume_warp(k, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                kStatusTimeoutSoftmax, ok);
             if (!ok || item >= p.n_items) break;
-            const FwdItem g = fwd_item(p, item);
+            const FwdItem g = fwd_item<kOffset>(p, item);
             if (t == 1 && !g.valid1) continue;
             const long long qt0 = g.q0 + t * 128;    // first row of this tile
-            const long long q = qt0 + row;           // global query index of this thread
+            const long long q = qt0 + row;           // query row of this thread (position g.L + q)
             const int jlo = t ? g.jlo1 : g.jlo0, jhi = t ? g.jhi1 : g.jhi0;
             float m_run = -INFINITY, l_run = 0.f;
             int nloc = 0;
@@ -368,7 +377,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 // Tiles that cut the diagonal or the window's left edge: keep columns clo..chi of this
                 // row (keys k0+c with q-W < k0+c <= q).  The test is uniform across the CTA.
-                const long long k0 = (long long)j * C::BN;
+                // k0: the key tile's first position, counted like the query rows (absolute - g.L)
+                const long long k0 = (long long)j * C::BN - g.L;
                 const bool full = (k0 + C::BN - 1 <= qt0) && (k0 > qt0 + C::BM - 1 - W);
                 if (!full) {
                     const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN));
@@ -448,9 +458,10 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             tc_fence_before();
             mbar_arrive(o_free(t));   // the next item's first PV may overwrite O_t now
-            if (q < T) {
+            const long long qrow = q;
+            if (qrow < T) {
                 const float inv_l = 1.f / l_run;
-                __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D;
+                __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(qrow)) * p.H + g.h) * D;
 #pragma unroll
                 for (int v8 = 0; v8 < D / 8; ++v8) {
                     uint4 w;
@@ -460,7 +471,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     w.w = pack_bf16x2(ov[v8 * 8 + 6] * inv_l, ov[v8 * 8 + 7] * inv_l);
                     *reinterpret_cast<uint4*>(orow + v8 * 8) = w;
                 }
-                p.lse[(size_t(g.b) * p.H + g.h) * T + q] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+                p.lse[(size_t(g.b) * p.H + g.h) * T + qrow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
             }
         }
     }
@@ -469,6 +480,50 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Chunked prefill, append step: a chunk of Tn tokens' K and V goes to cache slots
+// cache_len[b] .. cache_len[b] + Tn - 1 of each sequence, and the slots after it up to the end of
+// that 128-slot tile are zeroed: they hold no token, and the forward's last key tile reads them
+// (their scores are masked, and zero V rows keep P*V finite whatever the slots held).  Slots at or
+// beyond cap are not written; a chunk that needs them sets kStatusCacheOverflow.
+// One thread per 16 bytes of a (slot, K/V head) row.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __restrict__ k_new,
+                                                         const __nv_bfloat16* __restrict__ v_new,
+                                                         __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
+                                                         const int* __restrict__ cache_len, int B, int Tn, int cap,
+                                                         int Hkv) {
+    constexpr int CPR = D / 8;   // 16-byte chunks per head row
+    const int span = Tn + 128;   // chunk rows plus the largest zeroed tail
+    const long long total = (long long)B * span * Hkv * CPR;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+        const int c = int(e % CPR);
+        const long long r = e / CPR;
+        const int hk = int(r % Hkv);
+        const int t = int((r / Hkv) % span);
+        const int b = int(r / ((long long)Hkv * span));
+        const long long L = cache_len[b] < 0 ? 0 : cache_len[b];
+        const long long slot = L + t;
+        const long long tile_end = (L + Tn + 127) / 128 * 128;
+        if (t >= Tn && slot >= tile_end) continue;
+        if (slot >= cap) {
+            if (t < Tn) atomicOr(&g_attn_status, kStatusCacheOverflow);
+            continue;
+        }
+        const size_t dst = ((size_t(b) * cap + size_t(slot)) * Hkv + hk) * D + c * 8;
+        uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
+        if (t < Tn) {
+            const size_t src = ((size_t(b) * Tn + t) * Hkv + hk) * D + c * 8;
+            kw = *reinterpret_cast<const uint4*>(k_new + src);
+            vw = *reinterpret_cast<const uint4*>(v_new + src);
+        }
+        *reinterpret_cast<uint4*>(kc + dst) = kw;
+        *reinterpret_cast<uint4*>(vc + dst) = vw;
+    }
 }
 
 }  // namespace swa

@@ -179,6 +179,7 @@ int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, att
     p.T = T;
     p.H = H;
     p.G = H / Hkv;
+    p.q_offset = nullptr;
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_qblk = n_qblk;
@@ -199,6 +200,62 @@ int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, att
 int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B, int T,
              int H, int D, int W, float scale, void* stream) {
     return attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, W, scale, stream);
+}
+
+int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                 attn_bf16* v_cache, const int32_t* cache_len, attn_bf16* o, float* lse, int B, int Tn, int cap,
+                 int H, int Hkv, int D, int W, float scale, void* stream) {
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_len || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k_new, v_new, k_cache, v_cache, o, lse};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, Tn, H, D, W, scale) || !valid_kv_heads(H, Hkv) || cap < Tn) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    const int n_qblk = (Tn + 255) / 256;
+    const long long n_items = (long long)n_qblk * B * H;
+    if (n_items > 0x7fffffffLL || (long long)B * (Tn + 128) * Hkv * (D / 8) > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // 1. append the chunk's K / V (and zero the rest of its last 128-slot tile)
+    const long long chunks = (long long)B * (Tn + 128) * Hkv * (D / 8);
+    const long long blocks = std::min<long long>((chunks + 255) / 256, 148LL * 16);
+    const auto* kn = reinterpret_cast<const __nv_bfloat16*>(k_new);
+    const auto* vn = reinterpret_cast<const __nv_bfloat16*>(v_new);
+    auto* kc = reinterpret_cast<__nv_bfloat16*>(k_cache);
+    auto* vc = reinterpret_cast<__nv_bfloat16*>(v_cache);
+    if (D == 128)
+        swa_append_kernel<128><<<unsigned(blocks), 256, 0, s>>>(kn, vn, kc, vc, cache_len, B, Tn, cap, Hkv);
+    else
+        swa_append_kernel<64><<<unsigned(blocks), 256, 0, s>>>(kn, vn, kc, vc, cache_len, B, Tn, cap, Hkv);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
+    // 2. the forward of the chunk's queries at absolute positions cache_len[b] + t over the cache
+    const long long grid = n_items < sm_count() ? n_items : sm_count();
+    CUtensorMap mq, mk, mv;
+    if (!make_bthd_map(&mq, q, B, Tn, H, D) || !make_bthd_map(&mk, k_cache, B, cap, Hkv, D) ||
+        !make_bthd_map(&mv, v_cache, B, cap, Hkv, D))
+        return ATTN_ERR_LAUNCH;
+    FwdParams p;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.T = Tn;
+    p.H = H;
+    p.G = H / Hkv;
+    p.q_offset = cache_len;
+    p.W = W;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.n_qblk = n_qblk;
+    p.n_items = int(n_items);
+    p.work_slot = next_work_slot();
+    p.wait_limit = kDefaultWaitLimit;
+    if (D == 128) {
+        if (!ensure_smem((const void*)swa_fwd_kernel<128, true>, FwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_fwd_kernel<128, true><<<unsigned(grid), FwdCfg<128>::THREADS, FwdCfg<128>::SMEM, s>>>(mq, mk, mv, p);
+    } else {
+        if (!ensure_smem((const void*)swa_fwd_kernel<64, true>, FwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
+        swa_fwd_kernel<64, true><<<unsigned(grid), FwdCfg<64>::THREADS, FwdCfg<64>::SMEM, s>>>(mq, mk, mv, p);
+    }
+    return launch_status();
 }
 
 // Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128).
@@ -386,6 +443,7 @@ int attn_device_status(int clear) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(swa::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
     }
+    if (v & swa::kStatusCacheOverflow) return ATTN_ERR_CACHE_OVERFLOW;
     return v ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
 }
 
@@ -403,6 +461,7 @@ const char* attn_status_string(int status) {
         case ATTN_ERR_LAUNCH: return "kernel launch failed";
         case ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case ATTN_ERR_WORKSPACE: return "workspace too small";
+        case ATTN_ERR_CACHE_OVERFLOW: return "cache capacity exceeded";
         default: return "unknown status";
     }
 }

@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libswa_b200.so")
 
 ATTN_OK = 0
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported configuration", -3: "kernel launch failed",
-          -4: "device wait timed out", -5: "workspace too small"}
+          -4: "device wait timed out", -5: "workspace too small", -6: "cache capacity exceeded"}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m causal_sliding_window_b200.build`")
@@ -49,6 +49,8 @@ _lib.attn_bwd_gqa.argtypes = [_p] * 10 + [_sz, _i, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_bwd_gqa.restype = _i
 _lib.attn_decode_gqa.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode_gqa.restype = _i
+_lib.attn_prefill.argtypes = [_p] * 8 + [_i, _i, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_prefill.restype = _i
 _lib.attn_decode_noalloc.argtypes = [_p] * 6 + [_i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode_noalloc.restype = _i
 _lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
@@ -61,7 +63,7 @@ _lib.attn_status_string.argtypes = [_i]
 _lib.attn_status_string.restype = ctypes.c_char_p
 
 EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_gqa",
-            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
+            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
             "attn_status_string"]
 
 
@@ -160,6 +162,31 @@ def attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W: int, scale
     else:
         _check(_lib.attn_decode_gqa(*ptrs, ws_bytes, B, cap, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)),
                "attn_decode_gqa")
+
+
+def attn_prefill(q, k_new, v_new, k_cache, v_cache, cache_len, o, lse, W: int, scale=None, stream=None):
+    """Append a chunk's K / V to the caches and attend its queries (see attn_prefill in the header)."""
+    B, Tn, H, D = _bthd(q, o)
+    Hkv = _kv_heads((B, Tn, H, D), k_new, v_new)
+    Bc, cap, Hc, Dc = _bthd(k_cache, v_cache)
+    if (Bc, Hc, Dc) != (B, Hkv, D):
+        raise ValueError("caches must be [B, cap, Hkv, D] matching k_new")
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or not cache_len.is_cuda:
+        raise ValueError("cache_len must be an int32 CUDA tensor of shape [B]")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Tn) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, Tn] tensor")
+    _check(_lib.attn_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len),
+                             _ptr(o), _ptr(lse), B, Tn, cap, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)),
+           "attn_prefill")
+
+
+def prefill(q, k_new, v_new, k_cache, v_cache, cache_len, W: int, scale=None, stream=None):
+    """attn_prefill with freshly allocated outputs; returns (o, lse)."""
+    B, Tn, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Tn), dtype=torch.float32, device=q.device)
+    attn_prefill(q, k_new, v_new, k_cache, v_cache, cache_len, o, lse, W, scale, stream)
+    return o, lse
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, cache_len, o, lse, W: int, scale=None, stream=None):

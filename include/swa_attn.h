@@ -35,7 +35,9 @@
  *    be executing on the device at the same time (on different streams).
  *  - Device-side waits are bounded.  If one gives up (a condition that
  *    correct use never produces), the kernel stops early and records a flag
- *    that attn_device_status() reports as ATTN_ERR_DEVICE_TIMEOUT.
+ *    that attn_device_status() reports as ATTN_ERR_DEVICE_TIMEOUT.  A prefill
+ *    chunk that does not fit its cache is reported there as
+ *    ATTN_ERR_CACHE_OVERFLOW.
  */
 #ifndef SWA_ATTN_H
 #define SWA_ATTN_H
@@ -55,7 +57,8 @@ typedef enum {
     ATTN_ERR_UNSUPPORTED = -2,
     ATTN_ERR_LAUNCH = -3,
     ATTN_ERR_DEVICE_TIMEOUT = -4,
-    ATTN_ERR_WORKSPACE = -5
+    ATTN_ERR_WORKSPACE = -5,
+    ATTN_ERR_CACHE_OVERFLOW = -6
 } attn_status;
 
 /*
@@ -79,6 +82,30 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
  */
 int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
                  int B, int T, int H, int Hkv, int D, int W, float scale, void* stream);
+
+/*
+ * Chunked prefill against a KV cache, with append: the engine's
+ * flash_attn_with_kvcache(q, k_cache, v_cache, k=k_new, v=v_new, cache_seqlens=...)
+ * (apidog guide, section 6 "Inference engine") with the window of attn_fwd.
+ *   q             [B, Tn, H, D] bf16: a chunk of Tn new tokens per sequence.
+ *   k_new, v_new  [B, Tn, Hkv, D] bf16: their keys and values.
+ *   k_cache, v_cache  [B, cap, Hkv, D] bf16, updated in place.
+ *   cache_len     [B] int32 in device memory: tokens already cached; the chunk's
+ *                 token t of sequence b sits at position cache_len[b] + t.
+ *   o             [B, Tn, H, D] bf16, written.   lse  [B, H, Tn] fp32, written.
+ * The call first writes k_new / v_new into slots cache_len[b] .. cache_len[b]+Tn-1
+ * and zeros the slots after them up to the end of that 128-slot block (slots that
+ * hold no token); then query t attends to cached positions p - W < j <= p,
+ * p = cache_len[b] + t (the previous tokens and the chunk's own, causally).  It does
+ * not change cache_len.  cache_len[b] + Tn must not exceed cap: slots past cap are
+ * not written and attn_device_status() then reports ATTN_ERR_CACHE_OVERFLOW (the
+ * outputs of that sequence are undefined).  Hkv divides H as in attn_fwd_gqa; cap
+ * must be >= Tn.  With every cache_len 0 the result equals attn_fwd_gqa on
+ * (q, k_new, v_new); with Tn = 1 it is one decode step with append.
+ */
+int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                 attn_bf16* v_cache, const int32_t* cache_len, attn_bf16* o, float* lse, int B, int Tn,
+                 int cap, int H, int Hkv, int D, int W, float scale, void* stream);
 
 /* Bytes of workspace attn_bwd needs: fp32 rows of lse*log2(e) and Delta, [B*H, T rounded up
  * to 128] each (256-byte padded). */

@@ -17,5 +17,6 @@ from .swa_oracle import (  # noqa: F401
     oracle_dq_rows,
     oracle_fwd,
     oracle_fwd_rows,
+    oracle_prefill,
     oracle_threads,
 )

@@ -167,3 +167,34 @@ def oracle_decode(q, k_cache, v_cache, cache_len, W: int, scale: float | None = 
     _load().swa_oracle_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), bf, cl.ctypes.data_as(ctypes.c_void_p),
                               B, cap, H, Hk, D, int(W), float(scale), _ptr(o), _ptr(lse))
     return o, lse
+
+
+def oracle_prefill(q, k_new, v_new, k_cache, v_cache, cache_len, W: int, scale: float | None = None):
+    """Chunked prefill with append, written out as its definition (the engine's
+    flash_attn_with_kvcache with new K / V, apidog guide section 6): for sequence b the cache
+    afterwards holds its first cache_len[b] tokens followed by the chunk, and the chunk's query t
+    is row cache_len[b] + t of the forward over that token sequence.
+
+    q [B,Tn,H,D]; k_new, v_new [B,Tn,Hk,D]; caches [B,cap,Hk,D]; cache_len [B] (tokens cached
+    before the chunk).  Returns (o [B,Tn,H,D], lse [B,H,Tn], k_cache_after, v_cache_after); the
+    inputs are not modified and cache slots past cache_len[b] + Tn keep their input values."""
+    (q, k_new, v_new, k_cache, v_cache), _ = _prep(q, k_new, v_new, k_cache, v_cache)
+    B, Tn, H, D = q.shape
+    cap = k_cache.shape[1]
+    kc, vc = k_cache.copy(), v_cache.copy()
+    o = np.empty((B, Tn, H, D), np.float64)
+    lse = np.empty((B, H, Tn), np.float64)
+    for b in range(B):
+        L = int(cache_len[b])
+        n = L + Tn
+        if L < 0 or n > cap:
+            raise ValueError("cache_len[b] + Tn must lie in [Tn, cap]")
+        kc[b, L:n] = k_new[b]
+        vc[b, L:n] = v_new[b]
+        qs = np.zeros((1, n, H, D), dtype=q.dtype)
+        qs[0, L:] = q[b]
+        rows = np.array([(0, h, L + t) for h in range(H) for t in range(Tn)], dtype=np.int64)
+        ob, lb = oracle_fwd_rows(qs, kc[b:b + 1, :n], vc[b:b + 1, :n], W, rows, scale)
+        o[b] = ob.reshape(H, Tn, D).transpose(1, 0, 2)
+        lse[b] = lb.reshape(H, Tn)
+    return o, lse, kc, vc

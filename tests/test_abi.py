@@ -131,3 +131,15 @@ def test_grouped_kv_heads_argument_checks():
     assert ops._lib.attn_decode_gqa(A, A, A, A, A, A, A, dws, 2, 64, 6, 4, 128, 8, 0.1, None) == ERR_INVALID
     assert ops._lib.attn_fwd_gqa(A, A, A, A, A, 1, 16, 6, 2, 96, 4, 0.1, None) == ERR_UNSUPPORTED
 
+
+def test_prefill_argument_checks():
+    args = lambda **kw: dict(dict(B=2, Tn=16, cap=64, H=4, Hkv=2, D=128, W=8, scale=0.1), **kw)  # noqa: E731
+    call = lambda a, cl=A: ops._lib.attn_prefill(A, A, A, A, A, cl, A, A, a["B"], a["Tn"], a["cap"], a["H"],  # noqa: E731
+                                                  a["Hkv"], a["D"], a["W"], a["scale"], None)
+    assert call(args(cap=15)) == ERR_INVALID          # cap < Tn
+    assert call(args(Hkv=3)) == ERR_INVALID           # Hkv must divide H
+    assert call(args(), cl=A + 2) == ERR_INVALID      # cache_len misaligned
+    assert call(args(W=0)) == ERR_INVALID
+    assert call(args(D=96)) == ERR_UNSUPPORTED
+    assert ops.attn_status_string(-6) == "cache capacity exceeded"
+

@@ -15,7 +15,7 @@ import torch
 
 from causal_sliding_window_b200 import inputs
 from oracle import (oracle_bwd, oracle_decode, oracle_dkv_rows, oracle_dq_rows, oracle_fwd,
-                    oracle_fwd_rows)
+                    oracle_fwd_rows, oracle_prefill)
 
 pytestmark = pytest.mark.gpu
 
@@ -287,4 +287,64 @@ def test_grouped_kv_heads_decode(ops, H, Hkv):
     ro, rl = oracle_decode(x["q"], kc, vc, x["cache_len"], W)
     assert rel_l2(host_f64(o), ro) <= O_REL and np.max(np.abs(host_f64(o) - ro)) <= O_ABS
     assert np.max(np.abs(host_f64(lse) - rl)) <= LSE_ABS
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill with append against a KV cache.
+# ---------------------------------------------------------------------------
+NAN_BF16 = 0x7FC0
+
+PREFILL = [
+    # (B, Tn, cap, H, Hkv, D, W, cache_len before the chunk)
+    (3, 77, 700, 4, 2, 128, 129, (0, 5, 600)),
+    (2, 300, 1024, 4, 4, 128, 10 ** 9, (0, 700)),
+    (2, 1, 300, 8, 2, 128, 64, (0, 299)),
+    (2, 256, 640, 2, 2, 64, 100, (128, 300)),
+]
+
+
+@pytest.mark.parametrize("B,Tn,cap,H,Hkv,D,W,lens", PREFILL)
+def test_prefill_matches_oracle_and_appends(ops, B, Tn, cap, H, Hkv, D, W, lens):
+    L = np.array(lens, dtype=np.int32)
+    x = inputs.attention_inputs(B, Tn, H, D, seed=700 + Tn + cap)
+    c = inputs.decode_inputs(B, cap, Hkv, D, seed=701 + Tn)
+    kn, vn = (np.ascontiguousarray(x[n][:, :, :Hkv]) for n in ("k", "v"))
+    kc, vc = c["k_cache"].copy(), c["v_cache"].copy()
+    for b in range(B):   # slots that hold no token: a read that reached P*V would poison the output
+        kc[b, L[b] + Tn:] = NAN_BF16
+        vc[b, L[b] + Tn:] = NAN_BF16
+    dkc, dvc = dev_bf16(kc), dev_bf16(vc)
+    o, lse = ops.prefill(dev_bf16(x["q"]), dev_bf16(kn), dev_bf16(vn), dkc, dvc, torch.from_numpy(L).cuda(), W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    ro, rl, rkc, rvc = oracle_prefill(x["q"], kn, vn, kc, vc, L, W)
+    go, gl = host_f64(o), host_f64(lse)
+    assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
+    assert np.max(np.abs(gl - rl)) <= LSE_ABS
+    got_k = dkc.cpu().view(torch.int16).numpy().view(np.uint16)
+    got_v = dvc.cpu().view(torch.int16).numpy().view(np.uint16)
+    for b in range(B):
+        n = int(L[b]) + Tn
+        end = min(cap, (n + 127) // 128 * 128)
+        np.testing.assert_array_equal(got_k[b, :n], rkc[b, :n])   # prefix untouched, chunk appended
+        np.testing.assert_array_equal(got_v[b, :n], rvc[b, :n])
+        assert not got_k[b, n:end].any() and not got_v[b, n:end].any()   # rest of the 128-slot block zeroed
+        np.testing.assert_array_equal(got_k[b, end:], kc[b, end:])      # beyond it untouched
+        np.testing.assert_array_equal(got_v[b, end:], vc[b, end:])
+
+
+def test_prefill_overflow_is_reported_and_stays_in_bounds(ops):
+    B, Tn, cap, H, D, W = 2, 64, 100, 2, 128, 50
+    x = inputs.attention_inputs(B, Tn, H, D, seed=9)
+    kc, vc = Guarded((B, cap, H, D), torch.bfloat16), Guarded((B, cap, H, D), torch.bfloat16)
+    kc.t.zero_()
+    vc.t.zero_()
+    L = torch.tensor([0, 50], dtype=torch.int32, device="cuda")   # 50 + 64 > 100 for sequence 1
+    o, lse = ops.prefill(dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"]), kc.t, vc.t, L, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == -6   # ATTN_ERR_CACHE_OVERFLOW
+    assert kc.guards_intact() and vc.guards_intact()
+    ro, rl, _, _ = oracle_prefill(x["q"][:1], x["k"][:1], x["v"][:1], np.zeros((1, cap, H, D), np.uint16),
+                                  np.zeros((1, cap, H, D), np.uint16), np.array([0]), W)
+    assert rel_l2(host_f64(o[:1]), ro) <= O_REL   # the sequence that fits is unaffected
 

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from causal_sliding_window_b200 import inputs
-from oracle import (oracle_bwd, oracle_decode, oracle_dkv_rows, oracle_dq_rows, oracle_fwd,
+from oracle import (oracle_bwd, oracle_decode, oracle_dkv_rows, oracle_dq_rows, oracle_fwd, oracle_prefill,
                     oracle_fwd_rows)
 
 
@@ -328,4 +328,42 @@ def test_grouped_kv_heads_must_divide():
     x = inputs.attention_inputs(1, 8, 3, 8, seed=1)
     with pytest.raises(ValueError):
         oracle_fwd(x["q"], x["k"][:, :, :2].copy(), x["v"][:, :, :2].copy(), 4)
+
+
+def prefill_inputs(B, Tn, cap, H, Hk, D, seed):
+    x = inputs.attention_inputs(B, Tn, H, D, seed=seed)
+    c = inputs.decode_inputs(B, cap, Hk, D, seed=seed + 1)
+    return (x["q"], np.ascontiguousarray(x["k"][:, :, :Hk]), np.ascontiguousarray(x["v"][:, :, :Hk]),
+            c["k_cache"], c["v_cache"])
+
+
+def test_prefill_on_an_empty_cache_is_the_forward():
+    q, kn, vn, kc, vc = prefill_inputs(2, 40, 64, 4, 2, 16, seed=5)
+    o, lse, kc2, vc2 = oracle_prefill(q, kn, vn, kc, vc, np.array([0, 0]), 13)
+    ro, rl = oracle_fwd(q, kn, vn, 13)
+    np.testing.assert_array_equal(o, ro)
+    np.testing.assert_array_equal(lse, rl)
+    np.testing.assert_array_equal(kc2[:, :40], kn)
+    np.testing.assert_array_equal(vc2[:, 40:], vc[:, 40:])
+
+
+def test_prefill_of_one_token_is_a_decode_step():
+    q, kn, vn, kc, vc = prefill_inputs(3, 1, 50, 4, 2, 16, seed=8)
+    L = np.array([0, 17, 49])
+    o, lse, kc2, vc2 = oracle_prefill(q, kn, vn, kc, vc, L, 9)
+    od, ld_ = oracle_decode(np.ascontiguousarray(q[:, 0]), kc2, vc2, L + 1, 9)
+    np.testing.assert_allclose(o[:, 0], od, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, :, 0], ld_, rtol=0, atol=1e-13)
+
+
+def test_prefill_in_two_chunks_equals_one_chunk():
+    """Chunked prefill: chunk A then chunk B over the updated cache gives chunk A+B's outputs."""
+    q, kn, vn, kc, vc = prefill_inputs(2, 30, 80, 4, 1, 16, seed=12)
+    L = np.array([3, 25])
+    o, lse, kc_ab, vc_ab = oracle_prefill(q, kn, vn, kc, vc, L, 17)
+    oa, la, kc_a, vc_a = oracle_prefill(q[:, :12], kn[:, :12], vn[:, :12], kc, vc, L, 17)
+    ob, lb, kc_b, vc_b = oracle_prefill(q[:, 12:], kn[:, 12:], vn[:, 12:], kc_a, vc_a, L + 12, 17)
+    np.testing.assert_allclose(np.concatenate([oa, ob], axis=1), o, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(np.concatenate([la, lb], axis=2), lse, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(kc_b, kc_ab)
 
