@@ -8,9 +8,11 @@
 //
 // Layout: caches [B, cap, H, D] bf16, so one cache slot of one sequence is a
 // contiguous H*D*2-byte row (3 KB at H=12, D=128).  A CTA takes a chunk of
-// CHUNK consecutive slots of one sequence and a group of up to 256*8/D heads
-// (all 12 heads at D=128): thread slot (h, c) owns the 16-byte piece c of
-// head h, so every slot row is read as one fully coalesced, vectorised sweep.  Per head, the D/8 threads reduce q.k
+// CHUNK consecutive slots of one sequence and a group of up to kDecodeThreads*8/D consecutive
+// heads (4 at D = 128): thread slot (h, c) owns the 16-byte piece c of head h, so each slot's
+// heads of the group are read as one contiguous, coalesced, vectorised sweep (1 KB at D = 128).
+// Small head groups put more CTAs, and so more loads, in flight (measured: 64 threads per CTA
+// beat 256 by about 4% on the decode workload).  Per head, the D/8 threads reduce q.k
 // with warp shuffles and keep an online softmax (m, l) and 8 output
 // accumulators in registers.  Each CTA writes its partial (m, l, o) to the
 // workspace; the last CTA of a sequence (atomic ticket) merges the partials:
@@ -45,7 +47,7 @@ struct DecParams {
     int nsplit_max;                // stride of the partial arrays
 };
 
-constexpr int kDecodeThreads = 256;
+constexpr int kDecodeThreads = 64;   // threads per CTA: D/8 per head, so 4 heads of D = 128 (more CTAs in flight)
 
 template <int D>
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {

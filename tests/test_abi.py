@@ -76,10 +76,13 @@ def test_workspace_sizes():
     assert ops.attn_bwd_workspace_bytes(1, 130, 1, 64) == 2 * 256 * 4   # Tp = 256
     assert ops.attn_bwd_workspace_bytes(1, 1, 1, 128) == 2 * 512   # 128 floats per row, no 256-byte padding needed
     assert ops.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
-    # ticket counters [B] + partial (m, l) and o for ceil(cap / 128) chunks of 128 cache slots
+    # ticket counters [B, head groups of 4 heads (D = 128) / 8 heads (D = 64)] + partial (m, l) and o
+    # for ceil(cap / 128) chunks of 128 cache slots
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert ops.attn_decode_workspace_bytes(32, 2048, 12, 128) == a256(32 * 4) + a256(32 * 16 * 12 * 2 * 4) + a256(
+    assert ops.attn_decode_workspace_bytes(32, 2048, 12, 128) == a256(32 * 3 * 4) + a256(32 * 16 * 12 * 2 * 4) + a256(
         32 * 16 * 12 * 128 * 4)
+    assert ops.attn_decode_workspace_bytes(2, 100, 9, 64) == a256(2 * 2 * 4) + a256(2 * 1 * 9 * 2 * 4) + a256(
+        2 * 1 * 9 * 64 * 4)
     assert ops.attn_decode_workspace_bytes(1, 0, 1, 64) == 0
     for bad_d in (0, 4, 7, 96):
         assert ops.attn_decode_workspace_bytes(1, 16, 1, bad_d) == 0
