@@ -349,12 +349,32 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     return attn_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, H, D, W, scale, stream);
 }
 
-size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
-    if (B < 1 || cap < 1 || H < 1 || (D != 64 && D != 128)) return 0;
-    const size_t nsm = size_t((cap + kDecodeChunk - 1) / kDecodeChunk);
-    const size_t nhg = size_t((H + kDecodeThreads / (D / 8) - 1) / (kDecodeThreads / (D / 8)));
-    return align256(size_t(B) * nhg * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
+// Decode geometry for H query heads over Hkv K/V heads: query heads per thread, slots per CTA,
+// (K/V head, query subgroup) pair groups per sequence.
+struct DecGeom {
+    int qpt, nsub, chunk, nzg;
+};
+static DecGeom decode_geom(int H, int Hkv, int D) {
+    DecGeom g;
+    const int kvg = H / Hkv;
+    g.qpt = decode_qpt(kvg);
+    g.nsub = (kvg + g.qpt - 1) / g.qpt;
+    g.chunk = g.qpt == 1 ? kDecodeChunk : kDecodeChunkGrp;
+    const int pairs_per_cta = kDecodeThreads / (D / 8);
+    g.nzg = (Hkv * g.nsub + pairs_per_cta - 1) / pairs_per_cta;
+    return g;
+}
+
+size_t attn_decode_gqa_workspace_bytes(int B, int cap, int H, int Hkv, int D) {
+    if (B < 1 || cap < 1 || H < 1 || (D != 64 && D != 128) || !valid_kv_heads(H, Hkv)) return 0;
+    const DecGeom g = decode_geom(H, Hkv, D);
+    const size_t nsm = size_t((cap + g.chunk - 1) / g.chunk);
+    return align256(size_t(B) * g.nzg * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
            align256(size_t(B) * nsm * H * D * 4);
+}
+
+size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
+    return attn_decode_gqa_workspace_bytes(B, cap, H, H, D);
 }
 
 int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
@@ -368,8 +388,10 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
     if (!valid_common(B, cap, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535) return ATTN_ERR_UNSUPPORTED;
-    if (ws_bytes < attn_decode_workspace_bytes(B, cap, H, D)) return ATTN_ERR_WORKSPACE;
-    const int nsm = (cap + kDecodeChunk - 1) / kDecodeChunk;
+    if (ws_bytes < attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)) return ATTN_ERR_WORKSPACE;
+    const DecGeom g = decode_geom(H, Hkv, D);
+    if (g.nzg > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int nsm = (cap + g.chunk - 1) / g.chunk;
     const int span = W < cap ? W : cap;
     DecParams p;
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -378,11 +400,8 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
     p.cache_len = cache_len;
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.lse = lse;
-    const int heads_per_cta = kDecodeThreads / (D / 8);
-    const int nhg = (H + heads_per_cta - 1) / heads_per_cta;
-    if (nhg > 65535) return ATTN_ERR_UNSUPPORTED;
     char* ws = static_cast<char*>(workspace);
-    const size_t cnt_bytes = align256(size_t(B) * nhg * 4);
+    const size_t cnt_bytes = align256(size_t(B) * g.nzg * 4);
     p.counters = reinterpret_cast<int*>(ws);
     p.part_ml = reinterpret_cast<float*>(ws + cnt_bytes);
     p.part_o = reinterpret_cast<float*>(ws + cnt_bytes + align256(size_t(B) * nsm * H * 2 * 4));
@@ -390,17 +409,33 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
     p.cap = cap;
     p.H = H;
     p.kv_group = H / Hkv;
+    p.nsub = g.nsub;
+    p.chunk = g.chunk;
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.nsplit = (span + kDecodeChunk - 1) / kDecodeChunk;
+    p.nsplit = (span + g.chunk - 1) / g.chunk;
     p.nsplit_max = nsm;
-    const int threads = ((std::min(H, heads_per_cta) * (D / 8)) + 31) / 32 * 32;
-    dim3 grid(p.nsplit, B, nhg);
+    const int pairs_per_cta = kDecodeThreads / (D / 8);
+    const int threads = ((std::min(Hkv * g.nsub, pairs_per_cta) * (D / 8)) + 31) / 32 * 32;
+    dim3 grid(p.nsplit, B, g.nzg);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (D == 128)
-        swa_decode_kernel<128><<<grid, threads, 0, s>>>(p);
-    else
-        swa_decode_kernel<64><<<grid, threads, 0, s>>>(p);
+#define SWA_DECODE_LAUNCH(DD, QQ) swa_decode_kernel<DD, QQ><<<grid, threads, 0, s>>>(p)
+    if (D == 128) {
+        switch (g.qpt) {
+            case 1: SWA_DECODE_LAUNCH(128, 1); break;
+            case 2: SWA_DECODE_LAUNCH(128, 2); break;
+            case 3: SWA_DECODE_LAUNCH(128, 3); break;
+            default: SWA_DECODE_LAUNCH(128, 4); break;
+        }
+    } else {
+        switch (g.qpt) {
+            case 1: SWA_DECODE_LAUNCH(64, 1); break;
+            case 2: SWA_DECODE_LAUNCH(64, 2); break;
+            case 3: SWA_DECODE_LAUNCH(64, 3); break;
+            default: SWA_DECODE_LAUNCH(64, 4); break;
+        }
+    }
+#undef SWA_DECODE_LAUNCH
     return launch_status();
 }
 
@@ -421,8 +456,7 @@ int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn
     void* ws = noalloc_scratch();
     if (ws == nullptr) return ATTN_ERR_LAUNCH;
     // The ticket counters at the start of the scratch must be zero when a call begins.
-    const int heads_per_cta = kDecodeThreads / (D / 8);
-    const size_t counter_bytes = size_t(B) * ((H + heads_per_cta - 1) / heads_per_cta) * 4;
+    const size_t counter_bytes = size_t(B) * decode_geom(H, H, D).nzg * 4;
     if (cudaMemsetAsync(ws, 0, counter_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return ATTN_ERR_LAUNCH;
     return attn_decode(q, k_cache, v_cache, cache_len, o, lse, ws, kNoAllocScratchBytes, B, cap, H, D, W, scale,

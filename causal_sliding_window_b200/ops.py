@@ -41,6 +41,8 @@ _lib.attn_bwd.argtypes = [_p] * 10 + [_sz, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_bwd.restype = _i
 _lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
 _lib.attn_decode_workspace_bytes.restype = _sz
+_lib.attn_decode_gqa_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+_lib.attn_decode_gqa_workspace_bytes.restype = _sz
 _lib.attn_decode.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode.restype = _i
 _lib.attn_fwd_gqa.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p]
@@ -63,7 +65,7 @@ _lib.attn_status_string.argtypes = [_i]
 _lib.attn_status_string.restype = ctypes.c_char_p
 
 EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_gqa",
-            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
+            "attn_decode_workspace_bytes", "attn_decode_gqa_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
             "attn_status_string"]
 
 
@@ -144,6 +146,10 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, W: int, scale=None, s
 
 def attn_decode_workspace_bytes(B: int, cap: int, H: int, D: int) -> int:
     return int(_lib.attn_decode_workspace_bytes(B, cap, H, D))
+
+
+def attn_decode_gqa_workspace_bytes(B: int, cap: int, H: int, Hkv: int, D: int) -> int:
+    return int(_lib.attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D))
 
 
 def attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W: int, scale=None, stream=None):
@@ -243,9 +249,11 @@ def backward(q, k, v, o, lse, dout, W: int, scale=None, stream=None, workspace=N
     return dq, dk, dv
 
 
-def decode_workspace(B: int, cap: int, H: int, D: int, device) -> torch.Tensor:
-    """Zero-filled decode workspace (the decode call keeps it zeroed between calls)."""
-    return torch.zeros(attn_decode_workspace_bytes(B, cap, H, D), dtype=torch.uint8, device=device)
+def decode_workspace(B: int, cap: int, H: int, D: int, device, Hkv=None) -> torch.Tensor:
+    """Zero-filled decode workspace (the decode call keeps it zeroed between calls); Hkv = number of
+    K/V heads of the caches (default H)."""
+    n = attn_decode_gqa_workspace_bytes(B, cap, H, H if Hkv is None else Hkv, D)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def decode(q, k_cache, v_cache, cache_len, W: int, scale=None, stream=None, workspace=None):
@@ -254,6 +262,6 @@ def decode(q, k_cache, v_cache, cache_len, W: int, scale=None, stream=None, work
     o = torch.empty((B, H, D), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = decode_workspace(B, cap, H, D, q.device)
+        workspace = decode_workspace(B, cap, H, D, q.device, Hkv=k_cache.shape[2])
     attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W, scale, stream)
     return o, lse

@@ -164,10 +164,19 @@ int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v
                 const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes,
                 int B, int cap, int H, int D, int W, float scale, void* stream);
 
+/* Bytes of workspace attn_decode_gqa needs (any W); 0 for sizes it rejects (as
+ * attn_decode_workspace_bytes, or Hkv not dividing H).  With grouped heads one thread serves
+ * several query heads of a K/V head over a shorter run of cache slots, so more partials per
+ * query head are kept than attn_decode_workspace_bytes(B, cap, H, D) provides for. */
+size_t attn_decode_gqa_workspace_bytes(int B, int cap, int H, int Hkv, int D);
+
 /*
  * Decode with grouped K/V heads: k_cache, v_cache are [B, cap, Hkv, D]; query head h
- * reads cache head h / (H / Hkv).  Workspace as attn_decode (per query head).
- * attn_decode is this call with Hkv = H.
+ * reads cache head h / (H / Hkv).  Each K/V row is loaded once for up to four of the query
+ * heads that share it.  workspace: at least attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)
+ * bytes, otherwise as attn_decode.  attn_decode is this call with Hkv = H.
+ * Defined by: the engine's KV cache (apidog guide, section 6 "Inference engine") with the
+ * grouped K/V heads of the model (same guide, section 1 "GPT model").
  */
 int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
                     const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes,

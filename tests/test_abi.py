@@ -88,6 +88,27 @@ def test_workspace_sizes():
         assert ops.attn_decode_workspace_bytes(1, 16, 1, bad_d) == 0
 
 
+def test_grouped_decode_workspace_size():
+    """With grouped K/V heads a thread serves up to 4 query heads of one K/V head (a divisor of the
+    group where there is one) over runs of 64 cache slots; counters per group of 4 (D = 128) or 8
+    (D = 64) (K/V head, query subgroup) pairs, partials per query head and 64-slot run."""
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    # 12 query heads over 4 K/V heads: 3 per thread, 4 pairs -> 1 counter per sequence, 32 runs
+    assert ops.attn_decode_gqa_workspace_bytes(32, 2048, 12, 4, 128) == a256(32 * 1 * 4) + a256(
+        32 * 32 * 12 * 2 * 4) + a256(32 * 32 * 12 * 128 * 4)
+    # MQA, 8 query heads: 4 per thread, 2 subgroups, 8 pairs per CTA at D = 64
+    assert ops.attn_decode_gqa_workspace_bytes(2, 100, 8, 1, 64) == a256(2 * 1 * 4) + a256(2 * 2 * 8 * 2 * 4) + a256(
+        2 * 2 * 8 * 64 * 4)
+    # 40 query heads over 8 K/V heads: groups of 5 -> 4 + 1 (ragged), 16 pairs -> 4 counters
+    assert ops.attn_decode_gqa_workspace_bytes(1, 64, 40, 8, 128) == a256(1 * 4 * 4) + a256(1 * 1 * 40 * 2 * 4) + a256(
+        1 * 1 * 40 * 128 * 4)
+    for B, cap, H, D in ((32, 2048, 12, 128), (2, 100, 9, 64), (3, 1, 1, 128)):
+        assert ops.attn_decode_gqa_workspace_bytes(B, cap, H, H, D) == ops.attn_decode_workspace_bytes(B, cap, H, D)
+    assert ops.attn_decode_gqa_workspace_bytes(2, 64, 6, 4, 128) == 0      # 4 does not divide 6
+    assert ops.attn_decode_gqa_workspace_bytes(2, 64, 6, 0, 128) == 0
+    assert ops.attn_decode_gqa_workspace_bytes(2, 64, 6, 3, 96) == 0
+
+
 def dec(q=A, cl=A, ws=A, ws_bytes=None, B=2, cap=64, H=2, D=128, W=8, scale=0.1, lse=A):
     if ws_bytes is None:
         ws_bytes = ops.attn_decode_workspace_bytes(B, cap, H, D) if B > 0 and cap > 0 and H > 0 else 0

@@ -274,19 +274,58 @@ def test_grouped_kv_heads_match_oracle(ops, B, T, H, Hkv, D, W):
     assert rel_l2(host_f64(dv.t), rdv) <= G_REL
 
 
-@pytest.mark.parametrize("H,Hkv", [(12, 4), (8, 1)])
-def test_grouped_kv_heads_decode(ops, H, Hkv):
-    B, cap, D, W = 5, 300, 128, 150
-    x = inputs.decode_inputs(B, cap, H, D, seed=H + Hkv, cache_len=np.array([1, 64, 149, 151, 300]))
+# (H, Hkv, D): query heads per thread 3, 4 (two subgroups), 3 (two subgroups), 4 with a ragged
+# subgroup of 1, 2, 4 with a ragged subgroup of 3
+@pytest.mark.parametrize("H,Hkv,D", [(12, 4, 128), (8, 1, 128), (12, 2, 128), (10, 2, 128), (4, 2, 64), (14, 2, 64)])
+def test_grouped_kv_heads_decode(ops, H, Hkv, D):
+    B, cap, W = 6, 300, 150
+    x = inputs.decode_inputs(B, cap, H, D, seed=H + Hkv + D, cache_len=np.array([1, 64, 149, 151, 300, 233]))
     kc = np.ascontiguousarray(x["k_cache"][:, :, :Hkv])
     vc = np.ascontiguousarray(x["v_cache"][:, :, :Hkv])
+    for b, L in enumerate(x["cache_len"]):   # NaN in every slot outside the window: never read
+        lo = max(0, int(L) - W)
+        kc[b, :lo] = vc[b, :lo] = 0x7FC0
+        kc[b, L:] = vc[b, L:] = 0x7FC0
+    cl = torch.from_numpy(x["cache_len"]).cuda()
+    o, lse = Guarded((B, H, D), torch.bfloat16), Guarded((B, H), torch.float32)
+    ws = ops.decode_workspace(B, cap, H, D, "cuda", Hkv=Hkv)
+    for _ in range(2):   # the second call checks that the first left the workspace zeroed
+        ops.attn_decode(dev_bf16(x["q"]), dev_bf16(kc), dev_bf16(vc), cl, o.t, lse.t, ws, W)
+        torch.cuda.synchronize()
+        assert ops.attn_device_status(clear=True) == 0
+        assert o.guards_intact() and lse.guards_intact()
+        ro, rl = oracle_decode(x["q"], kc, vc, x["cache_len"], W)
+        check_decode(host_f64(o.t), host_f64(lse.t), ro, rl)
+
+
+@pytest.mark.parametrize("W", [2048, 1024])
+def test_grouped_kv_heads_decode_workload(ops, W):
+    """The decode workload with 4 K/V heads for its 12 query heads."""
+    c = inputs.DECODE_WORKLOAD
+    x = inputs.decode_inputs(c["B"], c["cap"], c["H"], c["D"], seed=c["seed"])
+    kc = np.ascontiguousarray(x["k_cache"][:, :, :4])
+    vc = np.ascontiguousarray(x["v_cache"][:, :, :4])
     cl = torch.from_numpy(x["cache_len"]).cuda()
     o, lse = ops.decode(dev_bf16(x["q"]), dev_bf16(kc), dev_bf16(vc), cl, W)
     torch.cuda.synchronize()
     assert ops.attn_device_status(clear=True) == 0
     ro, rl = oracle_decode(x["q"], kc, vc, x["cache_len"], W)
-    assert rel_l2(host_f64(o), ro) <= O_REL and np.max(np.abs(host_f64(o) - ro)) <= O_ABS
-    assert np.max(np.abs(host_f64(lse) - rl)) <= LSE_ABS
+    check_decode(host_f64(o), host_f64(lse), ro, rl)
+
+
+def test_grouped_decode_rejects_the_plain_workspace_size(ops):
+    """Grouped heads keep more partials per query head than the plain decode workspace holds."""
+    B, cap, H, Hkv, D = 2, 300, 12, 4, 128
+    assert ops.attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D) > ops.attn_decode_workspace_bytes(B, cap, H, D)
+    x = inputs.decode_inputs(B, cap, H, D, seed=5, cache_len=np.array([10, 300]))
+    kc = dev_bf16(np.ascontiguousarray(x["k_cache"][:, :, :Hkv]))
+    vc = dev_bf16(np.ascontiguousarray(x["v_cache"][:, :, :Hkv]))
+    cl = torch.from_numpy(x["cache_len"]).cuda()
+    o = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+    ws = ops.decode_workspace(B, cap, H, D, "cuda")
+    with pytest.raises(ops.AttnError):
+        ops.attn_decode(dev_bf16(x["q"]), kc, vc, cl, o, lse, ws, 100)
 
 
 # ---------------------------------------------------------------------------
