@@ -20,3 +20,11 @@ from .swa_oracle import (  # noqa: F401
     oracle_prefill,
     oracle_threads,
 )
+from .rope_oracle import (  # noqa: F401
+    oracle_decode_rope,
+    oracle_fwd_rope,
+    oracle_prefill_rope,
+    oracle_rope_qknorm,
+    oracle_rope_qknorm_bwd,
+    rope_angles,
+)
