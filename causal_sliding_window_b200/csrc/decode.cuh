@@ -24,6 +24,7 @@
 
 #include <cuda_bf16.h>
 
+#include "rope.cuh"
 #include "sm100.cuh"
 
 namespace swa {
@@ -50,6 +51,11 @@ struct DecParams {
     float scale_log2;
     int nsplit;                    // splits launched per sequence
     int nsplit_max;                // stride of the partial arrays
+    // kRope: the query is rotated and normalised at its position cache_len[b] - 1 (rope.cuh)
+    const float* rope_cos;         // [max_pos, D/2]
+    const float* rope_sin;
+    int max_pos;
+    float eps;
 };
 
 constexpr int kDecodeThreads = 64;   // threads per CTA: D/8 per pair, so 4 pairs at D = 128 (more CTAs in flight)
@@ -75,7 +81,7 @@ inline int decode_qpt(int kv_group) {
     return 4;
 }
 
-template <int D, int QPT>
+template <int D, int QPT, bool kRope>
 __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecParams p) {
     constexpr int LPH = D / 8;                       // threads per (K/V head, query subgroup) pair
     constexpr int G = kDecodeThreads / LPH;          // pairs per CTA
@@ -107,11 +113,26 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
     const int end = min(start + p.chunk, L);
 
     float qv[QPT][8];
+    int rpos = 0;   // position of the new token (kRope); the same for every thread of the CTA
+    if (kRope) {
+        rpos = L - 1;
+        if (rpos >= p.max_pos) {
+            if (tid == 0 && split == 0) atomicOr(&g_attn_status, kStatusPositionRange);
+            rpos = 0;
+        }
+        rpos = rpos < 0 ? 0 : rpos;
+    }
 #pragma unroll
     for (int a = 0; a < QPT; ++a) {
         const uint4 u = hv[a] ? *reinterpret_cast<const uint4*>(p.q + (size_t(b) * H + hq[a]) * D + c * 8)
                               : make_uint4(0, 0, 0, 0);
         bf16x8_to_f32<D>(u, qv[a]);
+        if (kRope) {   // every thread of the warp takes part (rows are whole groups of D/8 lanes)
+            rope_qknorm8<D>(qv[a], c, p.rope_cos + size_t(rpos) * (D / 2), p.rope_sin + size_t(rpos) * (D / 2),
+                            p.eps, rope_group_mask<D>());
+            // a bf16 activation, as the rotated queries of prefill and training are
+            bf16x8_to_f32<D>(bf16x8_pack(qv[a]), qv[a]);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) qv[a][i] *= p.scale_log2;
     }

@@ -24,6 +24,7 @@
 // only tiles that cut the diagonal or the window's left edge are masked.
 #pragma once
 
+#include "rope.cuh"
 #include "sm100.cuh"
 
 namespace swa {
@@ -484,31 +485,38 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 // ---------------------------------------------------------------------------
 // Chunked prefill, append step: a chunk of Tn tokens' K and V goes to cache slots
-// cache_len[b] .. cache_len[b] + Tn - 1 of each sequence, and the slots after it up to the end of
-// that 128-slot tile are zeroed: they hold no token, and the forward's last key tile reads them
-// (their scores are masked, and zero V rows keep P*V finite whatever the slots held).  Slots at or
-// beyond cap are not written; a chunk that needs them sets kStatusCacheOverflow.
-// One thread per 16 bytes of a (slot, K/V head) row.
+// cache_len[b] + len_off .. cache_len[b] + len_off + Tn - 1 of each sequence, and with tail > 0
+// the slots after it up to the end of that 128-slot tile are zeroed: they hold no token, and the
+// forward's last key tile reads them (their scores are masked, and zero V rows keep P*V finite
+// whatever the slots held).  Slots at or beyond cap are not written; a chunk that needs them
+// sets kStatusCacheOverflow.  kRope: each key is rotated and normalised at its position (its
+// slot) on the way in (rope.cuh).
+// One thread per 16 bytes of a (slot, K/V head) row; a row's threads are consecutive lanes.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kRope>
 __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __restrict__ k_new,
                                                          const __nv_bfloat16* __restrict__ v_new,
                                                          __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
                                                          const int* __restrict__ cache_len, int B, int Tn, int cap,
-                                                         int Hkv) {
+                                                         int Hkv, int len_off, int tail, const float* __restrict__ cs,
+                                                         const float* __restrict__ sn, int max_pos, float eps) {
     constexpr int CPR = D / 8;   // 16-byte chunks per head row
-    const int span = Tn + 128;   // chunk rows plus the largest zeroed tail
+    const int span = Tn + tail;  // chunk rows plus the largest zeroed tail
     const long long total = (long long)B * span * Hkv * CPR;
     const long long stride = (long long)gridDim.x * blockDim.x;
+    const unsigned mask = rope_group_mask<D>();
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
         const int c = int(e % CPR);
         const long long r = e / CPR;
         const int hk = int(r % Hkv);
         const int t = int((r / Hkv) % span);
         const int b = int(r / ((long long)Hkv * span));
-        const long long L = cache_len[b] < 0 ? 0 : cache_len[b];
+        const long long L0 = (long long)cache_len[b] + len_off;
+        if (L0 < 0 && len_off < 0) continue;   // decode of an empty sequence: no slot for the token
+        const long long L = L0 < 0 ? 0 : L0;
         const long long slot = L + t;
         const long long tile_end = (L + Tn + 127) / 128 * 128;
+        // every branch below is uniform over the row's threads (it depends on b, t, hk only)
         if (t >= Tn && slot >= tile_end) continue;
         if (slot >= cap) {
             if (t < Tn) atomicOr(&g_attn_status, kStatusCacheOverflow);
@@ -520,6 +528,16 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
             const size_t src = ((size_t(b) * Tn + t) * Hkv + hk) * D + c * 8;
             kw = *reinterpret_cast<const uint4*>(k_new + src);
             vw = *reinterpret_cast<const uint4*>(v_new + src);
+            if (kRope) {
+                if (slot >= max_pos) {
+                    atomicOr(&g_attn_status, kStatusPositionRange);
+                    continue;
+                }
+                float f[8];
+                bf16x8_unpack(kw, f);
+                rope_qknorm8<D>(f, c, cs + slot * (D / 2), sn + slot * (D / 2), eps, mask);
+                kw = bf16x8_pack(f);
+            }
         }
         *reinterpret_cast<uint4*>(kc + dst) = kw;
         *reinterpret_cast<uint4*>(vc + dst) = vw;

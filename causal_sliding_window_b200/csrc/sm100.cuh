@@ -27,6 +27,7 @@ enum : int {
     kStatusTimeoutSelftest = 16,
     kStatusSmemLayout = 32,   // dynamic shared memory too misaligned for the tile layout
     kStatusCacheOverflow = 64,   // a prefill chunk did not fit in the cache capacity
+    kStatusPositionRange = 128,  // a token position outside the rotary tables
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

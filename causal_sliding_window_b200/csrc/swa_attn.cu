@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <mutex>
 #include <set>
@@ -15,6 +16,7 @@
 #include "bwd.cuh"
 #include "decode.cuh"
 #include "fwd.cuh"
+#include "rope.cuh"
 
 namespace {
 
@@ -202,9 +204,46 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
     return attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, W, scale, stream);
 }
 
-int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
-                 attn_bf16* v_cache, const int32_t* cache_len, attn_bf16* o, float* lse, int B, int Tn, int cap,
-                 int H, int Hkv, int D, int W, float scale, void* stream) {
+// RoPE arguments shared by the fused entry points (null table pointers: no rotation).
+struct RopeArgs {
+    const float* cs = nullptr;
+    const float* sn = nullptr;
+    int max_pos = 0;
+    float eps = 0.f;
+};
+
+static bool valid_rope(const float* cs, const float* sn, int max_pos, float eps) {
+    return cs && sn && aligned16(cs) && aligned16(sn) && max_pos >= 1 && eps >= 0.f && std::isfinite(eps);
+}
+
+// Launches the append kernel: k_new / v_new rows to slots cache_len[b] + len_off + t, tail zeroed
+// up to the 128-slot tile end when tail > 0; keys rotated and normalised when rope.cs is set.
+static int launch_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache, attn_bf16* v_cache,
+                         const int32_t* cache_len, int B, int Tn, int cap, int Hkv, int D, int len_off, int tail,
+                         const RopeArgs& rope, cudaStream_t s) {
+    const long long chunks = (long long)B * (Tn + tail) * Hkv * (D / 8);
+    const long long blocks = std::min<long long>((chunks + 255) / 256, 148LL * 16);
+    const auto* kn = reinterpret_cast<const __nv_bfloat16*>(k_new);
+    const auto* vn = reinterpret_cast<const __nv_bfloat16*>(v_new);
+    auto* kc = reinterpret_cast<__nv_bfloat16*>(k_cache);
+    auto* vc = reinterpret_cast<__nv_bfloat16*>(v_cache);
+    const bool r = rope.cs != nullptr;
+#define SWA_APPEND(DD, RR)                                                                                    \
+    swa_append_kernel<DD, RR><<<unsigned(blocks), 256, 0, s>>>(kn, vn, kc, vc, cache_len, B, Tn, cap, Hkv, len_off, \
+                                                               tail, rope.cs, rope.sn, rope.max_pos, rope.eps)
+    if (D == 128) {
+        if (r) SWA_APPEND(128, true); else SWA_APPEND(128, false);
+    } else {
+        if (r) SWA_APPEND(64, true); else SWA_APPEND(64, false);
+    }
+#undef SWA_APPEND
+    return launch_status();
+}
+
+static int prefill_impl(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                        attn_bf16* v_cache, const int32_t* cache_len, attn_bf16* o, float* lse, int B, int Tn,
+                        int cap, int H, int Hkv, int D, int W, float scale, const RopeArgs& rope,
+                        attn_bf16* q_rot, void* stream) {
     if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_len || !o || !lse) return ATTN_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k_new, v_new, k_cache, v_cache, o, lse};
     for (const void* ptr : ptrs)
@@ -216,22 +255,29 @@ int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_
     const long long n_items = (long long)n_qblk * B * H;
     if (n_items > 0x7fffffffLL || (long long)B * (Tn + 128) * Hkv * (D / 8) > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // 0. with RoPE: the chunk's queries rotated and normalised at positions cache_len[b] + t
+    const attn_bf16* q_in = q;
+    if (rope.cs) {
+        const long long rows = (long long)B * Tn * H * (D / 8);
+        const unsigned blocks = unsigned(std::min<long long>((rows + 255) / 256, 148LL * 16));
+        const auto* x = reinterpret_cast<const __nv_bfloat16*>(q);
+        auto* y = reinterpret_cast<__nv_bfloat16*>(q_rot);
+        if (D == 128)
+            swa_rope_qknorm_kernel<128, false><<<blocks, 256, 0, s>>>(x, nullptr, y, B, Tn, H, cache_len, rope.cs,
+                                                                       rope.sn, rope.max_pos, rope.eps);
+        else
+            swa_rope_qknorm_kernel<64, false><<<blocks, 256, 0, s>>>(x, nullptr, y, B, Tn, H, cache_len, rope.cs,
+                                                                      rope.sn, rope.max_pos, rope.eps);
+        if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
+        q_in = q_rot;
+    }
     // 1. append the chunk's K / V (and zero the rest of its last 128-slot tile)
-    const long long chunks = (long long)B * (Tn + 128) * Hkv * (D / 8);
-    const long long blocks = std::min<long long>((chunks + 255) / 256, 148LL * 16);
-    const auto* kn = reinterpret_cast<const __nv_bfloat16*>(k_new);
-    const auto* vn = reinterpret_cast<const __nv_bfloat16*>(v_new);
-    auto* kc = reinterpret_cast<__nv_bfloat16*>(k_cache);
-    auto* vc = reinterpret_cast<__nv_bfloat16*>(v_cache);
-    if (D == 128)
-        swa_append_kernel<128><<<unsigned(blocks), 256, 0, s>>>(kn, vn, kc, vc, cache_len, B, Tn, cap, Hkv);
-    else
-        swa_append_kernel<64><<<unsigned(blocks), 256, 0, s>>>(kn, vn, kc, vc, cache_len, B, Tn, cap, Hkv);
-    if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
+    if (launch_append(k_new, v_new, k_cache, v_cache, cache_len, B, Tn, cap, Hkv, D, 0, 128, rope, s) != ATTN_OK)
+        return ATTN_ERR_LAUNCH;
     // 2. the forward of the chunk's queries at absolute positions cache_len[b] + t over the cache
     const long long grid = n_items < sm_count() ? n_items : sm_count();
     CUtensorMap mq, mk, mv;
-    if (!make_bthd_map(&mq, q, B, Tn, H, D) || !make_bthd_map(&mk, k_cache, B, cap, Hkv, D) ||
+    if (!make_bthd_map(&mq, q_in, B, Tn, H, D) || !make_bthd_map(&mk, k_cache, B, cap, Hkv, D) ||
         !make_bthd_map(&mv, v_cache, B, cap, Hkv, D))
         return ATTN_ERR_LAUNCH;
     FwdParams p;
@@ -256,6 +302,81 @@ int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_
         swa_fwd_kernel<64, true><<<unsigned(grid), FwdCfg<64>::THREADS, FwdCfg<64>::SMEM, s>>>(mq, mk, mv, p);
     }
     return launch_status();
+}
+
+int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                 attn_bf16* v_cache, const int32_t* cache_len, attn_bf16* o, float* lse, int B, int Tn, int cap,
+                 int H, int Hkv, int D, int W, float scale, void* stream) {
+    return prefill_impl(q, k_new, v_new, k_cache, v_cache, cache_len, o, lse, B, Tn, cap, H, Hkv, D, W, scale,
+                        RopeArgs{}, nullptr, stream);
+}
+
+size_t attn_prefill_rope_workspace_bytes(int B, int Tn, int H, int D) {
+    if (B < 1 || Tn < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+    return align256(size_t(B) * Tn * H * D * 2);
+}
+
+int attn_prefill_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                      attn_bf16* v_cache, const int32_t* cache_len, const float* rope_cos, const float* rope_sin,
+                      int max_pos, float eps, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                      int Tn, int cap, int H, int Hkv, int D, int W, float scale, void* stream) {
+    if (!valid_rope(rope_cos, rope_sin, max_pos, eps) || !workspace) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_prefill_rope_workspace_bytes(B, Tn, H, D);
+    if (need != 0 && ws_bytes < need) return ATTN_ERR_WORKSPACE;
+    RopeArgs r;
+    r.cs = rope_cos;
+    r.sn = rope_sin;
+    r.max_pos = max_pos;
+    r.eps = eps;
+    return prefill_impl(q, k_new, v_new, k_cache, v_cache, cache_len, o, lse, B, Tn, cap, H, Hkv, D, W, scale, r,
+                        static_cast<attn_bf16*>(workspace), stream);
+}
+
+int attn_rope_tables(float* rope_cos, float* rope_sin, int max_pos, int D, double base, void* stream) {
+    if (!rope_cos || !rope_sin || !aligned16(rope_cos) || !aligned16(rope_sin)) return ATTN_ERR_INVALID_ARG;
+    if (max_pos < 1 || D < 2 || D % 2 != 0 || !(base > 1.0) || !std::isfinite(base)) return ATTN_ERR_INVALID_ARG;
+    const long long total = (long long)max_pos * (D / 2);
+    const unsigned blocks = unsigned(std::min<long long>((total + 255) / 256, 148LL * 16));
+    swa_rope_tables_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(rope_cos, rope_sin, max_pos,
+                                                                                       D / 2, base);
+    return launch_status();
+}
+
+static int rope_qknorm_impl(const attn_bf16* x, const attn_bf16* dy, attn_bf16* y, const int32_t* pos0,
+                            const float* rope_cos, const float* rope_sin, int max_pos, int B, int T, int H, int D,
+                            float eps, bool bwd, void* stream) {
+    if (!x || !y || (bwd && !dy) || !aligned16(x) || !aligned16(y) || (bwd && !aligned16(dy)))
+        return ATTN_ERR_INVALID_ARG;
+    if (pos0 && (reinterpret_cast<uintptr_t>(pos0) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!valid_rope(rope_cos, rope_sin, max_pos, eps) || B < 1 || T < 1 || H < 1) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    const long long rows = (long long)B * T * H * (D / 8);
+    const unsigned blocks = unsigned(std::min<long long>((rows + 255) / 256, 148LL * 16));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const auto* xx = reinterpret_cast<const __nv_bfloat16*>(x);
+    const auto* gg = reinterpret_cast<const __nv_bfloat16*>(dy);
+    auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+#define SWA_ROPE(DD, BB) \
+    swa_rope_qknorm_kernel<DD, BB><<<blocks, 256, 0, s>>>(xx, gg, yy, B, T, H, pos0, rope_cos, rope_sin, max_pos, eps)
+    if (D == 128) {
+        if (bwd) SWA_ROPE(128, true); else SWA_ROPE(128, false);
+    } else {
+        if (bwd) SWA_ROPE(64, true); else SWA_ROPE(64, false);
+    }
+#undef SWA_ROPE
+    return launch_status();
+}
+
+int attn_rope_qknorm(const attn_bf16* x, attn_bf16* y, const int32_t* pos0, const float* rope_cos,
+                     const float* rope_sin, int max_pos, int B, int T, int H, int D, float eps, void* stream) {
+    return rope_qknorm_impl(x, nullptr, y, pos0, rope_cos, rope_sin, max_pos, B, T, H, D, eps, false, stream);
+}
+
+int attn_rope_qknorm_bwd(const attn_bf16* x, const attn_bf16* dy, attn_bf16* dx, const int32_t* pos0,
+                         const float* rope_cos, const float* rope_sin, int max_pos, int B, int T, int H, int D,
+                         float eps, void* stream) {
+    return rope_qknorm_impl(x, dy, dx, pos0, rope_cos, rope_sin, max_pos, B, T, H, D, eps, true, stream);
 }
 
 // Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128).
@@ -377,9 +498,9 @@ size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
     return attn_decode_gqa_workspace_bytes(B, cap, H, H, D);
 }
 
-int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
-                    const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
-                    int cap, int H, int Hkv, int D, int W, float scale, void* stream) {
+static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                       const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                       int cap, int H, int Hkv, int D, int W, float scale, const RopeArgs& rope, void* stream) {
     if (!q || !k_cache || !v_cache || !cache_len || !o || !workspace) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
@@ -415,11 +536,21 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
     p.scale_log2 = scale * 1.4426950408889634f;
     p.nsplit = (span + g.chunk - 1) / g.chunk;
     p.nsplit_max = nsm;
+    p.rope_cos = rope.cs;
+    p.rope_sin = rope.sn;
+    p.max_pos = rope.max_pos;
+    p.eps = rope.eps;
     const int pairs_per_cta = kDecodeThreads / (D / 8);
     const int threads = ((std::min(Hkv * g.nsub, pairs_per_cta) * (D / 8)) + 31) / 32 * 32;
     dim3 grid(p.nsplit, B, g.nzg);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-#define SWA_DECODE_LAUNCH(DD, QQ) swa_decode_kernel<DD, QQ><<<grid, threads, 0, s>>>(p)
+#define SWA_DECODE_LAUNCH(DD, QQ)                                      \
+    do {                                                               \
+        if (rope.cs)                                                   \
+            swa_decode_kernel<DD, QQ, true><<<grid, threads, 0, s>>>(p);  \
+        else                                                           \
+            swa_decode_kernel<DD, QQ, false><<<grid, threads, 0, s>>>(p); \
+    } while (0)
     if (D == 128) {
         switch (g.qpt) {
             case 1: SWA_DECODE_LAUNCH(128, 1); break;
@@ -437,6 +568,39 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
     }
 #undef SWA_DECODE_LAUNCH
     return launch_status();
+}
+
+int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
+                    const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                    int cap, int H, int Hkv, int D, int W, float scale, void* stream) {
+    return decode_impl(q, k_cache, v_cache, cache_len, o, lse, workspace, ws_bytes, B, cap, H, Hkv, D, W, scale,
+                       RopeArgs{}, stream);
+}
+
+int attn_decode_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                     attn_bf16* v_cache, const int32_t* cache_len, const float* rope_cos, const float* rope_sin,
+                     int max_pos, float eps, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                     int cap, int H, int Hkv, int D, int W, float scale, void* stream) {
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new) || !valid_rope(rope_cos, rope_sin, max_pos, eps))
+        return ATTN_ERR_INVALID_ARG;
+    if (!k_cache || !v_cache || !cache_len || !aligned16(k_cache) || !aligned16(v_cache)) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, cap, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (ws_bytes < attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)) return ATTN_ERR_WORKSPACE;
+    RopeArgs r;
+    r.cs = rope_cos;
+    r.sn = rope_sin;
+    r.max_pos = max_pos;
+    r.eps = eps;
+    // 1. the new token's key (rotated, normalised) and value into slot cache_len[b] - 1
+    if (launch_append(k_new, v_new, k_cache, v_cache, cache_len, B, 1, cap, Hkv, D, -1, 0, r,
+                      reinterpret_cast<cudaStream_t>(stream)) != ATTN_OK)
+        return ATTN_ERR_LAUNCH;
+    // 2. decode with the query rotated and normalised inside the kernel
+    return decode_impl(q, k_cache, v_cache, cache_len, o, lse, workspace, ws_bytes, B, cap, H, Hkv, D, W, scale, r,
+                       stream);
 }
 
 int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache, const int32_t* cache_len,
@@ -478,6 +642,7 @@ int attn_device_status(int clear) {
         if (cudaMemcpyToSymbol(swa::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
     }
     if (v & swa::kStatusCacheOverflow) return ATTN_ERR_CACHE_OVERFLOW;
+    if (v & swa::kStatusPositionRange) return ATTN_ERR_POSITION_RANGE;
     return v ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
 }
 
@@ -496,6 +661,7 @@ const char* attn_status_string(int status) {
         case ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case ATTN_ERR_WORKSPACE: return "workspace too small";
         case ATTN_ERR_CACHE_OVERFLOW: return "cache capacity exceeded";
+        case ATTN_ERR_POSITION_RANGE: return "token position outside the rotary tables";
         default: return "unknown status";
     }
 }

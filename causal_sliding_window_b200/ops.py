@@ -11,7 +11,11 @@ Low-level calls (caller provides every buffer, torch tensors on one CUDA device)
   attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W, scale=None, stream=None)
 K and V (and dK, dV, the caches) may have fewer heads than Q (grouped K/V heads, Hkv dividing H);
 the calls then go to the C entry points' _gqa forms.
-Convenience wrappers that allocate outputs: forward, backward, decode.
+Rotary embedding + QK norm (the attention prologue): attn_rope_tables, attn_rope_qknorm,
+attn_rope_qknorm_bwd, attn_prefill_rope, attn_decode_rope; cos / sin tables are float32
+[max_pos, D/2] CUDA tensors.
+Convenience wrappers that allocate outputs: forward, backward, decode, rope_tables, prefill_rope,
+decode_rope.
 """
 from __future__ import annotations
 
@@ -26,7 +30,8 @@ LIB_PATH = os.path.join(_HERE, "libswa_b200.so")
 
 ATTN_OK = 0
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported configuration", -3: "kernel launch failed",
-          -4: "device wait timed out", -5: "workspace too small", -6: "cache capacity exceeded"}
+          -4: "device wait timed out", -5: "workspace too small", -6: "cache capacity exceeded",
+          -7: "token position outside the rotary tables"}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m causal_sliding_window_b200.build`")
@@ -55,6 +60,19 @@ _lib.attn_prefill.argtypes = [_p] * 8 + [_i, _i, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_prefill.restype = _i
 _lib.attn_decode_noalloc.argtypes = [_p] * 6 + [_i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode_noalloc.restype = _i
+_d = ctypes.c_double
+_lib.attn_rope_tables.argtypes = [_p, _p, _i, _i, _d, _p]
+_lib.attn_rope_tables.restype = _i
+_lib.attn_rope_qknorm.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_rope_qknorm.restype = _i
+_lib.attn_rope_qknorm_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _f, _p]
+_lib.attn_rope_qknorm_bwd.restype = _i
+_lib.attn_prefill_rope_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.attn_prefill_rope_workspace_bytes.restype = _sz
+_lib.attn_prefill_rope.argtypes = [_p] * 8 + [_i, _f, _p, _p, _p, _sz] + [_i] * 7 + [_f, _p]
+_lib.attn_prefill_rope.restype = _i
+_lib.attn_decode_rope.argtypes = [_p] * 8 + [_i, _f, _p, _p, _p, _sz] + [_i] * 6 + [_f, _p]
+_lib.attn_decode_rope.restype = _i
 _lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
 _lib.attn_bwd_set_profile_events.restype = _i
 _lib.attn_device_status.argtypes = [_i]
@@ -66,7 +84,8 @@ _lib.attn_status_string.restype = ctypes.c_char_p
 
 EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_gqa",
             "attn_decode_workspace_bytes", "attn_decode_gqa_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
-            "attn_status_string"]
+            "attn_status_string", "attn_rope_tables", "attn_rope_qknorm", "attn_rope_qknorm_bwd",
+            "attn_prefill_rope_workspace_bytes", "attn_prefill_rope", "attn_decode_rope"]
 
 
 class AttnError(RuntimeError):
@@ -264,4 +283,117 @@ def decode(q, k_cache, v_cache, cache_len, W: int, scale=None, stream=None, work
     if workspace is None:
         workspace = decode_workspace(B, cap, H, D, q.device, Hkv=k_cache.shape[2])
     attn_decode(q, k_cache, v_cache, cache_len, o, lse, workspace, W, scale, stream)
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Rotary embedding + QK norm
+# ---------------------------------------------------------------------------
+
+def _tables(cos, sin, D):
+    if (cos.dtype != torch.float32 or sin.dtype != torch.float32 or not cos.is_cuda or not cos.is_contiguous()
+            or not sin.is_contiguous() or cos.dim() != 2 or cos.shape != sin.shape or cos.shape[1] != D // 2):
+        raise ValueError("rotary tables must be contiguous float32 CUDA tensors [max_pos, D/2]")
+    return cos.shape[0]
+
+
+def _pos0(pos0, B):
+    if pos0 is None:
+        return None
+    if pos0.dtype != torch.int32 or tuple(pos0.shape) != (B,) or not pos0.is_cuda:
+        raise ValueError("pos0 must be an int32 CUDA tensor of shape [B]")
+    return pos0
+
+
+def attn_rope_tables(cos, sin, base: float = 10000.0, stream=None):
+    """Fill cos / sin [max_pos, D/2] for th_i = base^(-2i/D)."""
+    D = 2 * cos.shape[1]
+    max_pos = _tables(cos, sin, D)
+    _check(_lib.attn_rope_tables(_ptr(cos), _ptr(sin), max_pos, D, float(base), _stream(stream)), "attn_rope_tables")
+
+
+def rope_tables(max_pos: int, D: int, device, base: float = 10000.0, stream=None):
+    cos = torch.empty((max_pos, D // 2), dtype=torch.float32, device=device)
+    sin = torch.empty_like(cos)
+    attn_rope_tables(cos, sin, base, stream)
+    return cos, sin
+
+
+def attn_rope_qknorm(x, y, cos, sin, eps: float, pos0=None, stream=None):
+    B, T, H, D = _bthd(x, y)
+    max_pos = _tables(cos, sin, D)
+    _check(_lib.attn_rope_qknorm(_ptr(x), _ptr(y), _ptr(_pos0(pos0, B)), _ptr(cos), _ptr(sin), max_pos, B, T, H, D,
+                                 float(eps), _stream(stream)), "attn_rope_qknorm")
+
+
+def attn_rope_qknorm_bwd(x, dy, dx, cos, sin, eps: float, pos0=None, stream=None):
+    B, T, H, D = _bthd(x, dy, dx)
+    max_pos = _tables(cos, sin, D)
+    _check(_lib.attn_rope_qknorm_bwd(_ptr(x), _ptr(dy), _ptr(dx), _ptr(_pos0(pos0, B)), _ptr(cos), _ptr(sin),
+                                     max_pos, B, T, H, D, float(eps), _stream(stream)), "attn_rope_qknorm_bwd")
+
+
+def attn_prefill_rope_workspace_bytes(B: int, Tn: int, H: int, D: int) -> int:
+    return int(_lib.attn_prefill_rope_workspace_bytes(B, Tn, H, D))
+
+
+def attn_prefill_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps: float, o, lse, workspace, W: int,
+                      scale=None, stream=None):
+    B, Tn, H, D = _bthd(q, o)
+    Hkv = _kv_heads((B, Tn, H, D), k_new, v_new)
+    Bc, cap, Hc, Dc = _bthd(k_cache, v_cache)
+    if (Bc, Hc, Dc) != (B, Hkv, D):
+        raise ValueError("caches must be [B, cap, Hkv, D] matching k_new")
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or not cache_len.is_cuda:
+        raise ValueError("cache_len must be an int32 CUDA tensor of shape [B]")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Tn) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, Tn] tensor")
+    max_pos = _tables(cos, sin, D)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.attn_prefill_rope(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len),
+                                  _ptr(cos), _ptr(sin), max_pos, float(eps), _ptr(o), _ptr(lse), _ptr(workspace),
+                                  ws_bytes, B, Tn, cap, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)),
+           "attn_prefill_rope")
+
+
+def prefill_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps: float, W: int, scale=None, stream=None):
+    """attn_prefill_rope with freshly allocated outputs and workspace; returns (o, lse)."""
+    B, Tn, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Tn), dtype=torch.float32, device=q.device)
+    ws = torch.empty(attn_prefill_rope_workspace_bytes(B, Tn, H, D), dtype=torch.uint8, device=q.device)
+    attn_prefill_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps, o, lse, ws, W, scale, stream)
+    return o, lse
+
+
+def attn_decode_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps: float, o, lse, workspace, W: int,
+                     scale=None, stream=None):
+    B, cap, Hkv, D = _bthd(k_cache, v_cache)
+    H = q.shape[1] if q.dim() == 3 else -1
+    if (tuple(q.shape) != (B, H, D) or tuple(o.shape) != (B, H, D) or q.dtype != torch.bfloat16 or H % Hkv != 0
+            or not q.is_contiguous() or not o.is_contiguous()):
+        raise ValueError("q and o must be contiguous bf16 [B, H, D] with the caches' head count dividing H")
+    for t in (k_new, v_new):
+        if tuple(t.shape) != (B, Hkv, D) or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("k_new and v_new must be contiguous bf16 [B, Hkv, D]")
+    if cache_len.dtype != torch.int32 or tuple(cache_len.shape) != (B,) or not cache_len.is_cuda:
+        raise ValueError("cache_len must be an int32 CUDA tensor of shape [B]")
+    max_pos = _tables(cos, sin, D)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.attn_decode_rope(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len),
+                                 _ptr(cos), _ptr(sin), max_pos, float(eps), _ptr(o), _ptr(lse), _ptr(workspace),
+                                 ws_bytes, B, cap, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)),
+           "attn_decode_rope")
+
+
+def decode_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps: float, W: int, scale=None, stream=None,
+                workspace=None):
+    """attn_decode_rope with freshly allocated outputs (and workspace unless given); returns (o, lse)."""
+    B, H, D = q.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    o = torch.empty((B, H, D), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(B, cap, H, D, q.device, Hkv=Hkv)
+    attn_decode_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps, o, lse, workspace, W, scale, stream)
     return o, lse

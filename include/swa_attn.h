@@ -37,7 +37,8 @@
  *    correct use never produces), the kernel stops early and records a flag
  *    that attn_device_status() reports as ATTN_ERR_DEVICE_TIMEOUT.  A prefill
  *    chunk that does not fit its cache is reported there as
- *    ATTN_ERR_CACHE_OVERFLOW.
+ *    ATTN_ERR_CACHE_OVERFLOW, a token position outside the rotary tables as
+ *    ATTN_ERR_POSITION_RANGE.
  */
 #ifndef SWA_ATTN_H
 #define SWA_ATTN_H
@@ -58,7 +59,8 @@ typedef enum {
     ATTN_ERR_LAUNCH = -3,
     ATTN_ERR_DEVICE_TIMEOUT = -4,
     ATTN_ERR_WORKSPACE = -5,
-    ATTN_ERR_CACHE_OVERFLOW = -6
+    ATTN_ERR_CACHE_OVERFLOW = -6,
+    ATTN_ERR_POSITION_RANGE = -7
 } attn_status;
 
 /*
@@ -106,6 +108,63 @@ int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, att
 int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
                  attn_bf16* v_cache, const int32_t* cache_len, attn_bf16* o, float* lse, int B, int Tn,
                  int cap, int H, int Hkv, int D, int W, float scale, void* stream);
+
+/*
+ * Rotary embedding + QK norm, the prologue of attention in the GPT model (apidog guide,
+ * section 1 "GPT model", architecture features: rotary embeddings, QK normalisation; an
+ * RMSNorm without learnable parameters).  The pages give no formula; the reading used here:
+ * for a head vector x at position pos, the pairs (x[i], x[i + D/2]), i < D/2, are rotated by
+ * pos * th_i,  r1 = x1 cos - x2 sin,  r2 = x1 sin + x2 cos  (RoFormer), and
+ * y = r / sqrt(mean(r^2) + eps).  cos / sin come from fp32 tables [max_pos, D/2] that the
+ * caller owns (row pos, column i = angle pos * th_i); eps >= 0 and finite; max_pos >= 1.
+ * A token whose position is outside [0, max_pos) is not written, and attn_device_status()
+ * reports ATTN_ERR_POSITION_RANGE.
+ */
+
+/* Fills the tables for th_i = base^(-2i/D) (base > 1), angles in double precision.
+ *   rope_cos, rope_sin  [max_pos, D/2] fp32, written (D even, any size here). */
+int attn_rope_tables(float* rope_cos, float* rope_sin, int max_pos, int D, double base, void* stream);
+
+/* y[b,t,h,:] = rotate-and-normalise x[b,t,h,:] at position pos0[b] + t (pos0 NULL: t).
+ *   x, y  [B, T, H, D] bf16 (y may be x: in place).  pos0  [B] int32 in device memory, or NULL. */
+int attn_rope_qknorm(const attn_bf16* x, attn_bf16* y, const int32_t* pos0, const float* rope_cos,
+                     const float* rope_sin, int max_pos, int B, int T, int H, int D, float eps, void* stream);
+
+/* Backward of attn_rope_qknorm: dx = J^T dy at x (same positions), recomputing the rotation:
+ * with r = rope(x) and s = (mean(r^2) + eps)^(-1/2), dr = s dy - (s^3 / D) r (dy . r) and dx
+ * is dr rotated back.   x, dy, dx  [B, T, H, D] bf16 (dx may be dy). */
+int attn_rope_qknorm_bwd(const attn_bf16* x, const attn_bf16* dy, attn_bf16* dx, const int32_t* pos0,
+                         const float* rope_cos, const float* rope_sin, int max_pos, int B, int T, int H, int D,
+                         float eps, void* stream);
+
+/* Bytes of workspace attn_prefill_rope needs (the chunk's rotated queries, bf16). */
+size_t attn_prefill_rope_workspace_bytes(int B, int Tn, int H, int D);
+
+/*
+ * attn_prefill with the prologue: q, k_new are the chunk's queries and keys before rotation and
+ * norm.  Token t of sequence b is at position cache_len[b] + t: its query is rotated and
+ * normalised into the workspace (at least attn_prefill_rope_workspace_bytes bytes, 256-byte
+ * aligned), its key on the way into the cache (the append writes the rotated, normalised key),
+ * and the forward runs as in attn_prefill.  Tables and eps as attn_rope_qknorm.
+ */
+int attn_prefill_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                      attn_bf16* v_cache, const int32_t* cache_len, const float* rope_cos, const float* rope_sin,
+                      int max_pos, float eps, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                      int Tn, int cap, int H, int Hkv, int D, int W, float scale, void* stream);
+
+/*
+ * One decode step with the prologue and append: the new token of sequence b sits in slot
+ * cache_len[b] - 1 (its position; cache_len counts it, each in [1, cap]).  Its key k_new
+ * [B, Hkv, D] is rotated, normalised and written there with its value v_new [B, Hkv, D];
+ * its query q [B, H, D] is rotated and normalised inside the decode kernel, which then
+ * attends as attn_decode_gqa.  workspace: attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)
+ * bytes, zero-filled before first use (every call leaves it zeroed).  Tables and eps as
+ * attn_rope_qknorm.
+ */
+int attn_decode_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
+                     attn_bf16* v_cache, const int32_t* cache_len, const float* rope_cos, const float* rope_sin,
+                     int max_pos, float eps, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
+                     int cap, int H, int Hkv, int D, int W, float scale, void* stream);
 
 /* Bytes of workspace attn_bwd needs: fp32 rows of lse*log2(e) and Delta, [B*H, T rounded up
  * to 128] each (256-byte padded). */

@@ -27,4 +27,5 @@ from .rope_oracle import (  # noqa: F401
     oracle_rope_qknorm,
     oracle_rope_qknorm_bwd,
     rope_angles,
+    round_bf16,
 )

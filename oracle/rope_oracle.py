@@ -18,6 +18,9 @@ this module takes the plainest reading, written out here:
 A rotation keeps the vector's length, so the two steps commute; the order is not
 a reading.  The position of a token is its index in its sequence (training and
 prefill: cache_len[b] + t; decode: cache_len[b] - 1, the new token's slot).
+The model's activations are bf16, so the rotated, normalised q and k that attention
+reads are bf16 values: the compositions below round them (to nearest, ties to even)
+before the attention step.
 
 Functions take bf16 bit patterns (uint16) or float64 and return float64.
 """
@@ -35,6 +38,21 @@ def _f64(x):
     if x.dtype != np.float64:
         raise TypeError("inputs must be bf16 bits (uint16) or float64")
     return x
+
+
+def round_bf16(x):
+    """x (float64) rounded to the nearest bf16 value, ties to even.  The float64 -> float32 step
+    rounds to odd (truncate, then set the last bit when inexact), so the final rounding to bf16's
+    8 significant bits is the correct one (no double rounding)."""
+    x = np.asarray(x, dtype=np.float64)
+    f = x.astype(np.float32)
+    over = np.abs(f.astype(np.float64)) > np.abs(x)
+    f = np.where(over, np.nextafter(f, np.float32(0)), f).astype(np.float32)   # truncated toward zero
+    inexact = (f.astype(np.float64) != x).astype(np.uint64)
+    b = np.ascontiguousarray(f).view(np.uint32).astype(np.uint64) | inexact
+    lsb = (b >> 16) & 1
+    r = ((b + 0x7FFF + lsb) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
 def rope_angles(pos, D: int, base: float = 10000.0):
@@ -78,11 +96,11 @@ def oracle_rope_qknorm_bwd(x, pos, dy, eps: float, base: float = 10000.0):
 
 def oracle_fwd_rope(q, k, v, W: int, eps: float, base: float = 10000.0, scale: float | None = None):
     """Training forward with the prologue: attention of rope_qknorm(q), rope_qknorm(k) (token t of
-    every sequence at position t) and v.  Returns (o, lse) float64."""
+    every sequence at position t, rounded to bf16) and v.  Returns (o, lse) float64."""
     T = np.asarray(q).shape[1]
     pos = np.arange(T)[None, :]
-    qr = oracle_rope_qknorm(q, pos, eps, base)
-    kr = oracle_rope_qknorm(k, pos, eps, base)
+    qr = round_bf16(oracle_rope_qknorm(q, pos, eps, base))
+    kr = round_bf16(oracle_rope_qknorm(k, pos, eps, base))
     return oracle_fwd(qr, kr, _f64(v), W, scale)
 
 
@@ -94,8 +112,8 @@ def oracle_prefill_rope(q, k_new, v_new, k_cache, v_cache, cache_len, W: int, ep
     Returns (o, lse, k_cache_after, v_cache_after) float64."""
     Tn = np.asarray(q).shape[1]
     pos = np.asarray(cache_len, dtype=np.int64)[:, None] + np.arange(Tn)[None, :]
-    qr = oracle_rope_qknorm(q, pos, eps, base)
-    kr = oracle_rope_qknorm(k_new, pos, eps, base)
+    qr = round_bf16(oracle_rope_qknorm(q, pos, eps, base))
+    kr = round_bf16(oracle_rope_qknorm(k_new, pos, eps, base))
     return oracle_prefill(qr, kr, _f64(v_new), _f64(k_cache), _f64(v_cache), cache_len, W, scale)
 
 
@@ -108,8 +126,8 @@ def oracle_decode_rope(q, k_new, v_new, k_cache, v_cache, cache_len, W: int, eps
     Returns (o, lse, k_cache_after, v_cache_after) float64."""
     cl = np.asarray(cache_len, dtype=np.int64)
     pos = cl - 1
-    qr = oracle_rope_qknorm(np.asarray(q)[:, None], pos[:, None], eps, base)[:, 0]
-    kr = oracle_rope_qknorm(np.asarray(k_new)[:, None], pos[:, None], eps, base)[:, 0]
+    qr = round_bf16(oracle_rope_qknorm(np.asarray(q)[:, None], pos[:, None], eps, base)[:, 0])
+    kr = round_bf16(oracle_rope_qknorm(np.asarray(k_new)[:, None], pos[:, None], eps, base)[:, 0])
     kc, vc = _f64(k_cache).copy(), _f64(v_cache).copy()
     vn = _f64(v_new)
     for b in range(len(cl)):

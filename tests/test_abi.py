@@ -167,3 +167,47 @@ def test_prefill_argument_checks():
     assert call(args(D=96)) == ERR_UNSUPPORTED
     assert ops.attn_status_string(-6) == "cache capacity exceeded"
 
+
+
+def test_rope_argument_checks():
+    """Each rotary entry point rejects bad arguments before launching anything."""
+    lib = ops._lib
+    # tables: pointers, sizes, base
+    assert lib.attn_rope_tables(None, A, 16, 128, 10000.0, None) == ERR_INVALID
+    assert lib.attn_rope_tables(A, A + 4, 16, 128, 10000.0, None) == ERR_INVALID   # misaligned
+    assert lib.attn_rope_tables(A, A, 0, 128, 10000.0, None) == ERR_INVALID
+    assert lib.attn_rope_tables(A, A, 16, 127, 10000.0, None) == ERR_INVALID       # odd D
+    assert lib.attn_rope_tables(A, A, 16, 128, 1.0, None) == ERR_INVALID           # base must exceed 1
+    assert lib.attn_rope_tables(A, A, 16, 128, float("nan"), None) == ERR_INVALID
+    # rotate-and-normalise (forward and backward)
+    args = dict(pos0=None, cs=A, sn=A, max_pos=64, B=2, T=8, H=3, D=128, eps=1e-6)
+    fwd = lambda **kw: (lambda a: lib.attn_rope_qknorm(A, A, a["pos0"], a["cs"], a["sn"], a["max_pos"], a["B"],  # noqa: E731
+                                                        a["T"], a["H"], a["D"], a["eps"], None))(dict(args, **kw))
+    bwd = lambda **kw: (lambda a: lib.attn_rope_qknorm_bwd(A, A, A, a["pos0"], a["cs"], a["sn"], a["max_pos"],  # noqa: E731
+                                                            a["B"], a["T"], a["H"], a["D"], a["eps"], None))(dict(args, **kw))
+    for call in (fwd, bwd):
+        assert call(cs=None) == ERR_INVALID
+        assert call(max_pos=0) == ERR_INVALID
+        assert call(eps=-1.0) == ERR_INVALID
+        assert call(eps=float("inf")) == ERR_INVALID
+        assert call(pos0=A + 2) == ERR_INVALID
+        assert call(B=0) == ERR_INVALID
+        assert call(D=96) == ERR_UNSUPPORTED
+    assert lib.attn_rope_qknorm_bwd(A, None, A, None, A, A, 64, 2, 8, 3, 128, 1e-6, None) == ERR_INVALID
+    # prefill with the prologue: workspace size is checked first
+    assert ops.attn_prefill_rope_workspace_bytes(2, 77, 4, 128) == (2 * 77 * 4 * 128 * 2 + 255) // 256 * 256
+    assert ops.attn_prefill_rope_workspace_bytes(2, 77, 4, 96) == 0
+    need = ops.attn_prefill_rope_workspace_bytes(2, 16, 4, 128)
+    pre = lambda ws_bytes, ws=A, cs=A, eps=1e-6: lib.attn_prefill_rope(  # noqa: E731
+        A, A, A, A, A, A, cs, A, 64, eps, A, A, ws, ws_bytes, 2, 16, 64, 4, 2, 128, 8, 0.1, None)
+    assert pre(need - 1) == ERR_WORKSPACE
+    assert pre(need, ws=A + 16) == ERR_INVALID      # workspace must be 256-byte aligned
+    assert pre(need, cs=None) == ERR_INVALID
+    assert pre(need, eps=-0.5) == ERR_INVALID
+    # decode with the prologue: grouped workspace size, new token's K / V present
+    dneed = ops.attn_decode_gqa_workspace_bytes(2, 64, 4, 2, 128)
+    dec_r = lambda ws_bytes, kn=A, Hkv=2: lib.attn_decode_rope(  # noqa: E731
+        A, kn, A, A, A, A, A, A, 64, 1e-6, A, A, A, ws_bytes, 2, 64, 4, Hkv, 128, 8, 0.1, None)
+    assert dec_r(dneed - 1) == ERR_WORKSPACE
+    assert dec_r(dneed, kn=None) == ERR_INVALID
+    assert dec_r(dneed, Hkv=3) == ERR_INVALID        # 3 does not divide 4

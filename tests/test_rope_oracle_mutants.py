@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 
 import oracle
+from oracle import round_bf16
 from tests.test_rope_oracle_pins import complex_reference
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rope_oracle.py")
@@ -64,7 +65,7 @@ def _pins_hold(m) -> bool:
     # the appended key sits at its position: rotate-and-normalise of k_new at cache_len - 1
     _, _, kc_after, _ = m.oracle_decode_rope(q, kn, vn, kc, vc, lens, W, eps)
     for b in range(B):
-        want = complex_reference(kn[b][None, None], [[lens[b] - 1]], eps)[0, 0]
+        want = round_bf16(complex_reference(kn[b][None, None], [[lens[b] - 1]], eps)[0, 0])
         if not np.allclose(kc_after[b, lens[b] - 1], want, rtol=0, atol=1e-12):
             return False
     return True

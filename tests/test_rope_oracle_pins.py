@@ -13,7 +13,7 @@ import pytest
 
 from causal_sliding_window_b200 import inputs
 from oracle import (oracle_decode_rope, oracle_fwd_rope, oracle_prefill_rope, oracle_rope_qknorm,
-                    oracle_rope_qknorm_bwd)
+                    oracle_rope_qknorm_bwd, round_bf16)
 
 
 def _rng(seed):
@@ -104,7 +104,7 @@ def test_prefill_from_empty_cache_is_the_training_forward():
     o, lse, kc2, _ = oracle_prefill_rope(x["q"], k, v, kc, kc.copy(), np.zeros(B, np.int64), W, eps)
     assert np.allclose(o, o_ref, rtol=0, atol=1e-12) and np.allclose(lse, lse_ref, rtol=0, atol=1e-12)
     pos = np.arange(T)[None, :]
-    assert np.allclose(kc2[:, :T], oracle_rope_qknorm(k, pos, eps), rtol=0, atol=0)
+    assert np.array_equal(kc2[:, :T], round_bf16(oracle_rope_qknorm(k, pos, eps)))
 
 
 def test_decode_is_the_last_row_of_a_one_token_prefill():
@@ -121,3 +121,17 @@ def test_decode_is_the_last_row_of_a_one_token_prefill():
     for b in range(B):
         n = lens[b]
         assert np.array_equal(kc_d[b, :n], kc_p[b, :n]) and np.array_equal(vc_d[b, :n], vc_p[b, :n])
+
+
+def test_bf16_rounding_is_to_nearest_even():
+    # exact bf16 values stay; halfway cases go to the even neighbour; others to the nearest
+    ulp1 = 2.0 ** -7                      # bf16 spacing in [1, 2)
+    cases = {1.0: 1.0, 1.0 + ulp1: 1.0 + ulp1, 1.0 + ulp1 / 2: 1.0, 1.0 + 1.5 * ulp1: 1.0 + 2 * ulp1,
+             1.0 + 0.49 * ulp1: 1.0, 1.0 + 0.51 * ulp1: 1.0 + ulp1, -3.0 - 0.51 * 2 * ulp1: -3.0 - 2 * ulp1,
+             0.0: 0.0}
+    for x, want in cases.items():
+        assert round_bf16(np.array([x]))[0] == want, x
+    x = np.random.default_rng(12).standard_normal(10000) * 7.0
+    r = round_bf16(x)
+    spacing = 2.0 ** (np.floor(np.log2(np.abs(r))) - 7)
+    assert np.all(np.abs(x - r) <= spacing / 2 * (1 + 1e-9))
