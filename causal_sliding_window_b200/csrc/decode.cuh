@@ -51,7 +51,12 @@ struct DecParams {
     float scale_log2;
     int nsplit;                    // splits launched per sequence
     int nsplit_max;                // stride of the partial arrays
-    // kRope: the query is rotated and normalised at its position cache_len[b] - 1 (rope.cuh)
+    // kRope: the query is rotated and normalised at its position cache_len[b] - 1 (rope.cuh), and
+    // the new token's key (rotated, normalised) and value are written into that slot first
+    const __nv_bfloat16* k_new;    // [B, Hk, D]
+    const __nv_bfloat16* v_new;
+    __nv_bfloat16* kc_out;         // the caches kc / vc, written at slot cache_len[b] - 1
+    __nv_bfloat16* vc_out;
     const float* rope_cos;         // [max_pos, D/2]
     const float* rope_sin;
     int max_pos;
@@ -121,6 +126,22 @@ __global__ void __launch_bounds__(kDecodeThreads) swa_decode_kernel(const DecPar
             rpos = 0;
         }
         rpos = rpos < 0 ? 0 : rpos;
+    }
+    if (kRope && start < end && end == L && L - 1 < p.max_pos) {
+        // This CTA's chunk holds the new token's slot: write the token's rotated, normalised key
+        // and its value there before any load.  Other CTAs of the sequence that read the slot
+        // write the same bytes themselves first, so no CTA waits for another.
+        if (live) {   // uniform over a pair's threads
+            const size_t src = (size_t(b) * (H / kvg) + hk) * D + c * 8;
+            float f[8];
+            bf16x8_to_f32<D>(*reinterpret_cast<const uint4*>(p.k_new + src), f);
+            rope_qknorm8<D>(f, c, p.rope_cos + size_t(rpos) * (D / 2), p.rope_sin + size_t(rpos) * (D / 2), p.eps,
+                            rope_group_mask<D>());
+            const size_t dst = (size_t(b) * p.cap + size_t(L - 1)) * (size_t(H / kvg) * D) + size_t(hk) * D + c * 8;
+            *reinterpret_cast<uint4*>(p.kc_out + dst) = bf16x8_pack(f);
+            *reinterpret_cast<uint4*>(p.vc_out + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
+        }
+        __syncthreads();   // the block's loads below see the slot
     }
 #pragma unroll
     for (int a = 0; a < QPT; ++a) {

@@ -500,7 +500,8 @@ size_t attn_decode_workspace_bytes(int B, int cap, int H, int D) {
 
 static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
                        const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
-                       int cap, int H, int Hkv, int D, int W, float scale, const RopeArgs& rope, void* stream) {
+                       int cap, int H, int Hkv, int D, int W, float scale, const RopeArgs& rope,
+                       const attn_bf16* k_new, const attn_bf16* v_new, void* stream) {
     if (!q || !k_cache || !v_cache || !cache_len || !o || !workspace) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
@@ -536,6 +537,10 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     p.scale_log2 = scale * 1.4426950408889634f;
     p.nsplit = (span + g.chunk - 1) / g.chunk;
     p.nsplit_max = nsm;
+    p.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+    p.kc_out = const_cast<__nv_bfloat16*>(p.kc);   // written only with the prologue (attn_decode_rope)
+    p.vc_out = const_cast<__nv_bfloat16*>(p.vc);
     p.rope_cos = rope.cs;
     p.rope_sin = rope.sn;
     p.max_pos = rope.max_pos;
@@ -574,7 +579,7 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
                     const int32_t* cache_len, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
                     int cap, int H, int Hkv, int D, int W, float scale, void* stream) {
     return decode_impl(q, k_cache, v_cache, cache_len, o, lse, workspace, ws_bytes, B, cap, H, Hkv, D, W, scale,
-                       RopeArgs{}, stream);
+                       RopeArgs{}, nullptr, nullptr, stream);
 }
 
 int attn_decode_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
@@ -594,13 +599,10 @@ int attn_decode_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16
     r.sn = rope_sin;
     r.max_pos = max_pos;
     r.eps = eps;
-    // 1. the new token's key (rotated, normalised) and value into slot cache_len[b] - 1
-    if (launch_append(k_new, v_new, k_cache, v_cache, cache_len, B, 1, cap, Hkv, D, -1, 0, r,
-                      reinterpret_cast<cudaStream_t>(stream)) != ATTN_OK)
-        return ATTN_ERR_LAUNCH;
-    // 2. decode with the query rotated and normalised inside the kernel
+    // One launch: the decode kernel writes the new token's rotated key and its value into slot
+    // cache_len[b] - 1 (in the CTAs that read that slot) and rotates the query in registers.
     return decode_impl(q, k_cache, v_cache, cache_len, o, lse, workspace, ws_bytes, B, cap, H, Hkv, D, W, scale, r,
-                       stream);
+                       k_new, v_new, stream);
 }
 
 int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache, const int32_t* cache_len,

@@ -153,11 +153,11 @@ int attn_prefill_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf1
                       int Tn, int cap, int H, int Hkv, int D, int W, float scale, void* stream);
 
 /*
- * One decode step with the prologue and append: the new token of sequence b sits in slot
- * cache_len[b] - 1 (its position; cache_len counts it, each in [1, cap]).  Its key k_new
- * [B, Hkv, D] is rotated, normalised and written there with its value v_new [B, Hkv, D];
- * its query q [B, H, D] is rotated and normalised inside the decode kernel, which then
- * attends as attn_decode_gqa.  workspace: attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)
+ * One decode step with the prologue and append, in one launch: the new token of sequence b
+ * sits in slot cache_len[b] - 1 (its position; cache_len counts it, each in [1, cap]).  Its
+ * key k_new [B, Hkv, D] is rotated, normalised and written there with its value v_new
+ * [B, Hkv, D] by the decode kernel itself, which also rotates and normalises the query
+ * q [B, H, D] in registers and then attends as attn_decode_gqa.  workspace: attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)
  * bytes, zero-filled before first use (every call leaves it zeroed).  Tables and eps as
  * attn_rope_qknorm.
  */
