@@ -285,6 +285,104 @@ def run_case(args):
     return 0 if status == 0 else 1
 
 
+def run_widened(args):
+    """Standalone CUDA-event timings of the widened rows on seeded synthetic inputs (10 calls after
+    3 warm-ups each, one JSON line per measurement): grouped K/V heads (d24 shape with 4 K/V heads,
+    forward and backward; decode workload with 4 K/V heads), the RoPE + QK-norm op and its backward
+    on a d24-shaped q, chunked prefill (32 sequences, a 512-token chunk after U[0, 1536] cached
+    tokens, capacity 2048) with and without the prologue, and decode with and without it."""
+    import torch
+
+    from causal_sliding_window_b200 import inputs, ops
+
+    dev = torch.device("cuda", 0)
+    reps = 10
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps   # ms
+
+    def emit(**kw):
+        print(json.dumps(kw), flush=True)
+
+    cfg = inputs.WORKLOADS["d24"]
+    B, T, H, D, Hkv = cfg["B"], cfg["T"], cfg["H"], cfg["D"], 4
+    x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"])
+    q, do = to_bf16(x["q"], dev), to_bf16(x["do"], dev)
+    k = to_bf16(np.ascontiguousarray(x["k"][:, :, :Hkv]), dev)
+    v = to_bf16(np.ascontiguousarray(x["v"][:, :, :Hkv]), dev)
+    del x
+    o, lse = torch.empty_like(q), torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+    for W in (2048, 512):
+        pairs = band_pairs(T, W) * B * H
+        tf = timed(lambda: ops.attn_fwd(q, k, v, o, lse, W))
+        tb = timed(lambda: ops.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, W))
+        emit(row="grouped K/V heads, d24 shape, 4 K/V heads", W=W, fwd_ms=round(tf, 4),
+             fwd_tflops=round(4 * D * pairs / tf / 1e9, 1), bwd_ms=round(tb, 4), bwd_tflops=round(10 * D * pairs / tb / 1e9, 1))
+    cos, sin = ops.rope_tables(4096, D, dev)
+    y = torch.empty_like(q)
+    t = timed(lambda: ops.attn_rope_qknorm(q, y, cos, sin, 1e-6))
+    emit(row="rope + qk norm, d24-shaped q", ms=round(t, 4), gbs=round(2 * q.numel() * 2 / t / 1e6, 1))
+    t = timed(lambda: ops.attn_rope_qknorm_bwd(q, do, y, cos, sin, 1e-6))
+    emit(row="rope + qk norm backward, d24-shaped q", ms=round(t, 4), gbs=round(3 * q.numel() * 2 / t / 1e6, 1))
+    del q, do, k, v, o, lse, dq, dk, dv, ws, y
+    torch.cuda.empty_cache()
+    # chunked prefill
+    Bp, Tn, cap = 32, 512, 2048
+    L = inputs.uniform_int(7, "cache_len", Bp, 0, cap - Tn)
+    xp = inputs.attention_inputs(Bp, Tn, H, D, seed=7)
+    qp, kn, vn = (to_bf16(xp[n], dev) for n in ("q", "k", "v"))
+    kc = torch.zeros((Bp, cap, H, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    cl = torch.from_numpy(L).to(dev)
+    for W in (2048, 512):
+        pairs = sum(min(int(L[b]) + t + 1, W) for b in range(Bp) for t in range(Tn)) * H
+        t0 = timed(lambda: ops.prefill(qp, kn, vn, kc, vc, cl, W))
+        t1 = timed(lambda: ops.prefill_rope(qp, kn, vn, kc, vc, cl, cos, sin, 1e-6, W))
+        emit(row="prefill, 32 x 512-token chunks after U[0,1536] cached", W=W, ms=round(t0, 4),
+             tflops=round(4 * D * pairs / t0 / 1e9, 1), rope_ms=round(t1, 4), rope_tflops=round(4 * D * pairs / t1 / 1e9, 1))
+    del qp, kn, vn, kc, vc
+    torch.cuda.empty_cache()
+    # decode, 12 and 4 K/V heads, with and without the prologue
+    dc = inputs.DECODE_WORKLOAD
+    xd = inputs.decode_inputs(dc["B"], dc["cap"], dc["H"], dc["D"], seed=dc["seed"])
+    qd = to_bf16(xd["q"], dev)
+    cl = torch.from_numpy(xd["cache_len"]).to(dev)
+    for hk in (dc["H"], 4):
+        # two cache sets used in turn, so that a call does not find its cache in L2
+        kc = to_bf16(np.ascontiguousarray(xd["k_cache"][:, :, :hk]), dev)
+        vc = to_bf16(np.ascontiguousarray(xd["v_cache"][:, :, :hk]), dev)
+        sets = [(kc, vc), (kc.roll(1, 0).contiguous(), vc.roll(1, 0).contiguous())]
+        turn = [0]
+
+        def pick():
+            turn[0] ^= 1
+            return sets[turn[0]]
+
+        kn = torch.zeros((dc["B"], hk, dc["D"]), dtype=torch.bfloat16, device=dev)
+        vn = torch.zeros_like(kn)
+        wsd = ops.decode_workspace(dc["B"], dc["cap"], dc["H"], dc["D"], dev, Hkv=hk)
+        for W in dc["windows"]:
+            nbytes = decode_bytes(xd["cache_len"], hk, dc["D"], W) + 2 * dc["B"] * (dc["H"] - hk) * dc["D"] * 2
+            t0 = timed(lambda: ops.decode(qd, *pick(), cl, W, workspace=wsd))
+            t1 = timed(lambda: ops.decode_rope(qd, kn, vn, *pick(), cl, cos, sin, 1e-6, W, workspace=wsd))
+            emit(row=f"decode workload, {hk} K/V heads", W=W, us=round(t0 * 1e3, 2), tbs=round(nbytes / t0 / 1e9, 3),
+                 rope_us=round(t1 * 1e3, 2), rope_tbs=round(nbytes / t1 / 1e9, 3))
+        del kc, vc, sets
+    status = ops.attn_device_status(clear=True)
+    emit(status=status)
+    return 0 if status == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -294,8 +392,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-log", default=None)
-    ap.add_argument("--case", default="step", choices=["step", "fwd", "bwd", "decode"],
-                    help="profiling mode: run only one call repeatedly on a reduced batch (no metric line)")
+    ap.add_argument("--case", default="step", choices=["step", "fwd", "bwd", "decode", "widened"],
+                    help="profiling mode: run only one call repeatedly on a reduced batch (no metric line); "
+                         "widened: standalone timings of the grouped-head, prologue and prefill rows")
     ap.add_argument("--batch", type=int, default=8, help="batch for --case (d24 shape otherwise)")
     ap.add_argument("--window", type=int, default=2048, help="window for --case")
     args = ap.parse_args()
@@ -304,6 +403,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.case == "widened":
+        return run_widened(args)
     if args.case != "step":
         return run_case(args)
     if args.warmup < 3:
