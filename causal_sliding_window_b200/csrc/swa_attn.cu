@@ -379,6 +379,41 @@ int attn_rope_qknorm_bwd(const attn_bf16* x, const attn_bf16* dy, attn_bf16* dx,
     return rope_qknorm_impl(x, dy, dx, pos0, rope_cos, rope_sin, max_pos, B, T, H, D, eps, true, stream);
 }
 
+int attn_fwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* q_rot, attn_bf16* k_rot,
+                  attn_bf16* o, float* lse, const float* rope_cos, const float* rope_sin, int max_pos, float eps,
+                  int B, int T, int H, int Hkv, int D, int W, float scale, void* stream) {
+    if (!q || !k || !v || !q_rot || !k_rot || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, q_rot, k_rot, o, lse};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv) || !valid_rope(rope_cos, rope_sin, max_pos, eps))
+        return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    int st = rope_qknorm_impl(q, nullptr, q_rot, nullptr, rope_cos, rope_sin, max_pos, B, T, H, D, eps, false, stream);
+    if (st == ATTN_OK)
+        st = rope_qknorm_impl(k, nullptr, k_rot, nullptr, rope_cos, rope_sin, max_pos, B, T, Hkv, D, eps, false, stream);
+    if (st == ATTN_OK) st = attn_fwd_gqa(q_rot, k_rot, v, o, lse, B, T, H, Hkv, D, W, scale, stream);
+    return st;
+}
+
+int attn_bwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* q_rot, const attn_bf16* k_rot,
+                  const attn_bf16* v, const attn_bf16* o, const float* lse, const attn_bf16* dout, attn_bf16* dq,
+                  attn_bf16* dk, attn_bf16* dv, void* workspace, size_t ws_bytes, const float* rope_cos,
+                  const float* rope_sin, int max_pos, float eps, int B, int T, int H, int Hkv, int D, int W,
+                  float scale, void* stream) {
+    if (!q || !k || !q_rot || !k_rot || !aligned16(q) || !aligned16(k) || !aligned16(q_rot) || !aligned16(k_rot))
+        return ATTN_ERR_INVALID_ARG;
+    if (!valid_rope(rope_cos, rope_sin, max_pos, eps)) return ATTN_ERR_INVALID_ARG;
+    // dQ', dK' at the rotated inputs, then back through rotate-and-normalise in place
+    int st = attn_bwd_gqa(q_rot, k_rot, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, Hkv, D, W, scale,
+                          stream);
+    if (st == ATTN_OK)
+        st = rope_qknorm_impl(q, dq, dq, nullptr, rope_cos, rope_sin, max_pos, B, T, H, D, eps, true, stream);
+    if (st == ATTN_OK)
+        st = rope_qknorm_impl(k, dk, dk, nullptr, rope_cos, rope_sin, max_pos, B, T, Hkv, D, eps, true, stream);
+    return st;
+}
+
 // Workspace: lse*log2(e) and Delta as [B*H, Tp] fp32 rows (Tp = T rounded up to 128).
 size_t attn_bwd_workspace_bytes(int B, int T, int H, int D) {
     if (B < 1 || T < 1 || H < 1 || D < 1) return 0;

@@ -73,6 +73,10 @@ _lib.attn_prefill_rope.argtypes = [_p] * 8 + [_i, _f, _p, _p, _p, _sz] + [_i] * 
 _lib.attn_prefill_rope.restype = _i
 _lib.attn_decode_rope.argtypes = [_p] * 8 + [_i, _f, _p, _p, _p, _sz] + [_i] * 6 + [_f, _p]
 _lib.attn_decode_rope.restype = _i
+_lib.attn_fwd_rope.argtypes = [_p] * 9 + [_i, _f] + [_i] * 6 + [_f, _p]
+_lib.attn_fwd_rope.restype = _i
+_lib.attn_bwd_rope.argtypes = [_p] * 12 + [_sz, _p, _p, _i, _f] + [_i] * 6 + [_f, _p]
+_lib.attn_bwd_rope.restype = _i
 _lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
 _lib.attn_bwd_set_profile_events.restype = _i
 _lib.attn_device_status.argtypes = [_i]
@@ -85,7 +89,8 @@ _lib.attn_status_string.restype = ctypes.c_char_p
 EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_gqa",
             "attn_decode_workspace_bytes", "attn_decode_gqa_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
             "attn_status_string", "attn_rope_tables", "attn_rope_qknorm", "attn_rope_qknorm_bwd",
-            "attn_prefill_rope_workspace_bytes", "attn_prefill_rope", "attn_decode_rope"]
+            "attn_prefill_rope_workspace_bytes", "attn_prefill_rope", "attn_decode_rope", "attn_fwd_rope",
+            "attn_bwd_rope"]
 
 
 class AttnError(RuntimeError):
@@ -397,3 +402,27 @@ def decode_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps: flo
         workspace = decode_workspace(B, cap, H, D, q.device, Hkv=Hkv)
     attn_decode_rope(q, k_new, v_new, k_cache, v_cache, cache_len, cos, sin, eps, o, lse, workspace, W, scale, stream)
     return o, lse
+
+
+def attn_fwd_rope(q, k, v, q_rot, k_rot, o, lse, cos, sin, eps: float, W: int, scale=None, stream=None):
+    """Training forward with the prologue; q_rot, k_rot receive the rotated, normalised inputs."""
+    B, T, H, D = _bthd(q, q_rot, o)
+    Hkv = _kv_heads((B, T, H, D), k, k_rot, v)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, T] tensor")
+    max_pos = _tables(cos, sin, D)
+    _check(_lib.attn_fwd_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(q_rot), _ptr(k_rot), _ptr(o), _ptr(lse), _ptr(cos),
+                              _ptr(sin), max_pos, float(eps), B, T, H, Hkv, D, int(W), _scale(scale, D),
+                              _stream(stream)), "attn_fwd_rope")
+
+
+def attn_bwd_rope(q, k, q_rot, k_rot, v, o, lse, dout, dq, dk, dv, workspace, cos, sin, eps: float, W: int, scale=None,
+                  stream=None):
+    """Training backward with the prologue: dq, dk, dv with respect to the raw q, k, v."""
+    B, T, H, D = _bthd(q, q_rot, o, dout, dq)
+    Hkv = _kv_heads((B, T, H, D), k, k_rot, v, dk, dv)
+    max_pos = _tables(cos, sin, D)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.attn_bwd_rope(_ptr(q), _ptr(k), _ptr(q_rot), _ptr(k_rot), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _ptr(cos), _ptr(sin), max_pos,
+                              float(eps), B, T, H, Hkv, D, int(W), _scale(scale, D), _stream(stream)), "attn_bwd_rope")

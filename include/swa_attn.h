@@ -137,6 +137,28 @@ int attn_rope_qknorm_bwd(const attn_bf16* x, const attn_bf16* dy, attn_bf16* dx,
                          const float* rope_cos, const float* rope_sin, int max_pos, int B, int T, int H, int D,
                          float eps, void* stream);
 
+/*
+ * Training forward with the prologue: q_rot = rotate-and-normalise(q), k_rot likewise (token t at
+ * position t), then attn_fwd_gqa(q_rot, k_rot, v).  q_rot [B, T, H, D] and k_rot [B, T, Hkv, D]
+ * bf16 are written (the caller keeps them for attn_bwd_rope).  Other arguments as attn_fwd_gqa
+ * and attn_rope_qknorm.
+ */
+int attn_fwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* q_rot, attn_bf16* k_rot,
+                  attn_bf16* o, float* lse, const float* rope_cos, const float* rope_sin, int max_pos, float eps,
+                  int B, int T, int H, int Hkv, int D, int W, float scale, void* stream);
+
+/*
+ * Training backward with the prologue: attn_bwd_gqa at (q_rot, k_rot, v), then dq and dk taken
+ * back through rotate-and-normalise at the raw q, k in place (the rounding of q_rot, k_rot to
+ * bf16 passes gradients through unchanged, as a cast does).  dq, dk, dv are the gradients with
+ * respect to the raw q, k and v.  Workspace as attn_bwd.
+ */
+int attn_bwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* q_rot, const attn_bf16* k_rot,
+                  const attn_bf16* v, const attn_bf16* o, const float* lse, const attn_bf16* dout, attn_bf16* dq,
+                  attn_bf16* dk, attn_bf16* dv, void* workspace, size_t ws_bytes, const float* rope_cos,
+                  const float* rope_sin, int max_pos, float eps, int B, int T, int H, int Hkv, int D, int W,
+                  float scale, void* stream);
+
 /* Bytes of workspace attn_prefill_rope needs (the chunk's rotated queries, bf16). */
 size_t attn_prefill_rope_workspace_bytes(int B, int Tn, int H, int D);
 

@@ -21,6 +21,7 @@ from .swa_oracle import (  # noqa: F401
     oracle_threads,
 )
 from .rope_oracle import (  # noqa: F401
+    oracle_bwd_rope,
     oracle_decode_rope,
     oracle_fwd_rope,
     oracle_prefill_rope,

@@ -28,7 +28,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .swa_oracle import oracle_decode, oracle_fwd, oracle_prefill
+from .swa_oracle import oracle_bwd, oracle_decode, oracle_fwd, oracle_prefill
 
 
 def _f64(x):
@@ -102,6 +102,19 @@ def oracle_fwd_rope(q, k, v, W: int, eps: float, base: float = 10000.0, scale: f
     qr = round_bf16(oracle_rope_qknorm(q, pos, eps, base))
     kr = round_bf16(oracle_rope_qknorm(k, pos, eps, base))
     return oracle_fwd(qr, kr, _f64(v), W, scale)
+
+
+def oracle_bwd_rope(q, k, v, do, W: int, eps: float, base: float = 10000.0, scale: float | None = None):
+    """Training backward with the prologue: the attention backward at the rotated, normalised
+    (bf16-rounded) q and k, then each of dq, dk taken back through rotate-and-normalise at the raw
+    q, k (the rounding to bf16 passes gradients through unchanged, as a cast does in training).
+    Returns (dq, dk, dv) float64, dq and dk with respect to the raw q and k."""
+    T = np.asarray(q).shape[1]
+    pos = np.arange(T)[None, :]
+    qr = round_bf16(oracle_rope_qknorm(q, pos, eps, base))
+    kr = round_bf16(oracle_rope_qknorm(k, pos, eps, base))
+    dqr, dkr, dv = oracle_bwd(qr, kr, _f64(v), _f64(do), W, scale)
+    return oracle_rope_qknorm_bwd(q, pos, dqr, eps, base), oracle_rope_qknorm_bwd(k, pos, dkr, eps, base), dv
 
 
 def oracle_prefill_rope(q, k_new, v_new, k_cache, v_cache, cache_len, W: int, eps: float,

@@ -211,3 +211,20 @@ def test_rope_argument_checks():
     assert dec_r(dneed - 1) == ERR_WORKSPACE
     assert dec_r(dneed, kn=None) == ERR_INVALID
     assert dec_r(dneed, Hkv=3) == ERR_INVALID        # 3 does not divide 4
+
+
+def test_training_rope_argument_checks():
+    lib = ops._lib
+    fwd = lambda qr=A, cs=A, eps=1e-6, Hkv=2, D=128: lib.attn_fwd_rope(  # noqa: E731
+        A, A, A, qr, A, A, A, cs, A, 64, eps, 2, 16, 4, Hkv, D, 8, 0.1, None)
+    assert fwd(qr=None) == ERR_INVALID
+    assert fwd(cs=None) == ERR_INVALID
+    assert fwd(eps=-1.0) == ERR_INVALID
+    assert fwd(Hkv=3) == ERR_INVALID
+    assert fwd(D=96) == ERR_UNSUPPORTED
+    ws = ops.attn_bwd_workspace_bytes(2, 16, 4, 128)
+    bwd = lambda ws_bytes=ws, kr=A, cs=A: lib.attn_bwd_rope(  # noqa: E731
+        A, A, A, kr, A, A, A, A, A, A, A, A, ws_bytes, cs, A, 64, 1e-6, 2, 16, 4, 2, 128, 8, 0.1, None)
+    assert bwd(kr=None) == ERR_INVALID
+    assert bwd(cs=None) == ERR_INVALID
+    assert bwd(ws_bytes=ws - 1) == ERR_WORKSPACE

@@ -160,3 +160,31 @@ def test_decode_with_rope_matches_oracle(ops, H, Hkv, D):
         d = np.abs(gk[b, L - 1] - rkc[b, L - 1])
         assert np.all(d <= 2.0 ** (np.floor(np.log2(np.maximum(np.abs(rkc[b, L - 1]), 1e-30))) - 6))
         assert np.isnan(gk[b, L:]).all()       # slots after the new token are not written
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,W", [(2, 300, 4, 2, 128, 129), (1, 257, 2, 2, 64, 10 ** 9)])
+def test_training_forward_and_backward_with_rope(ops, B, T, H, Hkv, D, W):
+    from oracle import oracle_bwd_rope, oracle_fwd_rope
+
+    x = inputs.attention_inputs(B, T, H, D, seed=T + H)
+    k, v = (np.ascontiguousarray(x[n][:, :, :Hkv]) for n in ("k", "v"))
+    cos, sin = ops.rope_tables(T, D, "cuda")
+    q_d, k_d, v_d, do_d = dev_bf16(x["q"]), dev_bf16(k), dev_bf16(v), dev_bf16(x["do"])
+    q_rot, k_rot = torch.empty_like(q_d), torch.empty_like(k_d)
+    o = Guarded((B, T, H, D), torch.bfloat16)
+    lse = Guarded((B, H, T), torch.float32)
+    ops.attn_fwd_rope(q_d, k_d, v_d, q_rot, k_rot, o.t, lse.t, cos, sin, EPS, W)
+    dq, dk, dv = Guarded((B, T, H, D), torch.bfloat16), Guarded((B, T, Hkv, D), torch.bfloat16), \
+        Guarded((B, T, Hkv, D), torch.bfloat16)
+    ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device="cuda")
+    ops.attn_bwd_rope(q_d, k_d, q_rot, k_rot, v_d, o.t, lse.t, do_d, dq.t, dk.t, dv.t, ws, cos, sin, EPS, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    assert all(g.guards_intact() for g in (o, lse, dq, dk, dv))
+    ro, rl = oracle_fwd_rope(x["q"], k, v, W, EPS)
+    go, gl = host_f64(o.t), host_f64(lse.t)
+    assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
+    assert np.max(np.abs(gl - rl)) <= LSE_ABS
+    rdq, rdk, rdv = oracle_bwd_rope(x["q"], k, v, x["do"], W, EPS)
+    for got, ref in ((dq, rdq), (dk, rdk), (dv, rdv)):
+        assert rel_l2(host_f64(got.t), ref) <= G_REL

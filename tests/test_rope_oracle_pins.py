@@ -135,3 +135,44 @@ def test_bf16_rounding_is_to_nearest_even():
     r = round_bf16(x)
     spacing = 2.0 ** (np.floor(np.log2(np.abs(r))) - 7)
     assert np.all(np.abs(x - r) <= spacing / 2 * (1 + 1e-9))
+
+
+def test_training_backward_with_the_prologue_matches_autograd():
+    """The composed backward equals torch fp64 autograd through rotate-and-normalise, a bf16
+    rounding that passes gradients straight through, and masked softmax attention."""
+    import torch
+
+    from oracle import oracle_bwd_rope
+    from tests.test_oracle_pins import f64
+
+    B, T, H, Hk, D, W, eps = 1, 33, 2, 1, 16, 9, 1e-6
+    x = inputs.attention_inputs(B, T, H, D, seed=21)
+    k, v = (np.ascontiguousarray(x[n][:, :, :Hk]) for n in ("k", "v"))
+    dq, dk, dv = oracle_bwd_rope(x["q"], k, v, x["do"], W, eps)
+
+    tq = torch.tensor(f64(x["q"]), requires_grad=True)
+    tk = torch.tensor(f64(k), requires_grad=True)
+    tv = torch.tensor(f64(v), requires_grad=True)
+    th = torch.tensor([10000.0 ** (-2.0 * i / D) for i in range(D // 2)], dtype=torch.float64)
+    ang = torch.arange(T, dtype=torch.float64)[:, None] * th        # [T, D/2]
+    c, s_ = torch.cos(ang)[None, :, None, :], torch.sin(ang)[None, :, None, :]
+
+    def prologue(t):
+        a, b = t[..., :D // 2], t[..., D // 2:]
+        r = torch.cat([a * c - b * s_, a * s_ + b * c], dim=-1)
+        y = r / torch.sqrt((r * r).mean(-1, keepdim=True) + eps)
+        yr = torch.tensor(round_bf16(y.detach().numpy()))
+        return y + (yr - y).detach()                                  # value rounded, gradient straight through
+
+    qr, kr = prologue(tq), prologue(tk)
+    kr = kr.repeat_interleave(H // Hk, dim=2)
+    vr = tv.repeat_interleave(H // Hk, dim=2)
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    mask = (j <= i) & (j > i - W)
+    sc = torch.einsum("bihd,bjhd->bhij", qr, kr) / np.sqrt(D)
+    p = torch.softmax(sc.masked_fill(~mask, float("-inf")), dim=-1)
+    o = torch.einsum("bhij,bjhd->bihd", p, vr)
+    o.backward(torch.tensor(f64(x["do"])))
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.allclose(got, ref.numpy(), rtol=0, atol=1e-9)
