@@ -228,3 +228,14 @@ def test_training_rope_argument_checks():
     assert bwd(kr=None) == ERR_INVALID
     assert bwd(cs=None) == ERR_INVALID
     assert bwd(ws_bytes=ws - 1) == ERR_WORKSPACE
+
+
+def test_header_is_plain_c(tmp_path):
+    """The boundary header compiles as C99, and every entry point it declares can be named from C."""
+    import subprocess
+
+    names = declared_functions()
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "swa_attn.h"\n' + "".join(f"void* p_{n} = (void*)&{n};\n" for n in names))
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-c", "-I", os.path.dirname(HEADER),
+                           str(src), "-o", str(tmp_path / "use_header.o")])
