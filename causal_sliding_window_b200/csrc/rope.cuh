@@ -121,10 +121,11 @@ __device__ __forceinline__ int rope_position(const int* pos0, int b, int t, int 
 // kBwd: dx from dy instead, with r = rope(x), s = (mean(r^2) + eps)^(-1/2):
 //   dr = s dy - (s^3 / D) r (dy . r),  dx = rope^(-1)(dr).
 // A row whose position has no table row is left unwritten.
+// x, dy and y may be the same array (in place): no __restrict__ on them.  Each thread reads its own
+// 16 bytes before writing them, and partner values travel through shuffles, not memory.
 template <int D, bool kBwd>
-__global__ void __launch_bounds__(256) swa_rope_qknorm_kernel(const __nv_bfloat16* __restrict__ x,
-                                                              const __nv_bfloat16* __restrict__ dy,
-                                                              __nv_bfloat16* __restrict__ y, int B, int T, int H,
+__global__ void __launch_bounds__(256) swa_rope_qknorm_kernel(const __nv_bfloat16* x, const __nv_bfloat16* dy,
+                                                              __nv_bfloat16* y, int B, int T, int H,
                                                               const int* __restrict__ pos0,
                                                               const float* __restrict__ cs,
                                                               const float* __restrict__ sn, int max_pos, float eps) {
