@@ -29,6 +29,7 @@
 //                take columns 0..63 of the 128-column score tiles, warps 4..7 columns 64..127.
 #pragma once
 
+#include "rope.cuh"
 #include "sm100.cuh"
 
 namespace swa {
@@ -46,9 +47,16 @@ struct BwdParams {
     float scale_log2;
     int n_blk;            // ceil(T / 128)
     int n_items;          // items of this launch: n_blk * B * H (dQ) or n_blk * B * H / G (dK/dV)
-    int work_slot;        // index into g_work_slots for this launch
+    int stream_slot;      // the launch's stream slot: its work counter and status word
     int Tp;               // T rounded up to 128
     long long wait_limit;
+    // dQ kernel with kRope: q is the rotated, normalised query; dq is taken back through that
+    // prologue at the raw query q_raw (token t at position t) before it is written (rope.cuh)
+    const __nv_bfloat16* q_raw;
+    const float* rope_cos;  // [max_pos, D/2]
+    const float* rope_sin;
+    int max_pos;
+    float eps;
 };
 
 // ---------------------------------------------------------------------------
@@ -208,7 +216,7 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
     if (int(base - raw) + C::SMEM_USED > C::SMEM) {   // uniform across the CTA: nothing started yet
-        if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusSmemLayout);
+        if (threadIdx.x == 0) report_status(p.stream_slot, kStatusSmemLayout);
         return;
     }
 
@@ -259,7 +267,8 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(item_full0 + 8u * e, 1);
             mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and warps 0..7
         }
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = p.stream_slot;   // read by a wait that gives up
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -286,7 +295,7 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = true;
             for (int ki = 0;; ++ki) {
                 const int item =
-                    item_produce(p.work_slot, ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                    item_produce(p.stream_slot, ki, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
                 const BwdKVItem g = bwd_kv_item(p, item);
                 // K and V are read by this CTA alone: start them towards L2 while the previous
@@ -337,14 +346,14 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (!ok) break;
             }
-            work_slot_finish(p.work_slot);
+            work_slot_finish(p.stream_slot);
             // Drain: no copy of this CTA may still be landing when it exits.
             for (int s = 0; s < C::NQ && s < nq; ++s)
-                mbar_drain(q_full(s), uint32_t(((nq - s + C::NQ - 1) / C::NQ - 1) & 1), p.wait_limit);
+                mbar_drain(q_full(s), uint32_t(((nq - s + C::NQ - 1) / C::NQ - 1) & 1), p.wait_limit, p.stream_slot);
             for (int s = 0; s < C::NDO && s < n; ++s)
-                mbar_drain(do_full(s), uint32_t(((n - s + C::NDO - 1) / C::NDO - 1) & 1), p.wait_limit);
-            if (nk > 0) mbar_drain(k_full, uint32_t((nk - 1) & 1), p.wait_limit);
-            if (nv > 0) mbar_drain(v_full, uint32_t((nv - 1) & 1), p.wait_limit);
+                mbar_drain(do_full(s), uint32_t(((n - s + C::NDO - 1) / C::NDO - 1) & 1), p.wait_limit, p.stream_slot);
+            if (nk > 0) mbar_drain(k_full, uint32_t((nk - 1) & 1), p.wait_limit, p.stream_slot);
+            if (nv > 0) mbar_drain(v_full, uint32_t((nv - 1) & 1), p.wait_limit, p.stream_slot);
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
@@ -644,7 +653,10 @@ __device__ __forceinline__ BwdQItem bwd_q_item(const BwdParams& p, int item) {
 //   dQ += dS K_j                (A operand from TMEM)
 // The row warps hold dP in registers as soon as they have loaded it, so dP(n+1) is issued
 // before dQ(n): MMA order S(n+1) | dP(n+1) | dQ(n).
-template <int D>
+// kRope: the item's dQ (the gradient at the rotated, normalised query) is taken back through the
+// rotary + QK-norm prologue in the epilogue, by warps 0..3 over whole rows: with r = rope(x),
+// s = (mean(r^2) + eps)^(-1/2) and dy = dQ:  dr = s dy - (s^3 / D) r (dy . r),  dx = rope^-1(dr).
+template <int D, bool kRope = false>
 __global__ void __launch_bounds__(BwdQCfg<D>::THREADS, 1)
 swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -655,7 +667,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
     if (int(base - raw) + C::SMEM_USED > C::SMEM) {   // uniform across the CTA: nothing started yet
-        if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusSmemLayout);
+        if (threadIdx.x == 0) report_status(p.stream_slot, kStatusSmemLayout);
         return;
     }
 
@@ -708,7 +720,8 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(item_full0 + 8u * e, 1);
             mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and warps 0..7
         }
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = p.stream_slot;   // read by a wait that gives up
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -738,7 +751,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             };
             for (int qi = 0;; ++qi) {
                 const int item =
-                    item_produce(p.work_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                    item_produce(p.stream_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
                 const BwdQItem g = bwd_q_item(p, item);
                 // Q and dO are read by this CTA alone: start them towards L2 while the previous
@@ -771,12 +784,12 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 if (!ok) break;
             }
-            work_slot_finish(p.work_slot);
+            work_slot_finish(p.stream_slot);
             // Drain: no copy of this CTA may still be landing when it exits.
-            for (int s = 0; s < C::NK && s < nk; ++s) mbar_drain(k_full(s), uint32_t(((nk - s + C::NK - 1) / C::NK - 1) & 1), p.wait_limit);
-            for (int s = 0; s < C::NV && s < nv; ++s) mbar_drain(v_full(s), uint32_t(((nv - s + C::NV - 1) / C::NV - 1) & 1), p.wait_limit);
-            if (nq > 0) mbar_drain(q_full, uint32_t((nq - 1) & 1), p.wait_limit);
-            if (ndo > 0) mbar_drain(do_full, uint32_t((ndo - 1) & 1), p.wait_limit);
+            for (int s = 0; s < C::NK && s < nk; ++s) mbar_drain(k_full(s), uint32_t(((nk - s + C::NK - 1) / C::NK - 1) & 1), p.wait_limit, p.stream_slot);
+            for (int s = 0; s < C::NV && s < nv; ++s) mbar_drain(v_full(s), uint32_t(((nv - s + C::NV - 1) / C::NV - 1) & 1), p.wait_limit, p.stream_slot);
+            if (nq > 0) mbar_drain(q_full, uint32_t((nq - 1) & 1), p.wait_limit, p.stream_slot);
+            if (ndo > 0) mbar_drain(do_full, uint32_t((ndo - 1) & 1), p.wait_limit, p.stream_slot);
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
@@ -867,10 +880,92 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             return true;
         };
+        // kRope epilogue of item pqi, query row pq of head (pb, ph): warps 4..7 only release the
+        // accumulator; warps 0..3 read whole rows (pairs (i, i + D/2) together) in two passes, the
+        // first for the row's two sums, the second for the output.
+        auto epilogue_rope = [&](int pqi, long long pq, int pb, int ph) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(dq_full, uint32_t(pqi & 1), abort_flag, p.wait_limit,
+                                                   kStatusTimeoutEpilogue)))
+                return false;
+            tc_fence_after();
+            if (rh == 0) {
+                const uint32_t src = tDQ + lane_off;
+                const bool in = pq < T, posok = pq < p.max_pos;
+                const size_t roff = ((size_t(pb) * T + size_t(in ? pq : 0)) * p.H + ph) * D;
+                const __nv_bfloat16* xr = p.q_raw + roff;
+                __nv_bfloat16* dst = p.dq + roff;
+                const float* cr = p.rope_cos + size_t(posok ? pq : 0) * (D / 2);
+                const float* sr = p.rope_sin + size_t(posok ? pq : 0) * (D / 2);
+                if (in && !posok) report_status(p.stream_slot, kStatusPositionRange);
+                float sxx = 0.f, sdr = 0.f, s_ = 0.f, k3 = 0.f;
+#pragma unroll 1
+                for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll 1
+                    for (int c = 0; c < D / 2; c += 32) {
+                        uint32_t a1[32], a2[32];   // dQ columns c.. and their partners c + D/2..
+                        __syncwarp();              // the TMEM loads are warp-collective
+                        tmem_ld32(src + c, a1);
+                        tmem_ld32(src + D / 2 + c, a2);
+                        tmem_ld_wait(a1);
+                        tmem_ld_wait(a2);
+                        if (!in) continue;
+                        if (!posok) {   // no table row: the gradient at the rotated query, as is
+                            if (pass == 1) {
+                                store_row32_bf16(dst + c, a1, p.scale);
+                                store_row32_bf16(dst + D / 2 + c, a2, p.scale);
+                            }
+                            continue;
+                        }
+#pragma unroll
+                        for (int v = 0; v < 32; v += 8) {
+                            float x1[8], x2[8];
+                            bf16x8_unpack(*reinterpret_cast<const uint4*>(xr + c + v), x1);
+                            bf16x8_unpack(*reinterpret_cast<const uint4*>(xr + D / 2 + c + v), x2);
+                            const float4 c0 = *reinterpret_cast<const float4*>(cr + c + v);
+                            const float4 c1 = *reinterpret_cast<const float4*>(cr + c + v + 4);
+                            const float4 s0 = *reinterpret_cast<const float4*>(sr + c + v);
+                            const float4 s1 = *reinterpret_cast<const float4*>(sr + c + v + 4);
+                            const float co[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                            const float si[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                            float o1[8], o2[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float r1 = fmaf(x1[i], co[i], -x2[i] * si[i]);
+                                const float r2 = fmaf(x1[i], si[i], x2[i] * co[i]);
+                                const float dy1 = __uint_as_float(a1[v + i]) * p.scale;
+                                const float dy2 = __uint_as_float(a2[v + i]) * p.scale;
+                                if (pass == 0) {
+                                    sxx = fmaf(r1, r1, fmaf(r2, r2, sxx));
+                                    sdr = fmaf(dy1, r1, fmaf(dy2, r2, sdr));
+                                } else {
+                                    const float dr1 = fmaf(s_, dy1, -k3 * r1), dr2 = fmaf(s_, dy2, -k3 * r2);
+                                    o1[i] = fmaf(dr1, co[i], dr2 * si[i]);    // rotated back
+                                    o2[i] = fmaf(dr2, co[i], -dr1 * si[i]);
+                                }
+                            }
+                            if (pass == 1) {
+                                *reinterpret_cast<uint4*>(dst + c + v) = bf16x8_pack(o1);
+                                *reinterpret_cast<uint4*>(dst + D / 2 + c + v) = bf16x8_pack(o2);
+                            }
+                        }
+                    }
+                    if (pass == 0) {
+                        const float ms = sxx * (1.f / D) + p.eps;
+                        s_ = ms > 0.f ? rsqrtf(ms) : 0.f;
+                        k3 = s_ * s_ * s_ * (1.f / D) * sdr;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(dq_free);
+            return true;
+        };
         bool ok = true;
         int n = 0;
         int prev_qi = -1;                  // item whose epilogue is still pending
         __nv_bfloat16* prev_dst = nullptr;
+        long long prev_q = 0;              // kRope: its query row and head
+        int prev_b = 0, prev_h = 0;
         for (int qi = 0;; ++qi) {
             const int item = item_consume_warp(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                kStatusTimeoutSoftmax, ok);
@@ -883,6 +978,10 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int j = g.jlo; j <= g.jhi && ok; ++j, ++n) {
                 const int buf = n & 1;
                 const uint32_t ph = uint32_t((n >> 1) & 1);
+                if (kRope && j == g.jlo && prev_qi >= 0) {   // before this step's scores: registers are free
+                    if (!(ok = epilogue_rope(prev_qi, prev_q, prev_b, prev_h))) break;
+                    prev_qi = -1;
+                }
                 ok = __all_sync(0xffffffffu,
                                 mbar_wait(s_full(buf), ph, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
@@ -916,7 +1015,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int c = 0; c < 64; ++c) pr[c] = (c >= clo && c <= chi) ? pr[c] : 0.f;
                 }
-                if (j == g.jlo && prev_qi >= 0) {
+                if (!kRope && j == g.jlo && prev_qi >= 0) {
                     if (!(ok = epilogue(prev_qi, prev_dst))) break;
                     prev_qi = -1;
                 }
@@ -955,8 +1054,16 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!ok) break;
             prev_qi = qi;
             prev_dst = q < T ? p.dq + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D + rh * (D / 2) : nullptr;
+            prev_q = q;
+            prev_b = g.b;
+            prev_h = g.h;
         }
-        if (ok && prev_qi >= 0) epilogue(prev_qi, prev_dst);
+        if (ok && prev_qi >= 0) {
+            if (kRope)
+                epilogue_rope(prev_qi, prev_q, prev_b, prev_h);
+            else
+                epilogue(prev_qi, prev_dst);
+        }
     }
 
     tc_fence_before();

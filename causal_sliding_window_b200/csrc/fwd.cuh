@@ -39,18 +39,25 @@ struct FwdCfg {
     static constexpr int NBOX = D / 64;
     static constexpr int NQBUF = 1;                 // Q buffers (2: the next item's Q loads a whole item ahead)
     static constexpr int NSTAGE = D == 128 ? 5 : 8; // K/V ring (a stage holds one K or one V tile)
+    // Exponentials of a score row evaluated on the FMA pipe (exp2_poly) instead of the special-
+    // function unit: pairs i of each 64-column half with (i & 7) >= 8 - POLY8, i.e. POLY8 / 8 of them.
+    static constexpr int POLY8 = 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = NQBUF * NQ * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    // kv_full, kv_empty per stage; q_full, q_empty per Q buffer; s_full, p_full, o_full, o_free per
-    // tile; mma_done; item_full, item_empty per entry of the item ring
-    static constexpr int NUM_BAR = 2 * NSTAGE + 2 * NQBUF + 4 * NQ + 1 + 2 * kItemRing;
+    // kv_full, kv_empty per stage; q_full, q_empty per Q buffer; s_full, p_full (keys 0..63 of P),
+    // o_full, o_free, p_full1 (keys 64..127) per tile; q_ready per Q buffer; mma_done; item_full,
+    // item_empty per entry of the item ring
+    static constexpr int NUM_BAR = 2 * NSTAGE + 3 * NQBUF + 5 * NQ + 1 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
     // the kernel checks at run time that the aligned layout fits what it was given.
     static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
     static constexpr int THREADS = 320;
+    // With the rotary + QK-norm prologue two more warps rotate and normalise each Q tile in shared
+    // memory (12 warps: still three per SM sub-partition, so the same register budget).
+    static constexpr int threads(bool rope) { return rope ? THREADS + 64 : THREADS; }
     static constexpr uint32_t TMEM_COLS = 512;      // S0 | S1 | O0 | O1
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
@@ -70,8 +77,15 @@ struct FwdParams {
     float scale_log2;     // softmax scale * log2(e)
     int n_qblk;           // ceil(T / 256)
     int n_items;          // n_qblk * B * H
-    int work_slot;        // index into g_work_slots for this launch
+    int stream_slot;      // the launch's stream slot: its work counter and status word
     long long wait_limit; // clock cycles before a wait gives up
+    // kRope: Q rows are rotated and normalised at their positions (q_offset[b] + t) before any S MMA
+    // reads them (rope.cuh); store_qrot: the rotated tiles are also written through tm_qr
+    const float* rope_cos;   // [max_pos, D/2]
+    const float* rope_sin;
+    int max_pos;
+    float eps;
+    int store_qrot;
 };
 
 // Geometry of one work item: query block qblk of head (b, h).
@@ -108,18 +122,21 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
 }
 
 // kOffset: chunked prefill (query rows start at q_offset[b]); false for training, where the
-// offset is zero and costs nothing.
-template <int D, bool kOffset = false>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+// offset is zero and costs nothing.  kRope: the rotary + QK-norm prologue of the queries runs
+// inside the kernel (warps 10 and 11), on each Q tile in shared memory between its load and the
+// first S MMA; tm_qr then describes where the rotated queries are stored (when p.store_qrot).
+template <int D, bool kOffset = false, bool kRope = false>
+__global__ void __launch_bounds__(FwdCfg<D>::threads(kRope), 1)
 swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qr,
+               const FwdParams p) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
     if (int(base - raw) + C::SMEM_USED > C::SMEM) {   // uniform across the CTA: nothing started yet
-        if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusSmemLayout);
+        if (threadIdx.x == 0) report_status(p.stream_slot, kStatusSmemLayout);
         return;
     }
 
@@ -135,7 +152,9 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto p_full = [&](int t) { return bt + 8u * (C::NQ + t); };
     auto o_full = [&](int t) { return bt + 8u * (2 * C::NQ + t); };
     auto o_free = [&](int t) { return bt + 8u * (3 * C::NQ + t); };
-    const uint32_t mma_done = bt + 8u * (4 * C::NQ);
+    auto p_full1 = [&](int t) { return bt + 8u * (4 * C::NQ + t); };
+    auto q_ready = [&](int qb) { return bt + 8u * (5 * C::NQ + qb); };   // kRope: Q rotated in place
+    const uint32_t mma_done = bt + 8u * (5 * C::NQ + C::NQBUF);
     const uint32_t item_full0 = mma_done + 8u, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
@@ -152,20 +171,23 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         for (int qb = 0; qb < C::NQBUF; ++qb) {
             mbar_init(q_full(qb), 1);
-            mbar_init(q_empty(qb), 1);
+            mbar_init(q_empty(qb), kRope ? 2 : 1);   // the S MMAs have read it (and the q_rot store)
+            mbar_init(q_ready(qb), 64);
         }
         for (int t = 0; t < C::NQ; ++t) {
             mbar_init(s_full(t), 1);
             mbar_init(p_full(t), 128);
+            mbar_init(p_full1(t), 128);
             mbar_init(o_full(t), 1);
             mbar_init(o_free(t), 128);
         }
         mbar_init(mma_done, 1);
         for (int e = 0; e < kItemRing; ++e) {
             mbar_init(item_full0 + 8u * e, 1);
-            mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and the 8 softmax warps
+            mbar_init(item_empty0 + 8u * e, 1 + 8 + (kRope ? 2 : 0));   // MMA thread, softmax (+ prologue) warps
         }
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = p.stream_slot;   // read by a wait that gives up
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -190,7 +212,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             bool ok = true;
             for (;; ++qi) {
                 const int item =
-                    item_produce(p.work_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                    item_produce(p.stream_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
                 const FwdItem g = fwd_item<kOffset>(p, item);
                 // A Q buffer is free once the S MMAs of the item that used it completed.
@@ -218,15 +240,15 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
             }
-            work_slot_finish(p.work_slot);
+            work_slot_finish(p.stream_slot);
             // Drain: make sure no copy is still landing when the CTA exits.
             for (int s = 0; s < C::NSTAGE && s < it; ++s) {
                 const int fills = (it - s + C::NSTAGE - 1) / C::NSTAGE;
-                mbar_drain(kv_full(s), uint32_t((fills - 1) & 1), p.wait_limit);
+                mbar_drain(kv_full(s), uint32_t((fills - 1) & 1), p.wait_limit, p.stream_slot);
             }
             for (int qb = 0; qb < C::NQBUF && qb < qi; ++qb) {
                 const int fills = (qi - qb + C::NQBUF - 1) / C::NQBUF;
-                mbar_drain(q_full(qb), uint32_t((fills - 1) & 1), p.wait_limit);
+                mbar_drain(q_full(qb), uint32_t((fills - 1) & 1), p.wait_limit, p.stream_slot);
             }
         }
     } else if (warp == 9) {
@@ -237,8 +259,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             int npv0 = 0, npv1 = 0;   // PV MMAs issued per tile (all items)
             int nep0 = 0, nep1 = 0;   // items processed per tile (= epilogues owed)
             int qbuf = 0;   // Q buffer of the current item
-            auto issue_s = [&](int t, int stage) {
-                const uint32_t qa = sQ + (qbuf * C::NQ + t) * C::TILE, ka = sKV + stage * C::TILE;
+            auto issue_s = [&](int t, int stage, int qb) {
+                const uint32_t qa = sQ + (qb * C::NQ + t) * C::TILE, ka = sKV + stage * C::TILE;
                 const uint32_t d = t ? tS1 : tS0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -247,37 +269,62 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 tc_commit(s_full(t));
             };
-            auto issue_pv = [&](int t, int stage, bool first) {
+            // PV over keys 0..63 (half 0) or 64..127 (half 1) of the tile: the softmax warps publish
+            // P in these two halves, so the first half's MMAs run while the second half is computed.
+            auto issue_pv = [&](int t, int stage, bool first, int half) {
                 const uint32_t va = sKV + stage * C::TILE;
                 const uint32_t a = t ? tS1 : tS0, d = t ? tO1 : tO0;
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
+                for (int kk = half * (C::BN / 32); kk < (half + 1) * (C::BN / 32); ++kk)
                     mma_ts(d, a + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX, 1024), C::IDESC_PV,
                            (!first || kk > 0) ? 1u : 0u);
-                tc_commit(o_full(t));
+                if (half) tc_commit(o_full(t));
             };
+            auto wait_q = [&](int k) {   // the Q tiles of this CTA's k-th item are in place
+                return mbar_wait(kRope ? q_ready(k % C::NQBUF) : q_full(k % C::NQBUF), uint32_t((k / C::NQBUF) & 1),
+                                 abort_flag, p.wait_limit, kStatusTimeoutMma);
+            };
+            // Early start (with two Q buffers): when tile 0 has finished an item one key step before
+            // tile 1, the next item's first S for tile 0 is issued before tile 1's last step, so that
+            // tile 0's softmax warps start the next item instead of idling for that step.  Its Q is
+            // already loaded (the other buffer), and its first K tile is the ring entry right after
+            // the current item's last V tile.
+            constexpr bool kEarly = C::NQBUF >= 2;
+            int next_item = 0;
+            bool have_next = false;   // next_item was drawn from the item ring already
+            bool pre0 = false;        // S_0 of the item's first key tile was issued early, from stage pre_sk
+            int pre_sk = 0;
             // S_t overwrites the columns the last PV_t read P from; both are issued by this thread,
             // and the MMAs of one thread execute in issue order, so S_t needs no wait for PV_t.
             for (;; ++qi) {
-                const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
-                                                     kStatusTimeoutMma, ok);
+                const int item = have_next ? next_item
+                                           : item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag,
+                                                                 p.wait_limit, kStatusTimeoutMma, ok);
+                have_next = false;
                 if (!ok || item >= p.n_items) break;
                 const FwdItem g = fwd_item<kOffset>(p, item);
                 auto act = [&](int t, int j) {
                     return t ? (g.valid1 && j >= g.jlo1 && j <= g.jhi1) : (j >= g.jlo0 && j <= g.jhi0);
                 };
                 qbuf = qi % C::NQBUF;
-                ok = mbar_wait(q_full(qbuf), uint32_t((qi / C::NQBUF) & 1), abort_flag, p.wait_limit,
-                               kStatusTimeoutMma);
-                if (!ok) break;
                 bool first0 = true, first1 = true;
-                int sk = it % C::NSTAGE;
-                ok = mbar_wait(kv_full(sk), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
-                ++it;
-                if (!ok) break;
-                tc_fence_after();
-                if (act(0, g.jbeg)) issue_s(0, sk);
-                if (act(1, g.jbeg)) issue_s(1, sk);
+                int sk;
+                if (pre0) {   // Q waited for and S_0(jbeg) issued at the end of the previous item
+                    sk = pre_sk;
+                    ++it;
+                    pre0 = false;
+                    tc_fence_after();
+                    if (act(1, g.jbeg)) issue_s(1, sk, qbuf);
+                } else {
+                    if (!(ok = wait_q(qi))) break;
+                    sk = it % C::NSTAGE;
+                    ok = mbar_wait(kv_full(sk), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
+                    ++it;
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (act(0, g.jbeg)) issue_s(0, sk, qbuf);
+                    if (act(1, g.jbeg)) issue_s(1, sk, qbuf);
+                }
                 for (int j = g.jbeg; j <= g.jend && ok; ++j) {
                     const int sv = it % C::NSTAGE;
                     ok = mbar_wait(kv_full(sv), (it / C::NSTAGE) & 1, abort_flag, p.wait_limit, kStatusTimeoutMma);
@@ -310,17 +357,38 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 }
                             }
                             tc_fence_after();
-                            issue_pv(t, sv, first);
+                            issue_pv(t, sv, first, 0);
+                            ok = mbar_wait(p_full1(t), uint32_t(npv & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(t, sv, first, 1);
                             first = false;
                             ++npv;
                         }
-                        if (more && act(t, j + 1)) issue_s(t, sk_next);
+                        if (more && act(t, j + 1)) issue_s(t, sk_next, qbuf);
                     }
                     // K_j (read by the S MMAs issued one step earlier) and V_j are free once the
                     // MMAs issued so far complete.
                     tc_commit(kv_empty(sk));
                     tc_commit(kv_empty(sv));
                     sk = sk_next;
+                    if (kEarly && ok && j + 1 == g.jend && !act(0, g.jend)) {
+                        // Tile 0 is done with this item; in use now: K_jend (S_1 issued), V_jend and
+                        // the next item's first K, loading behind it (ring index it + 1).
+                        next_item = item_consume_thread(qi + 1, ring, item_full0, item_empty0, abort_flag,
+                                                        p.wait_limit, kStatusTimeoutMma, ok);
+                        have_next = true;
+                        if (ok && next_item < p.n_items && (ok = wait_q(qi + 1))) {
+                            pre_sk = (it + 1) % C::NSTAGE;
+                            ok = mbar_wait(kv_full(pre_sk), ((it + 1) / C::NSTAGE) & 1, abort_flag, p.wait_limit,
+                                           kStatusTimeoutMma);
+                            if (ok) {
+                                tc_fence_after();
+                                issue_s(0, pre_sk, (qi + 1) % C::NQBUF);   // tile 0 is active at jbeg
+                                pre0 = true;
+                            }
+                        }
+                    }
                 }
                 tc_commit(q_empty(qbuf));   // every S MMA of this item has been issued
                 ++nep0;
@@ -329,6 +397,99 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
         }
+    } else if (kRope && warp >= 10) {
+        // --------------------- Q prologue: rotary embedding + QK norm in shared memory ---------------------
+        // Thread pt takes chunk pair j of a row: the 16-byte chunk j (elements 8j .. 8j+7) and chunk
+        // j + D/16 (their rotation partners, D/2 elements later), in the 128-byte-swizzled tile layout
+        // of the TMA load; the D/16 threads of a row reduce its sum of squares with shuffles.
+        constexpr int TPR = D / 16;                  // threads per row
+        constexpr int RPI = 64 / TPR;                // rows per pass of the 64 threads
+        const int pt = threadIdx.x - C::THREADS;
+        const int j = pt % TPR, rsub = pt / TPR;
+        const unsigned rmask = ((1u << TPR) - 1u) << ((threadIdx.x & 31) & ~(TPR - 1));
+        bool ok = true;
+        for (int qi = 0;; ++qi) {
+            const int item = item_consume_warp(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                               kStatusTimeoutEpilogue, ok);
+            if (!ok || item >= p.n_items) break;
+            const FwdItem g = fwd_item<kOffset>(p, item);
+            const int qb = qi % C::NQBUF;
+            ok = __all_sync(0xffffffffu, mbar_wait(q_full(qb), uint32_t((qi / C::NQBUF) & 1), abort_flag,
+                                                   p.wait_limit, kStatusTimeoutEpilogue));
+            if (!ok) break;
+            const int ntile = g.valid1 ? 2 : 1;
+            for (int t = 0; t < ntile; ++t) {
+                const uint32_t tb = sQ + (qb * C::NQ + t) * C::TILE;
+#pragma unroll 4
+                for (int r0 = 0; r0 < C::BM; r0 += RPI) {
+                    const int r = r0 + rsub;
+                    const long long qrow = g.q0 + t * C::BM + r;
+                    const long long pos = g.L + qrow;
+                    if (qrow >= p.T) continue;                 // zero rows past T: nothing to rotate
+                    if (pos >= p.max_pos) {                    // no table row: left as is, and reported
+                        if (j == 0) report_status(p.stream_slot, kStatusPositionRange);
+                        continue;
+                    }
+                    const int j2 = j + TPR;
+                    const uint32_t a1 = tb + (j / 8) * C::BOX + r * 128 + (((j % 8) ^ (r & 7)) * 16);
+                    const uint32_t a2 = tb + (j2 / 8) * C::BOX + r * 128 + (((j2 % 8) ^ (r & 7)) * 16);
+                    uint4 u1, u2;
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(u1.x), "=r"(u1.y), "=r"(u1.z), "=r"(u1.w) : "r"(a1));
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(u2.x), "=r"(u2.y), "=r"(u2.z), "=r"(u2.w) : "r"(a2));
+                    const float* crow = p.rope_cos + size_t(pos) * (D / 2) + 8 * j;
+                    const float* srow = p.rope_sin + size_t(pos) * (D / 2) + 8 * j;
+                    const float4 c0 = *reinterpret_cast<const float4*>(crow), c1 = *reinterpret_cast<const float4*>(crow + 4);
+                    const float4 s0 = *reinterpret_cast<const float4*>(srow), s1 = *reinterpret_cast<const float4*>(srow + 4);
+                    const float co[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    const float si[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                    float x1[8], x2[8];
+                    bf16x8_unpack(u1, x1);
+                    bf16x8_unpack(u2, x2);
+                    float ss = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {   // r1 = x1 cos - x2 sin,  r2 = x1 sin + x2 cos
+                        const float r1 = fmaf(x1[i], co[i], -x2[i] * si[i]);
+                        const float r2 = fmaf(x1[i], si[i], x2[i] * co[i]);
+                        x1[i] = r1;
+                        x2[i] = r2;
+                        ss = fmaf(r1, r1, ss);
+                        ss = fmaf(r2, r2, ss);
+                    }
+#pragma unroll
+                    for (int off = TPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(rmask, ss, off);
+                    const float ms = ss * (1.f / D) + p.eps;
+                    const float inv = ms > 0.f ? rsqrtf(ms) : 0.f;   // an all-zero row with eps = 0 stays zero
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        x1[i] *= inv;
+                        x2[i] *= inv;
+                    }
+                    u1 = bf16x8_pack(x1);
+                    u2 = bf16x8_pack(x2);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(u1.x), "r"(u1.y), "r"(u1.z),
+                                 "r"(u1.w) : "memory");
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a2), "r"(u2.x), "r"(u2.y), "r"(u2.z),
+                                 "r"(u2.w) : "memory");
+                }
+            }
+            fence_proxy_async_smem();   // the tensor core and the TMA store read the tile through the async proxy
+            mbar_arrive(q_ready(qb));
+            if (p.store_qrot) {
+                named_barrier_sync(2, 64);   // every prologue thread's writes are fenced
+                if (pt == 0) {
+                    for (int t = 0; t < ntile; ++t)
+                        for (int x = 0; x < C::NBOX; ++x)
+                            tma_store_4d(&tm_qr, sQ + (qb * C::NQ + t) * C::TILE + x * C::BOX, x * 64, g.h,
+                                         int(g.q0) + t * C::BM, g.b);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();   // the buffer may be refilled once the store has read it
+                }
+            }
+            if (pt == 0) mbar_arrive(q_empty(qb));
+        }
+        if (pt == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // stores complete before exit
     } else {
         // ------------------------------ softmax warpgroups ------------------------------
         const int t = warp >> 2;            // query tile of this warpgroup
@@ -410,37 +571,50 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_sub));
-                        const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
+                        const float x0 = fmaf(s[c * 64 + 2 * i], sl2, -m_sub);
+                        const float x1 = fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub);
+                        const bool poly = (i & 7) >= 8 - C::POLY8;   // compile-time after unrolling
+                        const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+                        const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
                         sp[(2 * i) & 7] += p0;
                         sp[(2 * i + 1) & 7] += p1;
                         pk[i] = pack_bf16x2_alu(p0, p1);   // integer pipe: exp2 keeps the SFU
                     }
                     tmem_st32(tS + c * 32, pk);
+                    if (c == 0 && !(warp_need && nloc > 0)) {   // keys 0..63 of P are stored
+                        tmem_st_wait();
+                        tc_fence_before();
+                        mbar_arrive(p_full(t));   // the first PV half may start
+                    }
                 }
-                const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-                l_run = l_run * alpha + rowsum;
-                tmem_st_wait();
                 if (warp_need && nloc > 0) {
-                    // O_t holds the sum up to key tile j-1: wait for PV_t(j-1), then rescale.
+                    // O_t must hold the rescaled sum up to key tile j-1 before this tile's first PV
+                    // half runs.  PV_t(j-1) has completed (S_t(j) was issued after it); the o_full
+                    // wait only tracks its phase.  Rare (the running max grew by more than 2^8), so
+                    // the first PV half simply waits for it.
                     ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((ns - 1) & 1), abort_flag,
                                                            p.wait_limit, kStatusTimeoutSoftmax));
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t r[32];
-                        tmem_ld32(tO + c * 32, r);
+                        tmem_ld32(tO + cc * 32, r);
                         tmem_ld_wait(r);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(tO + c * 32, r);
+                        tmem_st32(tO + cc * 32, r);
                     }
                     tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(p_full(t));
                 }
+                const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+                l_run = l_run * alpha + rowsum;
+                tmem_st_wait();
                 m_run = m_use;
                 tc_fence_before();
-                mbar_arrive(p_full(t));
+                mbar_arrive(p_full1(t));
             }
             if (!ok || nloc == 0) break;
             // ---- epilogue: O = O / l, lse = ln(sum exp S) ----
@@ -499,7 +673,8 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
                                                          __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
                                                          const int* __restrict__ cache_len, int B, int Tn, int cap,
                                                          int Hkv, int len_off, int tail, const float* __restrict__ cs,
-                                                         const float* __restrict__ sn, int max_pos, float eps) {
+                                                         const float* __restrict__ sn, int max_pos, float eps,
+                                                         int slot) {
     constexpr int CPR = D / 8;   // 16-byte chunks per head row
     const int span = Tn + tail;  // chunk rows plus the largest zeroed tail
     const long long total = (long long)B * span * Hkv * CPR;
@@ -519,7 +694,7 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
         // every branch below is uniform over the row's threads (it depends on b, t, hk only)
         if (t >= Tn && slot >= tile_end) continue;
         if (slot >= cap) {
-            if (t < Tn) atomicOr(&g_attn_status, kStatusCacheOverflow);
+            if (t < Tn) report_status(slot, kStatusCacheOverflow);
             continue;
         }
         const size_t dst = ((size_t(b) * cap + size_t(slot)) * Hkv + hk) * D + c * 8;
@@ -530,7 +705,7 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
             vw = *reinterpret_cast<const uint4*>(v_new + src);
             if (kRope) {
                 if (slot >= max_pos) {
-                    atomicOr(&g_attn_status, kStatusPositionRange);
+                    report_status(slot, kStatusPositionRange);
                     continue;
                 }
                 float f[8];

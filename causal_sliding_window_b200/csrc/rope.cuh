@@ -108,10 +108,10 @@ __global__ void __launch_bounds__(256) swa_rope_tables_kernel(float* __restrict_
 }
 
 // Position of token t of sequence b, or -1 (status flagged) when it has no table row.
-__device__ __forceinline__ int rope_position(const int* pos0, int b, int t, int max_pos) {
+__device__ __forceinline__ int rope_position(const int* pos0, int b, int t, int max_pos, int slot) {
     const long long pos = (long long)(pos0 ? pos0[b] : 0) + t;
     if (pos < 0 || pos >= max_pos) {
-        atomicOr(&g_attn_status, kStatusPositionRange);
+        report_status(slot, kStatusPositionRange);
         return -1;
     }
     return int(pos);
@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(256) swa_rope_qknorm_kernel(const __nv_bfloat1
                                                               __nv_bfloat16* y, int B, int T, int H,
                                                               const int* __restrict__ pos0,
                                                               const float* __restrict__ cs,
-                                                              const float* __restrict__ sn, int max_pos, float eps) {
+                                                              const float* __restrict__ sn, int max_pos, float eps,
+                                                              int slot) {
     constexpr int CPR = D / 8;
     const long long total = (long long)B * T * H * CPR;   // a multiple of CPR: rows are whole
     const unsigned mask = rope_group_mask<D>();
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(256) swa_rope_qknorm_kernel(const __nv_bfloat1
         const long long row = e / CPR;   // (b, t, h)
         const int t = int((row / H) % T);
         const int b = int(row / ((long long)H * T));
-        const int pos = rope_position(pos0, b, t, max_pos);
+        const int pos = rope_position(pos0, b, t, max_pos, slot);
         if (pos < 0) continue;   // uniform over the row group
         const float* crow = cs + (size_t)pos * (D / 2);
         const float* srow = sn + (size_t)pos * (D / 2);

@@ -14,10 +14,16 @@
 namespace swa {
 
 // ---------------------------------------------------------------------------
-// Device status word.  A wait that gives up (see mbar_wait) ORs a code in
-// here; the host reads it with attn_device_status().
+// Status words.  A wait that gives up (see mbar_wait), or a data-dependent error
+// (cache overflow, position outside the rotary tables), ORs a code into the
+// device-wide word g_attn_status (read by attn_device_status) and into the word
+// of the stream slot the launch was given (read by attn_poll_device_status).
+// The host maps each (device, stream) pair to one of kStreamSlots slots; the
+// same index names the launch's work counter (g_work_slots below).
 // ---------------------------------------------------------------------------
+constexpr int kStreamSlots = 64;
 __device__ int g_attn_status;
+__device__ int g_stream_status[kStreamSlots];
 
 enum : int {
     kStatusTimeoutProducer = 1,
@@ -32,6 +38,11 @@ enum : int {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void report_status(int slot, int code) {
+    atomicOr(&g_attn_status, code);
+    atomicOr(&g_stream_status[slot & (kStreamSlots - 1)], code);
 }
 
 __device__ __forceinline__ long long imax_ll(long long a, long long b) { return a > b ? a : b; }
@@ -72,9 +83,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Gives up after
 // `limit_cycles` SM clocks, or as soon as another role of the CTA has given up
-// (shared `abort_flag`).  On giving up it records `code` in g_attn_status and
-// returns false; callers then stop issuing work and fall through to the
-// kernel's teardown.
+// (shared `abort_flag[0]`).  On giving up it records `code` in the status words
+// (abort_flag[1] holds the launch's stream slot) and returns false; callers then
+// stop issuing work and fall through to the kernel's teardown.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           long long limit_cycles, int code) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -83,10 +94,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
+        if (abort_flag[0]) return false;
         if (clock64() - t0 > limit_cycles) {
-            *abort_flag = 1;
-            atomicOr(&g_attn_status, code);
+            abort_flag[0] = 1;
+            report_status(abort_flag[1], code);
             return false;
         }
     }
@@ -95,11 +106,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Bounded wait used before a CTA exits, for copies it issued itself: unlike mbar_wait it
 // keeps waiting after another role has given up (a TMA copy that was issued completes on
 // its own), but still stops after `limit_cycles`.
-__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, long long limit_cycles) {
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, long long limit_cycles, int slot) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > limit_cycles) {
-            atomicOr(&g_attn_status, kStatusTimeoutProducer);
+            report_status(slot, kStatusTimeoutProducer);
             return false;
         }
     }
@@ -115,9 +126,10 @@ __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, long l
 // the producer thread draws the index and hands it to the other roles through a small
 // shared-memory ring (item_full / item_empty mbarriers).  When a CTA stops drawing it
 // counts itself done; the last CTA of the launch zeroes the slot for a later launch.  The
-// host gives concurrent launches different slots (kWorkSlots of them, round robin).
+// slot is the launch's stream slot: launches on one stream run one after another, so they
+// can share it, and launches on streams with different slots never touch each other's.
 // ---------------------------------------------------------------------------
-constexpr int kWorkSlots = 64;
+constexpr int kWorkSlots = kStreamSlots;
 constexpr int kItemRing = 4;
 struct WorkSlot {
     int next;
@@ -191,6 +203,23 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
+}
+
+// 4-D tiled store shared -> global (bulk-group completion); rows outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk group of this thread has finished reading its shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Barrier over `nthreads` threads (whole warps) on named barrier `id` (1..15).
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Untiled bulk copy global -> shared (both 16-byte aligned, size a multiple of 16).
@@ -328,6 +357,23 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// 2^x on the FMA pipe, for a share of a softmax row's exponentials so that they do not all queue
+// on the special-function unit.  Cody-Waite range reduction: x = j + f with j = round(x), taken
+// from the low mantissa bits of x + 1.5 * 2^23, and |f| <= 1/2; 2^f is a degree-3 polynomial
+// whose coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez exchange;
+// fit_exp2_poly.py derives them: error <= 7.5e-5, far below the bf16 rounding of P); j is added
+// to the exponent field.  x below -125 is clamped there (2^-125 is negligible next to a row's
+// largest term, which is at least 2^-8); x must be at most 127.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = __fadd_rn(x, 12582912.0f);   // 1.5 * 2^23: round(x) in the low mantissa bits
+    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
+    float p = fmaf(f, 0.0551716685f, 0.2426111251f);
+    p = fmaf(p, f, 0.6932609677f);
+    p = fmaf(p, f, 0.9999280572f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Pack two fp32 into bf16x2 with round-to-nearest-even; `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

@@ -7,7 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
-#include <atomic>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -67,11 +67,22 @@ bool ensure_smem(const void* func, int bytes) {
     return true;
 }
 
-// Work-counter slot for the next persistent launch (round robin over kWorkSlots, so that
-// up to kWorkSlots launches may be in flight at once on different streams).
-int next_work_slot() {
-    static std::atomic<unsigned> ctr{0};
-    return int(ctr.fetch_add(1, std::memory_order_relaxed) % unsigned(kWorkSlots));
+// Stream slot of a launch: the first kStreamSlots - 1 distinct streams seen on a device get
+// slots 1, 2, ... of their own; later streams share slot 0.  A slot names both the work
+// counter of the persistent kernels (launches on one stream never overlap, so they can share
+// one) and the status word that attn_poll_device_status(stream) reads.
+int stream_slot(cudaStream_t s) {
+    static std::mutex mu;
+    static std::map<std::pair<int, cudaStream_t>, int> slots;
+    static int used[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> g(mu);
+    auto it = slots.find({dev, s});
+    if (it != slots.end()) return it->second;
+    const int slot = used[dev] + 1 < kStreamSlots ? ++used[dev] : 0;
+    slots[{dev, s}] = slot;
+    return slot;
 }
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -115,18 +126,19 @@ int grid_for(long long work_items, int threads) {
     return int(blocks);
 }
 
-__global__ void swa_selftest_wait_kernel(long long limit_cycles) {
+__global__ void swa_selftest_wait_kernel(long long limit_cycles, int slot) {
     __shared__ __align__(8) uint64_t bar;
-    __shared__ int abort_flag;
+    __shared__ int abort_flag[2];
     const uint32_t a = smem_u32(&bar);
     if (threadIdx.x == 0) {
         mbar_init(a, 1);
-        abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = slot;
         fence_barrier_init();
     }
     __syncthreads();
     // Nobody arrives on this barrier: the wait must give up after limit_cycles.
-    if (threadIdx.x == 0) mbar_wait(a, 0, &abort_flag, limit_cycles, kStatusTimeoutSelftest);
+    if (threadIdx.x == 0) mbar_wait(a, 0, abort_flag, limit_cycles, kStatusTimeoutSelftest);
     __syncthreads();
 }
 
@@ -159,50 +171,7 @@ void* noalloc_scratch() {
 
 extern "C" {
 
-int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B,
-                 int T, int H, int Hkv, int D, int W, float scale, void* stream) {
-    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-        return ATTN_ERR_INVALID_ARG;
-    if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
-    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    const int n_qblk = (T + 255) / 256;
-    const long long n_items = (long long)n_qblk * B * H;
-    if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
-    CUtensorMap mq, mk, mv;
-    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, T, Hkv, D) ||
-        !make_bthd_map(&mv, v, B, T, Hkv, D))
-        return ATTN_ERR_LAUNCH;
-    FwdParams p;
-    p.o = reinterpret_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.B = B;
-    p.T = T;
-    p.H = H;
-    p.G = H / Hkv;
-    p.q_offset = nullptr;
-    p.W = W;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.n_qblk = n_qblk;
-    p.n_items = int(n_items);
-    p.work_slot = next_work_slot();
-    p.wait_limit = kDefaultWaitLimit;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (D == 128) {
-        if (!ensure_smem((const void*)swa_fwd_kernel<128>, FwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_fwd_kernel<128><<<unsigned(grid), FwdCfg<128>::THREADS, FwdCfg<128>::SMEM, s>>>(mq, mk, mv, p);
-    } else {
-        if (!ensure_smem((const void*)swa_fwd_kernel<64>, FwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_fwd_kernel<64><<<unsigned(grid), FwdCfg<64>::THREADS, FwdCfg<64>::SMEM, s>>>(mq, mk, mv, p);
-    }
-    return launch_status();
-}
-
-int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B, int T,
-             int H, int D, int W, float scale, void* stream) {
-    return attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, W, scale, stream);
-}
+}  // extern "C"
 
 // RoPE arguments shared by the fused entry points (null table pointers: no rotation).
 struct RopeArgs {
@@ -214,6 +183,86 @@ struct RopeArgs {
 
 static bool valid_rope(const float* cs, const float* sn, int max_pos, float eps) {
     return cs && sn && aligned16(cs) && aligned16(sn) && max_pos >= 1 && eps >= 0.f && std::isfinite(eps);
+}
+
+// Launches the forward kernel over q [B, T, H, D] against k, v [B, Tk, Hkv, D] (Tk = T, or the cache
+// capacity with q_offset set: query t of sequence b at position q_offset[b] + t).  With rope.cs set
+// the kernel rotates and normalises the queries itself and writes them to q_rot.
+static int launch_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
+                      const int32_t* q_offset, int B, int T, int Tk, int H, int Hkv, int D, int W, float scale,
+                      const RopeArgs& rope, attn_bf16* q_rot, cudaStream_t s) {
+    const int n_qblk = (T + 255) / 256;
+    const long long n_items = (long long)n_qblk * B * H;
+    if (n_items > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    const long long grid = n_items < sm_count() ? n_items : sm_count();   // persistent: one CTA per SM
+    CUtensorMap mq, mk, mv, mqr;
+    if (!make_bthd_map(&mq, q, B, T, H, D) || !make_bthd_map(&mk, k, B, Tk, Hkv, D) ||
+        !make_bthd_map(&mv, v, B, Tk, Hkv, D) || !make_bthd_map(&mqr, q_rot ? q_rot : q, B, T, H, D))
+        return ATTN_ERR_LAUNCH;
+    FwdParams p;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.G = H / Hkv;
+    p.q_offset = q_offset;
+    p.W = W;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.n_qblk = n_qblk;
+    p.n_items = int(n_items);
+    p.stream_slot = stream_slot(s);
+    p.wait_limit = kDefaultWaitLimit;
+    p.rope_cos = rope.cs;
+    p.rope_sin = rope.sn;
+    p.max_pos = rope.max_pos;
+    p.eps = rope.eps;
+    p.store_qrot = q_rot != nullptr;
+    const bool off = q_offset != nullptr, r = rope.cs != nullptr;
+#define SWA_FWD(DD, OO, RR)                                                                                       \
+    do {                                                                                                          \
+        if (!ensure_smem((const void*)swa_fwd_kernel<DD, OO, RR>, FwdCfg<DD>::SMEM)) return ATTN_ERR_LAUNCH;     \
+        swa_fwd_kernel<DD, OO, RR><<<unsigned(grid), FwdCfg<DD>::threads(RR), FwdCfg<DD>::SMEM, s>>>(mq, mk, mv, \
+                                                                                                       mqr, p);  \
+    } while (0)
+    if (D == 128) {
+        if (off) {
+            if (r) SWA_FWD(128, true, true); else SWA_FWD(128, true, false);
+        } else {
+            if (r) SWA_FWD(128, false, true); else SWA_FWD(128, false, false);
+        }
+    } else {
+        if (off) {
+            if (r) SWA_FWD(64, true, true); else SWA_FWD(64, true, false);
+        } else {
+            if (r) SWA_FWD(64, false, true); else SWA_FWD(64, false, false);
+        }
+    }
+#undef SWA_FWD
+    return launch_status();
+}
+
+static int bwd_impl(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
+                    const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace,
+                    size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, const RopeArgs& rope,
+                    const attn_bf16* q_raw, void* stream);
+
+extern "C" {
+
+int attn_fwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B,
+                 int T, int H, int Hkv, int D, int W, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    return launch_fwd(q, k, v, o, lse, nullptr, B, T, T, H, Hkv, D, W, scale, RopeArgs{}, nullptr,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B, int T,
+             int H, int D, int W, float scale, void* stream) {
+    return attn_fwd_gqa(q, k, v, o, lse, B, T, H, H, D, W, scale, stream);
 }
 
 // Launches the append kernel: k_new / v_new rows to slots cache_len[b] + len_off + t, tail zeroed
@@ -228,9 +277,10 @@ static int launch_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf
     auto* kc = reinterpret_cast<__nv_bfloat16*>(k_cache);
     auto* vc = reinterpret_cast<__nv_bfloat16*>(v_cache);
     const bool r = rope.cs != nullptr;
+    const int slot = stream_slot(s);
 #define SWA_APPEND(DD, RR)                                                                                    \
     swa_append_kernel<DD, RR><<<unsigned(blocks), 256, 0, s>>>(kn, vn, kc, vc, cache_len, B, Tn, cap, Hkv, len_off, \
-                                                               tail, rope.cs, rope.sn, rope.max_pos, rope.eps)
+                                                               tail, rope.cs, rope.sn, rope.max_pos, rope.eps, slot)
     if (D == 128) {
         if (r) SWA_APPEND(128, true); else SWA_APPEND(128, false);
     } else {
@@ -255,53 +305,14 @@ static int prefill_impl(const attn_bf16* q, const attn_bf16* k_new, const attn_b
     const long long n_items = (long long)n_qblk * B * H;
     if (n_items > 0x7fffffffLL || (long long)B * (Tn + 128) * Hkv * (D / 8) > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // 0. with RoPE: the chunk's queries rotated and normalised at positions cache_len[b] + t
-    const attn_bf16* q_in = q;
-    if (rope.cs) {
-        const long long rows = (long long)B * Tn * H * (D / 8);
-        const unsigned blocks = unsigned(std::min<long long>((rows + 255) / 256, 148LL * 16));
-        const auto* x = reinterpret_cast<const __nv_bfloat16*>(q);
-        auto* y = reinterpret_cast<__nv_bfloat16*>(q_rot);
-        if (D == 128)
-            swa_rope_qknorm_kernel<128, false><<<blocks, 256, 0, s>>>(x, nullptr, y, B, Tn, H, cache_len, rope.cs,
-                                                                       rope.sn, rope.max_pos, rope.eps);
-        else
-            swa_rope_qknorm_kernel<64, false><<<blocks, 256, 0, s>>>(x, nullptr, y, B, Tn, H, cache_len, rope.cs,
-                                                                      rope.sn, rope.max_pos, rope.eps);
-        if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
-        q_in = q_rot;
-    }
-    // 1. append the chunk's K / V (and zero the rest of its last 128-slot tile)
+    // 1. append the chunk's K / V (and zero the rest of its last 128-slot block); with RoPE the keys
+    // are rotated and normalised on the way in
     if (launch_append(k_new, v_new, k_cache, v_cache, cache_len, B, Tn, cap, Hkv, D, 0, 128, rope, s) != ATTN_OK)
         return ATTN_ERR_LAUNCH;
-    // 2. the forward of the chunk's queries at absolute positions cache_len[b] + t over the cache
-    const long long grid = n_items < sm_count() ? n_items : sm_count();
-    CUtensorMap mq, mk, mv;
-    if (!make_bthd_map(&mq, q_in, B, Tn, H, D) || !make_bthd_map(&mk, k_cache, B, cap, Hkv, D) ||
-        !make_bthd_map(&mv, v_cache, B, cap, Hkv, D))
-        return ATTN_ERR_LAUNCH;
-    FwdParams p;
-    p.o = reinterpret_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.B = B;
-    p.T = Tn;
-    p.H = H;
-    p.G = H / Hkv;
-    p.q_offset = cache_len;
-    p.W = W;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.n_qblk = n_qblk;
-    p.n_items = int(n_items);
-    p.work_slot = next_work_slot();
-    p.wait_limit = kDefaultWaitLimit;
-    if (D == 128) {
-        if (!ensure_smem((const void*)swa_fwd_kernel<128, true>, FwdCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_fwd_kernel<128, true><<<unsigned(grid), FwdCfg<128>::THREADS, FwdCfg<128>::SMEM, s>>>(mq, mk, mv, p);
-    } else {
-        if (!ensure_smem((const void*)swa_fwd_kernel<64, true>, FwdCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_fwd_kernel<64, true><<<unsigned(grid), FwdCfg<64>::THREADS, FwdCfg<64>::SMEM, s>>>(mq, mk, mv, p);
-    }
-    return launch_status();
+    // 2. the forward of the chunk's queries at absolute positions cache_len[b] + t over the cache; with
+    // RoPE the forward kernel rotates and normalises the queries itself (and keeps them in q_rot)
+    return launch_fwd(q, k_cache, v_cache, o, lse, cache_len, B, Tn, cap, H, Hkv, D, W, scale, rope,
+                      rope.cs ? q_rot : nullptr, s);
 }
 
 int attn_prefill(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
@@ -357,8 +368,10 @@ static int rope_qknorm_impl(const attn_bf16* x, const attn_bf16* dy, attn_bf16* 
     const auto* xx = reinterpret_cast<const __nv_bfloat16*>(x);
     const auto* gg = reinterpret_cast<const __nv_bfloat16*>(dy);
     auto* yy = reinterpret_cast<__nv_bfloat16*>(y);
+    const int slot = stream_slot(s);
 #define SWA_ROPE(DD, BB) \
-    swa_rope_qknorm_kernel<DD, BB><<<blocks, 256, 0, s>>>(xx, gg, yy, B, T, H, pos0, rope_cos, rope_sin, max_pos, eps)
+    swa_rope_qknorm_kernel<DD, BB><<<blocks, 256, 0, s>>>(xx, gg, yy, B, T, H, pos0, rope_cos, rope_sin, max_pos, eps, \
+                                                          slot)
     if (D == 128) {
         if (bwd) SWA_ROPE(128, true); else SWA_ROPE(128, false);
     } else {
@@ -389,11 +402,18 @@ int attn_fwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, at
     if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv) || !valid_rope(rope_cos, rope_sin, max_pos, eps))
         return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    int st = rope_qknorm_impl(q, nullptr, q_rot, nullptr, rope_cos, rope_sin, max_pos, B, T, H, D, eps, false, stream);
-    if (st == ATTN_OK)
-        st = rope_qknorm_impl(k, nullptr, k_rot, nullptr, rope_cos, rope_sin, max_pos, B, T, Hkv, D, eps, false, stream);
-    if (st == ATTN_OK) st = attn_fwd_gqa(q_rot, k_rot, v, o, lse, B, T, H, Hkv, D, W, scale, stream);
-    return st;
+    // The keys go through one rotate-and-normalise pass (the backward reads k_rot too, so it is
+    // materialised); the queries are rotated and normalised inside the forward kernel, which also
+    // writes q_rot for the backward.
+    int st = rope_qknorm_impl(k, nullptr, k_rot, nullptr, rope_cos, rope_sin, max_pos, B, T, Hkv, D, eps, false, stream);
+    if (st != ATTN_OK) return st;
+    RopeArgs r;
+    r.cs = rope_cos;
+    r.sn = rope_sin;
+    r.max_pos = max_pos;
+    r.eps = eps;
+    return launch_fwd(q, k_rot, v, o, lse, nullptr, B, T, T, H, Hkv, D, W, scale, r, q_rot,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_bwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* q_rot, const attn_bf16* k_rot,
@@ -404,11 +424,16 @@ int attn_bwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* q_rot
     if (!q || !k || !q_rot || !k_rot || !aligned16(q) || !aligned16(k) || !aligned16(q_rot) || !aligned16(k_rot))
         return ATTN_ERR_INVALID_ARG;
     if (!valid_rope(rope_cos, rope_sin, max_pos, eps)) return ATTN_ERR_INVALID_ARG;
-    // dQ', dK' at the rotated inputs, then back through rotate-and-normalise in place
-    int st = attn_bwd_gqa(q_rot, k_rot, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, Hkv, D, W, scale,
-                          stream);
-    if (st == ATTN_OK)
-        st = rope_qknorm_impl(q, dq, dq, nullptr, rope_cos, rope_sin, max_pos, B, T, H, D, eps, true, stream);
+    // The attention backward at the rotated inputs; its dQ kernel takes dq back through
+    // rotate-and-normalise at the raw q in its epilogue.  dk goes back through it in place, in one
+    // pass after the backward.
+    RopeArgs r;
+    r.cs = rope_cos;
+    r.sn = rope_sin;
+    r.max_pos = max_pos;
+    r.eps = eps;
+    int st = bwd_impl(q_rot, k_rot, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, Hkv, D, W, scale, r, q,
+                      stream);
     if (st == ATTN_OK)
         st = rope_qknorm_impl(k, dk, dk, nullptr, rope_cos, rope_sin, max_pos, B, T, Hkv, D, eps, true, stream);
     return st;
@@ -421,9 +446,14 @@ size_t attn_bwd_workspace_bytes(int B, int T, int H, int D) {
     return 2 * align256(size_t(B) * H * Tp * 4);
 }
 
-int attn_bwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
-                 const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace,
-                 size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, void* stream) {
+}  // extern "C"
+
+// The backward's three launches.  With rope.cs set, q is the rotated, normalised query and the dQ
+// kernel takes dq back through that prologue at q_raw (token t at position t) before writing it.
+static int bwd_impl(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
+                    const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace,
+                    size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, const RopeArgs& rope,
+                    const attn_bf16* q_raw, void* stream) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
     for (const void* ptr : ptrs)
@@ -472,12 +502,18 @@ int attn_bwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, con
     p.n_items = int(n_items);
     p.Tp = Tp;
     p.wait_limit = kDefaultWaitLimit;
+    p.q_raw = reinterpret_cast<const __nv_bfloat16*>(q_raw);
+    p.rope_cos = rope.cs;
+    p.rope_sin = rope.sn;
+    p.max_pos = rope.max_pos;
+    p.eps = rope.eps;
+    const bool r = rope.cs != nullptr;
     // dK, dV (key-stationary, one item per key tile of a K/V head), then dQ (query-stationary, one
     // item per query tile of a query head); each launch draws from its own counter.
     const long long n_items_kv = (long long)n_blk * B * Hkv;
     const long long grid_kv = n_items_kv < sm_count() ? n_items_kv : sm_count();
     p.n_items = int(n_items_kv);
-    p.work_slot = next_work_slot();
+    p.stream_slot = stream_slot(s);
     if (D == 128) {
         if (!ensure_smem((const void*)swa_bwd_dkdv_kernel<128>, BwdKVCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
         swa_bwd_dkdv_kernel<128><<<unsigned(grid_kv), BwdKVCfg<128>::THREADS, BwdKVCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
@@ -488,15 +524,29 @@ int attn_bwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, con
     if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
     if (g_ev_after_main) cudaEventRecord(g_ev_after_main, s);
     p.n_items = int(n_items);
-    p.work_slot = next_work_slot();
+    p.stream_slot = stream_slot(s);
+#define SWA_DQ(DD, RR)                                                                                      \
+    do {                                                                                                    \
+        if (!ensure_smem((const void*)swa_bwd_dq_kernel<DD, RR>, BwdQCfg<DD>::SMEM)) return ATTN_ERR_LAUNCH; \
+        swa_bwd_dq_kernel<DD, RR><<<unsigned(grid), BwdQCfg<DD>::THREADS, BwdQCfg<DD>::SMEM, s>>>(mq, mk, mv,  \
+                                                                                                mdo, p);    \
+    } while (0)
     if (D == 128) {
-        if (!ensure_smem((const void*)swa_bwd_dq_kernel<128>, BwdQCfg<128>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_dq_kernel<128><<<unsigned(grid), BwdQCfg<128>::THREADS, BwdQCfg<128>::SMEM, s>>>(mq, mk, mv, mdo, p);
+        if (r) SWA_DQ(128, true); else SWA_DQ(128, false);
     } else {
-        if (!ensure_smem((const void*)swa_bwd_dq_kernel<64>, BwdQCfg<64>::SMEM)) return ATTN_ERR_LAUNCH;
-        swa_bwd_dq_kernel<64><<<unsigned(grid), BwdQCfg<64>::THREADS, BwdQCfg<64>::SMEM, s>>>(mq, mk, mv, mdo, p);
+        if (r) SWA_DQ(64, true); else SWA_DQ(64, false);
     }
+#undef SWA_DQ
     return launch_status();
+}
+
+extern "C" {
+
+int attn_bwd_gqa(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
+                 const attn_bf16* dout, attn_bf16* dq, attn_bf16* dk, attn_bf16* dv, void* workspace,
+                 size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, void* stream) {
+    return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, Hkv, D, W, scale, RopeArgs{},
+                    nullptr, stream);
 }
 
 int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const attn_bf16* o, const float* lse,
@@ -505,27 +555,38 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     return attn_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, H, D, W, scale, stream);
 }
 
-// Decode geometry for H query heads over Hkv K/V heads: query heads per thread, slots per CTA,
-// (K/V head, query subgroup) pair groups per sequence.
+// Decode geometry for H query heads over Hkv K/V heads: query heads per thread (qpt), query
+// subgroups per K/V head (nsub), K/V heads per head group (gh; a group's (K/V head, subgroup)
+// pairs are the CTA's consumer threads, at most decode_max_consumers(qpt) of them), head groups,
+// cache slots per shared-memory stage (ss, a power of two near 48 KB of K + V per stage) and
+// stages (nstage, about 192 KB in all).
 struct DecGeom {
-    int qpt, nsub, chunk, nzg;
+    int qpt, nsub, gh, ngroups, ss, nstage, threads;
+    size_t smem;
 };
 static DecGeom decode_geom(int H, int Hkv, int D) {
     DecGeom g;
     const int kvg = H / Hkv;
+    const int lph = D / 8;
     g.qpt = decode_qpt(kvg);
     g.nsub = (kvg + g.qpt - 1) / g.qpt;
-    g.chunk = g.qpt == 1 ? kDecodeChunk : kDecodeChunkGrp;
-    const int pairs_per_cta = kDecodeThreads / (D / 8);
-    g.nzg = (Hkv * g.nsub + pairs_per_cta - 1) / pairs_per_cta;
+    g.gh = std::max(1, std::min(Hkv, decode_max_consumers(g.qpt) / lph / g.nsub));
+    g.ngroups = (Hkv + g.gh - 1) / g.gh;
+    const size_t slot_bytes = size_t(2) * g.gh * D * 2;   // K and V of one slot
+    g.ss = 1;
+    while (g.ss < 32 && size_t(2 * g.ss) * slot_bytes <= 49152) g.ss *= 2;
+    const size_t stage = size_t(g.ss) * slot_bytes;
+    g.nstage = int(std::max<size_t>(2, std::min<size_t>(8, 196608 / stage)));
+    g.threads = 32 + (g.gh * g.nsub * lph + 31) / 32 * 32;
+    g.smem = size_t(g.nstage) * stage + 16 * size_t(g.nstage) + 16 * kDecodeItemRing + 64;
     return g;
 }
 
 size_t attn_decode_gqa_workspace_bytes(int B, int cap, int H, int Hkv, int D) {
     if (B < 1 || cap < 1 || H < 1 || (D != 64 && D != 128) || !valid_kv_heads(H, Hkv)) return 0;
     const DecGeom g = decode_geom(H, Hkv, D);
-    const size_t nsm = size_t((cap + g.chunk - 1) / g.chunk);
-    return align256(size_t(B) * g.nzg * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
+    const size_t nsm = size_t((cap + kDecodeChunk - 1) / kDecodeChunk);
+    return align256(size_t(B) * g.ngroups * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
            align256(size_t(B) * nsm * H * D * 4);
 }
 
@@ -544,12 +605,13 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
     if (!valid_common(B, cap, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)) return ATTN_ERR_WORKSPACE;
     const DecGeom g = decode_geom(H, Hkv, D);
-    if (g.nzg > 65535) return ATTN_ERR_UNSUPPORTED;
-    const int nsm = (cap + g.chunk - 1) / g.chunk;
+    const int nsm = (cap + kDecodeChunk - 1) / kDecodeChunk;
     const int span = W < cap ? W : cap;
+    const int nsplit = (span + kDecodeChunk - 1) / kDecodeChunk;
+    const long long n_items = (long long)nsplit * B * g.ngroups;
+    if (n_items > 0x7fff0000LL) return ATTN_ERR_UNSUPPORTED;
     DecParams p;
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
     p.kc = reinterpret_cast<const __nv_bfloat16*>(k_cache);
@@ -558,20 +620,25 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     char* ws = static_cast<char*>(workspace);
-    const size_t cnt_bytes = align256(size_t(B) * g.nzg * 4);
-    p.counters = reinterpret_cast<int*>(ws);
+    const size_t cnt_bytes = align256(size_t(B) * g.ngroups * 4);
+    p.tickets = reinterpret_cast<int*>(ws);
     p.part_ml = reinterpret_cast<float*>(ws + cnt_bytes);
     p.part_o = reinterpret_cast<float*>(ws + cnt_bytes + align256(size_t(B) * nsm * H * 2 * 4));
     p.B = B;
     p.cap = cap;
     p.H = H;
+    p.Hk = Hkv;
     p.kv_group = H / Hkv;
     p.nsub = g.nsub;
-    p.chunk = g.chunk;
+    p.gh = g.gh;
+    p.ngroups = g.ngroups;
+    p.ss = g.ss;
+    p.nstage = g.nstage;
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.nsplit = (span + g.chunk - 1) / g.chunk;
+    p.nsplit = nsplit;
     p.nsplit_max = nsm;
+    p.n_items = int(n_items);
     p.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
     p.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
     p.kc_out = const_cast<__nv_bfloat16*>(p.kc);   // written only with the prologue (attn_decode_rope)
@@ -580,32 +647,39 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     p.rope_sin = rope.sn;
     p.max_pos = rope.max_pos;
     p.eps = rope.eps;
-    const int pairs_per_cta = kDecodeThreads / (D / 8);
-    const int threads = ((std::min(Hkv * g.nsub, pairs_per_cta) * (D / 8)) + 31) / 32 * 32;
-    dim3 grid(p.nsplit, B, g.nzg);
+    p.wait_limit = kDefaultWaitLimit;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-#define SWA_DECODE_LAUNCH(DD, QQ)                                      \
-    do {                                                               \
-        if (rope.cs)                                                   \
-            swa_decode_kernel<DD, QQ, true><<<grid, threads, 0, s>>>(p);  \
-        else                                                           \
-            swa_decode_kernel<DD, QQ, false><<<grid, threads, 0, s>>>(p); \
+    p.stream_slot = stream_slot(s);
+    const long long grid = std::min<long long>(n_items, sm_count());   // persistent: one CTA per SM
+    if (g.smem > 232448) return ATTN_ERR_UNSUPPORTED;   // not reached: stages are sized to fit
+#define SWA_DECODE_LAUNCH(DD, QQ, RR)                                                                  \
+    do {                                                                                               \
+        if (!ensure_smem((const void*)swa_decode_kernel<DD, QQ, RR>, 232448)) return ATTN_ERR_LAUNCH;       \
+        swa_decode_kernel<DD, QQ, RR><<<unsigned(grid), g.threads, g.smem, s>>>(p);                      \
+    } while (0)
+#define SWA_DECODE_QPT(DD, QQ)                    \
+    do {                                          \
+        if (rope.cs)                              \
+            SWA_DECODE_LAUNCH(DD, QQ, true);      \
+        else                                      \
+            SWA_DECODE_LAUNCH(DD, QQ, false);     \
     } while (0)
     if (D == 128) {
         switch (g.qpt) {
-            case 1: SWA_DECODE_LAUNCH(128, 1); break;
-            case 2: SWA_DECODE_LAUNCH(128, 2); break;
-            case 3: SWA_DECODE_LAUNCH(128, 3); break;
-            default: SWA_DECODE_LAUNCH(128, 4); break;
+            case 1: SWA_DECODE_QPT(128, 1); break;
+            case 2: SWA_DECODE_QPT(128, 2); break;
+            case 3: SWA_DECODE_QPT(128, 3); break;
+            default: SWA_DECODE_QPT(128, 4); break;
         }
     } else {
         switch (g.qpt) {
-            case 1: SWA_DECODE_LAUNCH(64, 1); break;
-            case 2: SWA_DECODE_LAUNCH(64, 2); break;
-            case 3: SWA_DECODE_LAUNCH(64, 3); break;
-            default: SWA_DECODE_LAUNCH(64, 4); break;
+            case 1: SWA_DECODE_QPT(64, 1); break;
+            case 2: SWA_DECODE_QPT(64, 2); break;
+            case 3: SWA_DECODE_QPT(64, 3); break;
+            default: SWA_DECODE_QPT(64, 4); break;
         }
     }
+#undef SWA_DECODE_QPT
 #undef SWA_DECODE_LAUNCH
     return launch_status();
 }
@@ -627,7 +701,6 @@ int attn_decode_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16
     if ((reinterpret_cast<uintptr_t>(cache_len) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
     if (!valid_common(B, cap, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)) return ATTN_ERR_WORKSPACE;
     RopeArgs r;
     r.cs = rope_cos;
@@ -656,10 +729,9 @@ int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn
     if (need > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;
     void* ws = noalloc_scratch();
     if (ws == nullptr) return ATTN_ERR_LAUNCH;
-    // The ticket counters at the start of the scratch must be zero when a call begins.
-    const size_t counter_bytes = size_t(B) * decode_geom(H, H, D).nzg * 4;
-    if (cudaMemsetAsync(ws, 0, counter_bytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return ATTN_ERR_LAUNCH;
+    // The ticket counters at the start of the scratch must be zero when a call begins: the array
+    // starts zeroed, and the last CTA of every (sequence, head group) of a decode launch puts its
+    // counter back to zero, so nothing needs clearing here.
     return attn_decode(q, k_cache, v_cache, cache_len, o, lse, ws, kNoAllocScratchBytes, B, cap, H, D, W, scale,
                        stream);
 }
@@ -670,22 +742,45 @@ int attn_bwd_set_profile_events(void* after_pre, void* after_main) {
     return ATTN_OK;
 }
 
+static int status_code(int v) {
+    if (v & swa::kStatusCacheOverflow) return ATTN_ERR_CACHE_OVERFLOW;
+    if (v & swa::kStatusPositionRange) return ATTN_ERR_POSITION_RANGE;
+    return v ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+}
+
 int attn_device_status(int clear) {
     if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_LAUNCH;
     int v = 0;
     if (cudaMemcpyFromSymbol(&v, swa::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
     if (clear) {
         const int zero = 0;
-        if (cudaMemcpyToSymbol(swa::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+        static const int zeros[swa::kStreamSlots] = {0};
+        if (cudaMemcpyToSymbol(swa::g_attn_status, &zero, sizeof(int)) != cudaSuccess ||
+            cudaMemcpyToSymbol(swa::g_stream_status, zeros, sizeof(zeros)) != cudaSuccess)
+            return ATTN_ERR_LAUNCH;
     }
-    if (v & swa::kStatusCacheOverflow) return ATTN_ERR_CACHE_OVERFLOW;
-    if (v & swa::kStatusPositionRange) return ATTN_ERR_POSITION_RANGE;
-    return v ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+    return status_code(v);
+}
+
+int attn_poll_device_status(void* stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int slot = stream_slot(s);
+    int* word = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&word), swa::g_stream_status) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
+    word += slot;
+    int v = 0;
+    // The read is queued behind the stream's work; the clear behind the read.
+    if (cudaMemcpyAsync(&v, word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(word, 0, sizeof(int), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        return ATTN_ERR_LAUNCH;
+    return status_code(v);
 }
 
 int attn_selftest_wait_timeout(long long limit_cycles, void* stream) {
     if (limit_cycles < 1 || limit_cycles > (1LL << 34)) return ATTN_ERR_INVALID_ARG;
-    swa_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    swa_selftest_wait_kernel<<<1, 32, 0, s>>>(limit_cycles, stream_slot(s));
     return launch_status();
 }
 

@@ -81,13 +81,16 @@ _lib.attn_bwd_set_profile_events.argtypes = [_p, _p]
 _lib.attn_bwd_set_profile_events.restype = _i
 _lib.attn_device_status.argtypes = [_i]
 _lib.attn_device_status.restype = _i
+_lib.attn_poll_device_status.argtypes = [_p]
+_lib.attn_poll_device_status.restype = _i
 _lib.attn_selftest_wait_timeout.argtypes = [_ll, _p]
 _lib.attn_selftest_wait_timeout.restype = _i
 _lib.attn_status_string.argtypes = [_i]
 _lib.attn_status_string.restype = ctypes.c_char_p
 
 EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_gqa",
-            "attn_decode_workspace_bytes", "attn_decode_gqa_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_selftest_wait_timeout",
+            "attn_decode_workspace_bytes", "attn_decode_gqa_workspace_bytes", "attn_decode", "attn_decode_gqa", "attn_decode_noalloc", "attn_prefill", "attn_bwd_set_profile_events", "attn_device_status", "attn_poll_device_status",
+            "attn_selftest_wait_timeout",
             "attn_status_string", "attn_rope_tables", "attn_rope_qknorm", "attn_rope_qknorm_bwd",
             "attn_prefill_rope_workspace_bytes", "attn_prefill_rope", "attn_decode_rope", "attn_fwd_rope",
             "attn_bwd_rope"]
@@ -242,6 +245,12 @@ def attn_bwd_set_profile_events(after_pre=None, after_main=None):
 
 def attn_device_status(clear: bool = True) -> int:
     return int(_lib.attn_device_status(1 if clear else 0))
+
+
+def attn_poll_device_status(stream=None) -> int:
+    """Status recorded by the library's kernels on `stream` since its last poll (read and cleared;
+    waits for that stream only)."""
+    return int(_lib.attn_poll_device_status(_stream(stream)))
 
 
 def attn_selftest_wait_timeout(limit_cycles: int, stream=None) -> int:

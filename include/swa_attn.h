@@ -30,15 +30,21 @@
  *    (or ATTN_ERR_UNSUPPORTED for an unsupported D) before anything is
  *    launched.  A failed launch returns ATTN_ERR_LAUNCH.
  *  - Outputs are written with round-to-nearest-even to bf16; lse is fp32.
- *  - attn_fwd and attn_bwd run persistent kernels that draw work from one of 64
- *    counters inside the library (round robin per call); at most 64 such calls may
- *    be executing on the device at the same time (on different streams).
+ *  - Stream slots.  The library gives each (device, stream) pair it sees a slot: the
+ *    first 63 distinct streams of a device get one of their own, later streams share
+ *    slot 0.  A slot holds the work counter that the persistent kernels of attn_fwd,
+ *    attn_bwd and attn_prefill draw their work items from, and a status word.  Calls
+ *    on one stream run one after another and never collide on their slot; calls on
+ *    two streams that share slot 0 must not run at the same time.  A CUDA graph
+ *    captured from these calls keeps the slot of the stream it was captured on, so
+ *    it must not be replayed while eager calls on that stream (or another replay of
+ *    it) are running.
  *  - Device-side waits are bounded.  If one gives up (a condition that
  *    correct use never produces), the kernel stops early and records a flag
- *    that attn_device_status() reports as ATTN_ERR_DEVICE_TIMEOUT.  A prefill
- *    chunk that does not fit its cache is reported there as
- *    ATTN_ERR_CACHE_OVERFLOW, a token position outside the rotary tables as
- *    ATTN_ERR_POSITION_RANGE.
+ *    that attn_device_status() and attn_poll_device_status() report as
+ *    ATTN_ERR_DEVICE_TIMEOUT.  A prefill chunk that does not fit its cache is
+ *    reported there as ATTN_ERR_CACHE_OVERFLOW, a token position outside the
+ *    rotary tables as ATTN_ERR_POSITION_RANGE.
  */
 #ifndef SWA_ATTN_H
 #define SWA_ATTN_H
@@ -140,18 +146,23 @@ int attn_rope_qknorm_bwd(const attn_bf16* x, const attn_bf16* dy, attn_bf16* dx,
 /*
  * Training forward with the prologue: q_rot = rotate-and-normalise(q), k_rot likewise (token t at
  * position t), then attn_fwd_gqa(q_rot, k_rot, v).  q_rot [B, T, H, D] and k_rot [B, T, Hkv, D]
- * bf16 are written (the caller keeps them for attn_bwd_rope).  Other arguments as attn_fwd_gqa
- * and attn_rope_qknorm.
+ * bf16 are written (the caller keeps them for attn_bwd_rope).  The keys go through one
+ * rotate-and-normalise pass; the queries are rotated and normalised inside the forward kernel,
+ * on each query tile in shared memory, which also writes q_rot.  A position outside the tables is
+ * reported as ATTN_ERR_POSITION_RANGE, and the outputs of its token are then undefined.  Other
+ * arguments as attn_fwd_gqa and attn_rope_qknorm.
  */
 int attn_fwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* q_rot, attn_bf16* k_rot,
                   attn_bf16* o, float* lse, const float* rope_cos, const float* rope_sin, int max_pos, float eps,
                   int B, int T, int H, int Hkv, int D, int W, float scale, void* stream);
 
 /*
- * Training backward with the prologue: attn_bwd_gqa at (q_rot, k_rot, v), then dq and dk taken
- * back through rotate-and-normalise at the raw q, k in place (the rounding of q_rot, k_rot to
- * bf16 passes gradients through unchanged, as a cast does).  dq, dk, dv are the gradients with
- * respect to the raw q, k and v.  Workspace as attn_bwd.
+ * Training backward with the prologue: attn_bwd_gqa at (q_rot, k_rot, v), with dq and dk taken
+ * back through rotate-and-normalise at the raw q, k (the rounding of q_rot, k_rot to bf16 passes
+ * gradients through unchanged, as a cast does).  The dQ kernel does this for dq in its epilogue,
+ * before dq is written; dk goes back through it in one pass, in place, after the attention
+ * backward.  dq, dk, dv are the gradients with respect to the raw q, k and v.  Workspace as
+ * attn_bwd.
  */
 int attn_bwd_rope(const attn_bf16* q, const attn_bf16* k, const attn_bf16* q_rot, const attn_bf16* k_rot,
                   const attn_bf16* v, const attn_bf16* o, const float* lse, const attn_bf16* dout, attn_bf16* dq,
@@ -164,10 +175,11 @@ size_t attn_prefill_rope_workspace_bytes(int B, int Tn, int H, int D);
 
 /*
  * attn_prefill with the prologue: q, k_new are the chunk's queries and keys before rotation and
- * norm.  Token t of sequence b is at position cache_len[b] + t: its query is rotated and
- * normalised into the workspace (at least attn_prefill_rope_workspace_bytes bytes, 256-byte
- * aligned), its key on the way into the cache (the append writes the rotated, normalised key),
- * and the forward runs as in attn_prefill.  Tables and eps as attn_rope_qknorm.
+ * norm.  Token t of sequence b is at position cache_len[b] + t: its key is rotated and normalised
+ * on the way into the cache (the append writes the rotated, normalised key), its query inside the
+ * forward kernel, which also writes the rotated queries into the workspace (at least
+ * attn_prefill_rope_workspace_bytes bytes, 256-byte aligned); the forward runs as in
+ * attn_prefill.  Tables and eps as attn_rope_qknorm.
  */
 int attn_prefill_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_cache,
                       attn_bf16* v_cache, const int32_t* cache_len, const float* rope_cos, const float* rope_sin,
@@ -265,11 +277,10 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
 
 /*
  * attn_decode without a caller-provided workspace, for callers that cannot
- * allocate device memory: code that issues its work while a CUDA graph is
- * being captured (cudaMalloc is not allowed there), plugins whose host engine
- * owns a fixed device-memory arena and forbids allocation, and latency-bound
- * token loops where an allocation would synchronise the device.
- * The paper has no counterpart: this is a deployment convenience.
+ * allocate device memory: plugins whose host engine owns a fixed
+ * device-memory arena and forbids allocation outside it, and latency-bound
+ * token loops where an allocation could block on, or synchronise with, the
+ * device.  The paper has no counterpart: this is a deployment convenience.
  *   Arguments as for attn_decode, minus workspace / ws_bytes.
  *   Scratch: a fixed 8 MiB device array inside the library (held by every GPU
  *   that loads it until exit).  Sizes whose attn_decode_workspace_bytes
@@ -277,10 +288,12 @@ int attn_decode_gqa(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf1
  *   ATTN_ERR_UNSUPPORTED, other bad sizes ATTN_ERR_INVALID_ARG.
  *   The first call on a device looks up the array's device address (set-up,
  *   with that device current); make that first call before any stream capture.
- *   Each call zeroes the scratch's ticket counters on `stream`, then runs
- *   attn_decode on it.  All calls share the one array: calls that overlap on
- *   the GPU (other streams, other threads) race and must be serialised by the
- *   caller.  Allocates nothing.
+ *   The decode's ticket counters at the start of the array are zero when the
+ *   library loads and every call leaves them zero again; the partials are
+ *   rewritten by each call before they are read.  All calls share the one
+ *   array: calls that overlap on the GPU (other streams, other threads) race
+ *   and must be serialised by the caller.  Calls no cudaMalloc / cudaFree and
+ *   no allocating library routine.
  */
 int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,
                         const int32_t* cache_len, attn_bf16* o, float* lse, int B, int cap, int H, int D, int W,
@@ -297,18 +310,34 @@ int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn
 int attn_bwd_set_profile_events(void* after_pre, void* after_main);
 
 /*
- * Device status word: returns ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if any
+ * Device-wide status word: returns ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if any
  * kernel of this library gave up a bounded wait (or found its shared-memory
- * window unusable and did no work) since the last clear.
- * Synchronises the current device.  `clear` != 0 resets the word.
+ * window unusable and did no work) since the last clear (ATTN_ERR_CACHE_OVERFLOW /
+ * ATTN_ERR_POSITION_RANGE for those data errors), on any stream.
+ * Synchronises the current device.  `clear` != 0 resets the word and every
+ * stream slot's word.
  */
 int attn_device_status(int clear);
+
+/*
+ * Stream-scoped status: waits for the work already queued on `stream` (that stream
+ * only), then reads and clears the status word of the stream's slot (see "Stream
+ * slots" above) and returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT, ATTN_ERR_CACHE_OVERFLOW
+ * or ATTN_ERR_POSITION_RANGE for what the library's kernels on that stream recorded
+ * since the last poll of it (or since attn_device_status(1)).  Work on other streams
+ * is neither waited for nor reported, unless they share slot 0 with `stream`.
+ * ATTN_ERR_LAUNCH if the read itself fails.
+ * Defined by: the engine's decode loop, which keeps issuing token steps on its own
+ * stream (apidog guide, section 6 "Inference engine").
+ */
+int attn_poll_device_status(void* stream);
 
 /*
  * Diagnostic: launches one tiny kernel whose mbarrier wait can never complete,
  * bounded by `limit_cycles` SM clocks, so that the bounded-wait path can be
  * exercised without faulting or hanging the GPU.  Returns the launch status;
- * attn_device_status() then reports ATTN_ERR_DEVICE_TIMEOUT.
+ * attn_device_status() and attn_poll_device_status(stream) then report
+ * ATTN_ERR_DEVICE_TIMEOUT.
  */
 int attn_selftest_wait_timeout(long long limit_cycles, void* stream);
 

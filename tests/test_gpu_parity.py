@@ -146,7 +146,9 @@ def test_full_size_workloads_sampled(ops, name, W):
     rdq = oracle_dq_rows(x["q"], x["k"], x["v"], x["do"], W, rows)
     gdq = np.stack([got["dq"][b, i, h] for b, h, i in rows])
     assert rel_l2(gdq, rdq) <= G_REL
-    krows = sample_rows(rng, B, T, H, W, 4)[:10]
+    # key rows across the whole item order: the first head's, the last head's (the last items a
+    # CTA draws, after several others) and random ones
+    krows = sample_rows(rng, B, T, H, W, 12)
     rdk, rdv = oracle_dkv_rows(x["q"], x["k"], x["v"], x["do"], W, krows)
     gdk = np.stack([got["dk"][b, j, h] for b, h, j in krows])
     gdv = np.stack([got["dv"][b, j, h] for b, h, j in krows])
@@ -227,6 +229,31 @@ def test_bounded_wait_reports_timeout_without_hanging(ops):
     got = run_fwd_bwd(ops, x, 16, with_bwd=False)
     o, _ = oracle_fwd(x["q"], x["k"], x["v"], 16)
     assert rel_l2(got["o"], o) <= O_REL
+
+
+def test_stream_poll_reports_only_that_streams_timeout(ops):
+    """attn_poll_device_status(stream): a timeout recorded by a kernel on stream A is reported by
+    A's poll (and cleared by it), not by the poll of another stream B; the device-wide word still
+    sees it."""
+    a, b = torch.cuda.Stream(), torch.cuda.Stream()
+    assert ops.attn_device_status(clear=True) == 0
+    assert ops.attn_poll_device_status(a) == 0 and ops.attn_poll_device_status(b) == 0
+    assert ops.attn_selftest_wait_timeout(200_000, stream=a) == 0
+    # B's own work, a real forward, is clean and reported clean.
+    x = inputs.attention_inputs(1, 200, 2, 64, seed=5, with_do=False)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 2, 200), dtype=torch.float32, device="cuda")
+    b.wait_stream(torch.cuda.current_stream())            # the inputs were written on the current stream
+    with torch.cuda.stream(b):
+        ops.attn_fwd(q, k, v, o, lse, 64, stream=b)
+    assert ops.attn_poll_device_status(b) == 0
+    assert ops.attn_poll_device_status(a) == -4            # ATTN_ERR_DEVICE_TIMEOUT, read and cleared
+    assert ops.attn_poll_device_status(a) == 0
+    assert ops.attn_device_status(clear=True) == -4        # the device-wide word saw it too
+    assert ops.attn_device_status(clear=True) == 0
+    ro, _ = oracle_fwd(x["q"], x["k"], x["v"], 64)
+    assert rel_l2(host_f64(o), ro) <= O_REL
 
 
 # ---------------------------------------------------------------------------
@@ -313,17 +340,17 @@ def test_grouped_kv_heads_decode_workload(ops, W):
     check_decode(host_f64(o), host_f64(lse), ro, rl)
 
 
-def test_grouped_decode_rejects_the_plain_workspace_size(ops):
-    """Grouped heads keep more partials per query head than the plain decode workspace holds."""
+def test_grouped_decode_rejects_a_short_workspace(ops):
+    """A workspace below attn_decode_gqa_workspace_bytes is rejected before any launch."""
     B, cap, H, Hkv, D = 2, 300, 12, 4, 128
-    assert ops.attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D) > ops.attn_decode_workspace_bytes(B, cap, H, D)
     x = inputs.decode_inputs(B, cap, H, D, seed=5, cache_len=np.array([10, 300]))
     kc = dev_bf16(np.ascontiguousarray(x["k_cache"][:, :, :Hkv]))
     vc = dev_bf16(np.ascontiguousarray(x["v_cache"][:, :, :Hkv]))
     cl = torch.from_numpy(x["cache_len"]).cuda()
     o = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
-    ws = ops.decode_workspace(B, cap, H, D, "cuda")
+    need = ops.attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(ops.AttnError):
         ops.attn_decode(dev_bf16(x["q"]), kc, vc, cl, o, lse, ws, 100)
 
@@ -387,3 +414,104 @@ def test_prefill_overflow_is_reported_and_stays_in_bounds(ops):
                                   np.zeros((1, cap, H, D), np.uint16), np.array([0]), W)
     assert rel_l2(host_f64(o[:1]), ro) <= O_REL   # the sequence that fits is unaffected
 
+
+
+# ---------------------------------------------------------------------------
+# Multi-item persistent launches, compared element by element.  Every persistent kernel runs
+# one CTA per SM (148) and draws items from a counter, so the state that runs on from one item
+# to the next (K/V ring phases, the Q buffer, the O / dK / dV / dQ accumulators and their
+# free barriers, the item ring) is only exercised when a CTA processes several items.  These
+# shapes give every CTA at least two items in each kernel:
+#   forward items = ceil(T / 256) * B * H, dK/dV items = ceil(T / 128) * B * Hkv,
+#   dQ items = ceil(T / 128) * B * H.
+# ---------------------------------------------------------------------------
+SM_COUNT = 148
+MULTI = [
+    # (B, T, H, Hkv, D, W)
+    (2, 1024, 40, 40, 128, 256),
+    (2, 1024, 40, 40, 128, 1024),
+    (2, 1000, 40, 40, 64, 300),       # D = 64, ragged last query tile
+    (2, 1024, 40, 8, 128, 512),       # grouped K/V heads: 5 query heads per K/V head
+    (3, 700, 48, 48, 128, 10 ** 9),   # full causal, ragged tail
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,W", MULTI)
+def test_multi_item_launches_match_oracle_elementwise(ops, B, T, H, Hkv, D, W):
+    n_fwd = -(-T // 256) * B * H
+    n_dkdv = -(-T // 128) * B * Hkv
+    n_dq = -(-T // 128) * B * H
+    assert min(n_fwd, n_dkdv, n_dq) >= 2 * SM_COUNT, "shape too small to give every CTA two items"
+    x = inputs.attention_inputs(B, T, H, D, seed=900 + T + H + Hkv + (W % 997))
+    x["k"] = np.ascontiguousarray(x["k"][:, :, :Hkv])
+    x["v"] = np.ascontiguousarray(x["v"][:, :, :Hkv])
+    q, k, v, do = (dev_bf16(x[n]) for n in ("q", "k", "v", "do"))
+    o, lse = Guarded((B, T, H, D), torch.bfloat16), Guarded((B, H, T), torch.float32)
+    dq = Guarded((B, T, H, D), torch.bfloat16)
+    dk, dv = Guarded((B, T, Hkv, D), torch.bfloat16), Guarded((B, T, Hkv, D), torch.bfloat16)
+    ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device="cuda")
+    ops.attn_fwd(q, k, v, o.t, lse.t, W)
+    ops.attn_bwd(q, k, v, o.t, lse.t, do, dq.t, dk.t, dv.t, ws, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    for g in (o, lse, dq, dk, dv):
+        assert g.guards_intact(), "write outside an output buffer"
+    ro, rl = oracle_fwd(x["q"], x["k"], x["v"], W)
+    rdq, rdk, rdv = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    go, gl = host_f64(o.t), host_f64(lse.t)
+    assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
+    assert np.max(np.abs(gl - rl)) <= LSE_ABS
+    for name, got, ref in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
+        g = host_f64(got.t)
+        assert rel_l2(g, ref) <= G_REL, (name, rel_l2(g, ref))
+    # every (b, h) slice on its own, so that no slice hides behind the whole-tensor norm
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(go[b, :, h], ro[b, :, h]) <= O_REL, (b, h)
+            assert rel_l2(host_f64(dq.t[b, :, h]), rdq[b, :, h]) <= G_REL, (b, h)
+
+
+def test_multi_item_prefill_matches_oracle(ops):
+    """Chunked prefill whose forward launch has B * H * ceil(Tn / 256) = 320 items."""
+    B, Tn, cap, H, Hkv, D, W = 8, 512, 2048, 20, 4, 128, 700
+    assert B * H * -(-Tn // 256) >= 2 * SM_COUNT
+    L = inputs.uniform_int(31, "cache_len", B, 0, cap - Tn).astype(np.int32)
+    x = inputs.attention_inputs(B, Tn, H, D, seed=31)
+    c = inputs.decode_inputs(B, cap, Hkv, D, seed=32)
+    kn, vn = (np.ascontiguousarray(x[n][:, :, :Hkv]) for n in ("k", "v"))
+    kc, vc = c["k_cache"].copy(), c["v_cache"].copy()
+    for b in range(B):
+        kc[b, L[b] + Tn:] = NAN_BF16
+        vc[b, L[b] + Tn:] = NAN_BF16
+    o, lse = ops.prefill(dev_bf16(x["q"]), dev_bf16(kn), dev_bf16(vn), dev_bf16(kc), dev_bf16(vc),
+                         torch.from_numpy(L).cuda(), W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == 0
+    ro, rl, _, _ = oracle_prefill(x["q"], kn, vn, kc, vc, L, W)
+    go, gl = host_f64(o), host_f64(lse)
+    assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
+    assert np.max(np.abs(gl - rl)) <= LSE_ABS
+
+
+def test_depth24_short_window_complete_slices(ops):
+    """The depth-24 workload at W = 512, in the launch configuration the benchmark times: four
+    complete (b, h) slices spread over the item order (the first head, two middle ones and the
+    last, whose items are the last any CTA draws) compared on every row of O, lse and dQ and on
+    every key row of dK and dV."""
+    cfg = inputs.WORKLOADS["d24"]
+    B, T, H, D, W = cfg["B"], cfg["T"], cfg["H"], cfg["D"], 512
+    x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"])
+    got = run_fwd_bwd(ops, x, W)
+    slices = [(0, 0), (B // 3, H // 2), (2 * B // 3, 1), (B - 1, H - 1)]
+    rows = np.array([(b, h, i) for b, h in slices for i in range(T)], dtype=np.int64)
+    ro, rl = oracle_fwd_rows(x["q"], x["k"], x["v"], W, rows)
+    rdq = oracle_dq_rows(x["q"], x["k"], x["v"], x["do"], W, rows)
+    rdk, rdv = oracle_dkv_rows(x["q"], x["k"], x["v"], x["do"], W, rows)
+    for s, (b, h) in enumerate(slices):
+        sl = slice(s * T, (s + 1) * T)
+        go, gl = got["o"][b, :, h], got["lse"][b, h]
+        assert rel_l2(go, ro[sl]) <= O_REL and np.max(np.abs(go - ro[sl])) <= O_ABS, (b, h)
+        assert np.max(np.abs(gl - rl[sl])) <= LSE_ABS, (b, h)
+        assert rel_l2(got["dq"][b, :, h], rdq[sl]) <= G_REL, (b, h)
+        assert rel_l2(got["dk"][b, :, h], rdk[sl]) <= G_REL, (b, h)
+        assert rel_l2(got["dv"][b, :, h], rdv[sl]) <= G_REL, (b, h)

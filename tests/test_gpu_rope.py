@@ -162,7 +162,8 @@ def test_decode_with_rope_matches_oracle(ops, H, Hkv, D):
         assert np.isnan(gk[b, L:]).all()       # slots after the new token are not written
 
 
-@pytest.mark.parametrize("B,T,H,Hkv,D,W", [(2, 300, 4, 2, 128, 129), (1, 257, 2, 2, 64, 10 ** 9)])
+@pytest.mark.parametrize("B,T,H,Hkv,D,W", [(2, 300, 4, 2, 128, 129), (1, 257, 2, 2, 64, 10 ** 9),
+                                            (2, 1024, 40, 8, 128, 512)])   # every CTA runs several items
 def test_training_forward_and_backward_with_rope(ops, B, T, H, Hkv, D, W):
     from oracle import oracle_bwd_rope, oracle_fwd_rope
 
@@ -181,6 +182,10 @@ def test_training_forward_and_backward_with_rope(ops, B, T, H, Hkv, D, W):
     torch.cuda.synchronize()
     assert ops.attn_device_status(clear=True) == 0
     assert all(g.guards_intact() for g in (o, lse, dq, dk, dv))
+    # the rotated queries the forward kernel wrote (its in-kernel prologue) and the rotated keys
+    pos = np.arange(T)[None, :]
+    _check_rounded(host_f64(q_rot), oracle_rope_qknorm(x["q"], pos, EPS))
+    _check_rounded(host_f64(k_rot), oracle_rope_qknorm(k, pos, EPS))
     ro, rl = oracle_fwd_rope(x["q"], k, v, W, EPS)
     go, gl = host_f64(o.t), host_f64(lse.t)
     assert rel_l2(go, ro) <= O_REL and np.max(np.abs(go - ro)) <= O_ABS
@@ -188,3 +193,20 @@ def test_training_forward_and_backward_with_rope(ops, B, T, H, Hkv, D, W):
     rdq, rdk, rdv = oracle_bwd_rope(x["q"], k, v, x["do"], W, EPS)
     for got, ref in ((dq, rdq), (dk, rdk), (dv, rdv)):
         assert rel_l2(host_f64(got.t), ref) <= G_REL
+
+
+def test_training_forward_with_rope_reports_positions_outside_the_tables(ops):
+    """Tables shorter than the sequence: the forward's in-kernel prologue flags the positions it
+    cannot rotate (ATTN_ERR_POSITION_RANGE) and rotates the others."""
+    B, T, H, D, W = 1, 300, 2, 128, 64
+    x = inputs.attention_inputs(B, T, H, D, seed=77, with_do=False)
+    cos, sin = ops.rope_tables(200, D, "cuda")
+    q_d, k_d, v_d = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    q_rot, k_rot = torch.empty_like(q_d), torch.empty_like(k_d)
+    o = torch.empty_like(q_d)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    ops.attn_fwd_rope(q_d, k_d, v_d, q_rot, k_rot, o, lse, cos, sin, EPS, W)
+    torch.cuda.synchronize()
+    assert ops.attn_device_status(clear=True) == -7   # ATTN_ERR_POSITION_RANGE
+    _check_rounded(host_f64(q_rot)[:, :200], oracle_rope_qknorm(x["q"][:, :200], np.arange(200)[None, :], EPS))
+    assert ops.attn_device_status(clear=True) == 0
