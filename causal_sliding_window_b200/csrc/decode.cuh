@@ -39,6 +39,10 @@ constexpr int kDecodeChunk = 64;           // window slots per work item
 __host__ __device__ constexpr int decode_max_consumers(int qpt) { return qpt == 1 ? 384 : 256; }
 constexpr int kDecodeUnroll = 4;           // slots per batch of loads from shared memory
 constexpr int kDecodeItemRing = 4;
+// Up to this many sequences, every CTA first builds the prefix sum of the sequences' chunk counts
+// in shared memory, so that item i of the launch maps straight to a chunk that holds window slots;
+// larger batches enumerate every (chunk, sequence) and skip the empty ones while drawing.
+constexpr int kDecodePrefixMax = 4096;
 
 struct DecParams {
     const __nv_bfloat16* q;        // [B,H,D]
@@ -61,7 +65,7 @@ struct DecParams {
     float scale_log2;
     int nsplit;                    // chunks per sequence: ceil(min(W, cap) / kDecodeChunk)
     int nsplit_max;                // stride of the partial arrays: ceil(cap / kDecodeChunk)
-    int n_items;                   // nsplit * B * ngroups
+    int n_items;                   // nsplit * B * ngroups: items without the prefix (B > kDecodePrefixMax)
     // kRope: the query is rotated and normalised at its position cache_len[b] - 1 (rope.cuh), and
     // the new token's key (rotated, normalised) and value are written into that slot first
     const __nv_bfloat16* k_new;    // [B, Hk, D]
@@ -97,17 +101,29 @@ inline int decode_qpt(int kv_group) {
     return 4;
 }
 
-// Window geometry of sequence b and its chunk c.
+// Window geometry of sequence b and its chunk c.  With the prefix (pref[b] = chunks of sequences
+// before b, pref[B] = all of them) item = chunk index over all sequences * ngroups + group;
+// without it, item = (c * B + b) * ngroups + g over every possible chunk.
 struct DecItem {
     int b, c, g;
     int L, lo, start, end;
 };
-__device__ __forceinline__ DecItem dec_item(const DecParams& p, int item) {
+__device__ __forceinline__ DecItem dec_item(const DecParams& p, int item, const int* pref) {
     DecItem it;
     it.g = item % p.ngroups;
     const int r = item / p.ngroups;
-    it.b = r % p.B;
-    it.c = r / p.B;
+    if (pref) {   // largest b with pref[b] <= r
+        int lo = 0, hi = p.B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pref[mid] <= r) lo = mid; else hi = mid - 1;
+        }
+        it.b = lo;
+        it.c = r - pref[lo];
+    } else {
+        it.b = r % p.B;
+        it.c = r / p.B;
+    }
     int L = p.cache_len[it.b];
     it.L = L < 0 ? 0 : (L > p.cap ? p.cap : L);
     const long long lo_ll = (long long)it.L - p.W;
@@ -139,7 +155,37 @@ __global__ void __launch_bounds__(32 + decode_max_consumers(QPT), 1) swa_decode_
     volatile int* abort_flag = misc;                 // [0] abort, [1] stream slot
     volatile int* ring = misc + 2;                   // kDecodeItemRing entries
     volatile int* is_last = misc + 2 + kDecodeItemRing;
+    int* pref = p.B <= kDecodePrefixMax ? const_cast<int*>(misc + 8) : nullptr;   // [B + 1]
     const int tid = threadIdx.x, lane = tid & 31;
+    if (pref) {
+        // chunks per sequence (chunk 0 always counts), then their exclusive prefix sum: warp 0
+        // scans, each lane over a contiguous run of sequences
+        for (int b = tid; b < p.B; b += blockDim.x) {
+            int L = p.cache_len[b];
+            L = L < 0 ? 0 : (L > p.cap ? p.cap : L);
+            const long long lo = (long long)L - p.W;
+            const int n = L - (lo < 0 ? 0 : int(lo));
+            pref[b + 1] = max(1, (n + kDecodeChunk - 1) / kDecodeChunk);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            const int per = (p.B + 31) / 32, b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
+            int sum = 0;
+            for (int b = b0; b < b1; ++b) sum += pref[b + 1];
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            int run = incl - sum;   // chunks of the sequences before b0
+            if (tid == 0) pref[0] = 0;
+            for (int b = b0; b < b1; ++b) {
+                run += pref[b + 1];
+                pref[b + 1] = run;
+            }
+        }
+    }
 
     if (tid == 0) {
         for (int s = 0; s < p.nstage; ++s) {
@@ -155,6 +201,7 @@ __global__ void __launch_bounds__(32 + decode_max_consumers(QPT), 1) swa_decode_
         fence_barrier_init();
     }
     __syncthreads();
+    const int n_items = pref ? pref[p.B] * p.ngroups : p.n_items;
 
     if (tid < 32) {
         // ------------------------------ producer: bulk copies of K / V rows ------------------------------
@@ -169,8 +216,8 @@ __global__ void __launch_bounds__(32 + decode_max_consumers(QPT), 1) swa_decode_
                                    abort_flag, p.wait_limit, kStatusTimeoutProducer);
                 while (ok) {   // draw until an item holds window slots (chunk 0 always counts)
                     const int it = atomicAdd(&g_work_slots[p.stream_slot].next, 1);
-                    if (it >= p.n_items) break;
-                    g = dec_item(p, it);
+                    if (it >= n_items) break;
+                    g = dec_item(p, it, pref);
                     if (g.start < g.end || g.c == 0) {
                         item = it;
                         break;
@@ -226,7 +273,7 @@ __global__ void __launch_bounds__(32 + decode_max_consumers(QPT), 1) swa_decode_
         __syncwarp();
         if (lane == 0) mbar_arrive(item_empty0 + 8u * e);
         if (item == 0x7fffffff) break;
-        const DecItem g = dec_item(p, item);
+        const DecItem g = dec_item(p, item, pref);
         const int hk0 = g.g * p.gh;
         const int npairs = min(p.gh, p.Hk - hk0) * p.nsub;
         const bool live = lp < npairs;

@@ -39,16 +39,12 @@ struct FwdCfg {
     static constexpr int NBOX = D / 64;
     static constexpr int NQBUF = 1;                 // Q buffers (2: the next item's Q loads a whole item ahead)
     static constexpr int NSTAGE = D == 128 ? 5 : 8; // K/V ring (a stage holds one K or one V tile)
-    // Exponentials of a score row evaluated on the FMA pipe (exp2_poly) instead of the special-
-    // function unit: pairs i of each 64-column half with (i & 7) >= 8 - POLY8, i.e. POLY8 / 8 of them.
-    static constexpr int POLY8 = 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = NQBUF * NQ * TILE;
     static constexpr int OFF_BAR = OFF_KV + NSTAGE * TILE;
-    // kv_full, kv_empty per stage; q_full, q_empty per Q buffer; s_full, p_full (keys 0..63 of P),
-    // o_full, o_free, p_full1 (keys 64..127) per tile; q_ready per Q buffer; mma_done; item_full,
-    // item_empty per entry of the item ring
-    static constexpr int NUM_BAR = 2 * NSTAGE + 3 * NQBUF + 5 * NQ + 1 + 2 * kItemRing;
+    // kv_full, kv_empty per stage; q_full, q_empty per Q buffer; s_full, p_full, o_full, o_free per
+    // tile; q_ready per Q buffer; mma_done; item_full, item_empty per entry of the item ring
+    static constexpr int NUM_BAR = 2 * NSTAGE + 3 * NQBUF + 4 * NQ + 1 + 2 * kItemRing;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
@@ -152,9 +148,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto p_full = [&](int t) { return bt + 8u * (C::NQ + t); };
     auto o_full = [&](int t) { return bt + 8u * (2 * C::NQ + t); };
     auto o_free = [&](int t) { return bt + 8u * (3 * C::NQ + t); };
-    auto p_full1 = [&](int t) { return bt + 8u * (4 * C::NQ + t); };
-    auto q_ready = [&](int qb) { return bt + 8u * (5 * C::NQ + qb); };   // kRope: Q rotated in place
-    const uint32_t mma_done = bt + 8u * (5 * C::NQ + C::NQBUF);
+    auto q_ready = [&](int qb) { return bt + 8u * (4 * C::NQ + qb); };   // kRope: Q rotated in place
+    const uint32_t mma_done = bt + 8u * (4 * C::NQ + C::NQBUF);
     const uint32_t item_full0 = mma_done + 8u, item_empty0 = item_full0 + 8u * kItemRing;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
@@ -177,7 +172,6 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int t = 0; t < C::NQ; ++t) {
             mbar_init(s_full(t), 1);
             mbar_init(p_full(t), 128);
-            mbar_init(p_full1(t), 128);
             mbar_init(o_full(t), 1);
             mbar_init(o_free(t), 128);
         }
@@ -269,16 +263,14 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 tc_commit(s_full(t));
             };
-            // PV over keys 0..63 (half 0) or 64..127 (half 1) of the tile: the softmax warps publish
-            // P in these two halves, so the first half's MMAs run while the second half is computed.
-            auto issue_pv = [&](int t, int stage, bool first, int half) {
+            auto issue_pv = [&](int t, int stage, bool first) {
                 const uint32_t va = sKV + stage * C::TILE;
                 const uint32_t a = t ? tS1 : tS0, d = t ? tO1 : tO0;
 #pragma unroll
-                for (int kk = half * (C::BN / 32); kk < (half + 1) * (C::BN / 32); ++kk)
+                for (int kk = 0; kk < C::BN / 16; ++kk)
                     mma_ts(d, a + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX, 1024), C::IDESC_PV,
                            (!first || kk > 0) ? 1u : 0u);
-                if (half) tc_commit(o_full(t));
+                tc_commit(o_full(t));
             };
             auto wait_q = [&](int k) {   // the Q tiles of this CTA's k-th item are in place
                 return mbar_wait(kRope ? q_ready(k % C::NQBUF) : q_full(k % C::NQBUF), uint32_t((k / C::NQBUF) & 1),
@@ -357,11 +349,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 }
                             }
                             tc_fence_after();
-                            issue_pv(t, sv, first, 0);
-                            ok = mbar_wait(p_full1(t), uint32_t(npv & 1), abort_flag, p.wait_limit, kStatusTimeoutMma);
-                            if (!ok) break;
-                            tc_fence_after();
-                            issue_pv(t, sv, first, 1);
+                            issue_pv(t, sv, first);
                             first = false;
                             ++npv;
                         }
@@ -571,50 +559,37 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float x0 = fmaf(s[c * 64 + 2 * i], sl2, -m_sub);
-                        const float x1 = fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub);
-                        const bool poly = (i & 7) >= 8 - C::POLY8;   // compile-time after unrolling
-                        const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-                        const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+                        const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_sub));
+                        const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
                         sp[(2 * i) & 7] += p0;
                         sp[(2 * i + 1) & 7] += p1;
                         pk[i] = pack_bf16x2_alu(p0, p1);   // integer pipe: exp2 keeps the SFU
                     }
                     tmem_st32(tS + c * 32, pk);
-                    if (c == 0 && !(warp_need && nloc > 0)) {   // keys 0..63 of P are stored
-                        tmem_st_wait();
-                        tc_fence_before();
-                        mbar_arrive(p_full(t));   // the first PV half may start
-                    }
                 }
+                const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+                l_run = l_run * alpha + rowsum;
+                tmem_st_wait();
                 if (warp_need && nloc > 0) {
-                    // O_t must hold the rescaled sum up to key tile j-1 before this tile's first PV
-                    // half runs.  PV_t(j-1) has completed (S_t(j) was issued after it); the o_full
-                    // wait only tracks its phase.  Rare (the running max grew by more than 2^8), so
-                    // the first PV half simply waits for it.
+                    // O_t holds the sum up to key tile j-1: wait for PV_t(j-1), then rescale.
                     ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((ns - 1) & 1), abort_flag,
                                                            p.wait_limit, kStatusTimeoutSoftmax));
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
+                    for (int c = 0; c < D / 32; ++c) {
                         uint32_t r[32];
-                        tmem_ld32(tO + cc * 32, r);
+                        tmem_ld32(tO + c * 32, r);
                         tmem_ld_wait(r);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(tO + cc * 32, r);
+                        tmem_st32(tO + c * 32, r);
                     }
                     tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(p_full(t));
                 }
-                const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-                l_run = l_run * alpha + rowsum;
-                tmem_st_wait();
                 m_run = m_use;
                 tc_fence_before();
-                mbar_arrive(p_full1(t));
+                mbar_arrive(p_full(t));
             }
             if (!ok || nloc == 0) break;
             // ---- epilogue: O = O / l, lse = ln(sum exp S) ----

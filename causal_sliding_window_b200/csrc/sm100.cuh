@@ -357,23 +357,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// 2^x on the FMA pipe, for a share of a softmax row's exponentials so that they do not all queue
-// on the special-function unit.  Cody-Waite range reduction: x = j + f with j = round(x), taken
-// from the low mantissa bits of x + 1.5 * 2^23, and |f| <= 1/2; 2^f is a degree-3 polynomial
-// whose coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez exchange;
-// fit_exp2_poly.py derives them: error <= 7.5e-5, far below the bf16 rounding of P); j is added
-// to the exponent field.  x below -125 is clamped there (2^-125 is negligible next to a row's
-// largest term, which is at least 2^-8); x must be at most 127.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = __fadd_rn(x, 12582912.0f);   // 1.5 * 2^23: round(x) in the low mantissa bits
-    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
-    float p = fmaf(f, 0.0551716685f, 0.2426111251f);
-    p = fmaf(p, f, 0.6932609677f);
-    p = fmaf(p, f, 0.9999280572f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Pack two fp32 into bf16x2 with round-to-nearest-even; `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

@@ -651,11 +651,13 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     p.stream_slot = stream_slot(s);
     const long long grid = std::min<long long>(n_items, sm_count());   // persistent: one CTA per SM
-    if (g.smem > 232448) return ATTN_ERR_UNSUPPORTED;   // not reached: stages are sized to fit
+    // the prefix of the sequences' chunk counts, after the fixed scalars (kDecodePrefixMax sequences)
+    const size_t smem = g.smem + (B <= kDecodePrefixMax ? size_t(B + 1) * 4 : 0);
+    if (smem > 232448) return ATTN_ERR_UNSUPPORTED;   // not reached: stages are sized to fit
 #define SWA_DECODE_LAUNCH(DD, QQ, RR)                                                                  \
     do {                                                                                               \
         if (!ensure_smem((const void*)swa_decode_kernel<DD, QQ, RR>, 232448)) return ATTN_ERR_LAUNCH;       \
-        swa_decode_kernel<DD, QQ, RR><<<unsigned(grid), g.threads, g.smem, s>>>(p);                      \
+        swa_decode_kernel<DD, QQ, RR><<<unsigned(grid), g.threads, smem, s>>>(p);                        \
     } while (0)
 #define SWA_DECODE_QPT(DD, QQ)                    \
     do {                                          \

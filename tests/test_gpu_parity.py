@@ -431,7 +431,7 @@ MULTI = [
     (2, 1024, 40, 40, 128, 256),
     (2, 1024, 40, 40, 128, 1024),
     (2, 1000, 40, 40, 64, 300),       # D = 64, ragged last query tile
-    (2, 1024, 40, 8, 128, 512),       # grouped K/V heads: 5 query heads per K/V head
+    (4, 1024, 40, 10, 128, 512),      # grouped K/V heads: 4 query heads per K/V head
     (3, 700, 48, 48, 128, 10 ** 9),   # full causal, ragged tail
 ]
 
