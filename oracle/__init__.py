@@ -20,6 +20,7 @@ from .swa_oracle import (  # noqa: F401
     oracle_prefill,
     oracle_threads,
 )
+from .fp8_oracle import oracle_fwd_fp8, quantize_e4m3, round_e4m3  # noqa: F401
 from .rope_oracle import (  # noqa: F401
     oracle_bwd_rope,
     oracle_decode_rope,
