@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libswa_b200.so")
 SOURCES = ["swa_attn.cu"]
-DEPS = ["swa_attn.cu", "sm100.cuh", "fwd.cuh", "bwd.cuh", "decode.cuh", "rope.cuh"]
+DEPS = ["swa_attn.cu", "sm100.cuh", "fwd.cuh", "fwd_fp8.cuh", "bwd.cuh", "decode.cuh", "rope.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "swa_attn.h")
 
 NVCC_FLAGS = [

@@ -254,22 +254,22 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             int nep0 = 0, nep1 = 0;   // items processed per tile (= epilogues owed)
             int qbuf = 0;   // Q buffer of the current item
             auto issue_s = [&](int t, int stage, int qb) {
-                const uint32_t qa = sQ + (qb * C::NQ + t) * C::TILE, ka = sKV + stage * C::TILE;
+                const SDesc qd = sdesc_sw128_w(sQ + (qb * C::NQ + t) * C::TILE, 16, 1024);
+                const SDesc kd = sdesc_sw128_w(sKV + stage * C::TILE, 16, 1024);
                 const uint32_t d = t ? tS1 : tS0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), C::IDESC_S, kk > 0);
+                    const uint32_t off = ((kk >> 2) * C::BOX + (kk & 3) * 32) >> 4;
+                    mma_ss_w(d, qd.lo + off, qd.hi, kd.lo + off, kd.hi, C::IDESC_S, kk > 0);
                 }
                 tc_commit(s_full(t));
             };
             auto issue_pv = [&](int t, int stage, bool first) {
-                const uint32_t va = sKV + stage * C::TILE;
+                const SDesc vd = sdesc_sw128_w(sKV + stage * C::TILE, C::BOX, 1024);
                 const uint32_t a = t ? tS1 : tS0, d = t ? tO1 : tO0;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ts(d, a + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX, 1024), C::IDESC_PV,
-                           (!first || kk > 0) ? 1u : 0u);
+                    mma_ts_w(d, a + kk * 8, vd.lo + kk * (2048 >> 4), vd.hi, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
                 tc_commit(o_full(t));
             };
             auto wait_q = [&](int k) {   // the Q tiles of this CTA's k-th item are in place

@@ -298,6 +298,41 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// The same descriptor split into its two 32-bit words, for the issue loops: lo holds the start
+// address (>> 4, bits 0..13) and the leading byte offset (bits 16..29), hi the stride byte offset,
+// the version and the swizzle mode.  An operand n bytes further on is lo + (n >> 4) (shared-memory
+// addresses stay below 2^18, so the 14-bit address field never carries), which keeps the issuing
+// thread to one integer add per operand and MMA.
+struct SDesc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc_sw128_w(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return {((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16), ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29)};
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T (kind::f16), descriptors as (lo, hi) words.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "mov.b64 da, {%1, %2};\n\t"
+        "mov.b64 db, {%3, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc]^T (kind::f16), B as (lo, hi) words.
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t blo, uint32_t bhi,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // 32 lanes x 32 columns of 32-bit TMEM words: thread i of the warp gets
 // columns [c, c+32) of lane (warp quarter * 32 + i).
 #define SWA_R8(o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), \
@@ -318,6 +353,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
                   "+r"(r[o + 5]), "+r"(r[o + 6]), "+r"(r[o + 7])
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : SWA_W8(0), SWA_W8(8), SWA_W8(16), SWA_W8(24)::"memory");
+}
+#undef SWA_W8
+
+// 32 lanes x 16 columns.
+#define SWA_R8(o) "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), \
+                  "=r"(r[o + 5]), "=r"(r[o + 6]), "=r"(r[o + 7])
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : SWA_R8(0), SWA_R8(8)
+        : "r"(taddr));
+}
+#undef SWA_R8
+#define SWA_W8(o) "+r"(r[o + 0]), "+r"(r[o + 1]), "+r"(r[o + 2]), "+r"(r[o + 3]), "+r"(r[o + 4]), \
+                  "+r"(r[o + 5]), "+r"(r[o + 6]), "+r"(r[o + 7])
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : SWA_W8(0), SWA_W8(8)::"memory");
 }
 #undef SWA_W8
 

@@ -16,6 +16,7 @@
 #include "bwd.cuh"
 #include "decode.cuh"
 #include "fwd.cuh"
+#include "fwd_fp8.cuh"
 #include "rope.cuh"
 
 namespace {
@@ -555,38 +556,27 @@ int attn_bwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, const a
     return attn_bwd_gqa(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, T, H, H, D, W, scale, stream);
 }
 
-// Decode geometry for H query heads over Hkv K/V heads: query heads per thread (qpt), query
-// subgroups per K/V head (nsub), K/V heads per head group (gh; a group's (K/V head, subgroup)
-// pairs are the CTA's consumer threads, at most decode_max_consumers(qpt) of them), head groups,
-// cache slots per shared-memory stage (ss, a power of two near 48 KB of K + V per stage) and
-// stages (nstage, about 192 KB in all).
+// Decode geometry for H query heads over Hkv K/V heads: query heads per thread, slots per CTA,
+// (K/V head, query subgroup) pair groups per sequence.
 struct DecGeom {
-    int qpt, nsub, gh, ngroups, ss, nstage, threads;
-    size_t smem;
+    int qpt, nsub, chunk, nzg;
 };
 static DecGeom decode_geom(int H, int Hkv, int D) {
     DecGeom g;
     const int kvg = H / Hkv;
-    const int lph = D / 8;
     g.qpt = decode_qpt(kvg);
     g.nsub = (kvg + g.qpt - 1) / g.qpt;
-    g.gh = std::max(1, std::min(Hkv, decode_max_consumers(g.qpt) / lph / g.nsub));
-    g.ngroups = (Hkv + g.gh - 1) / g.gh;
-    const size_t slot_bytes = size_t(2) * g.gh * D * 2;   // K and V of one slot
-    g.ss = 1;
-    while (g.ss < 32 && size_t(2 * g.ss) * slot_bytes <= 49152) g.ss *= 2;
-    const size_t stage = size_t(g.ss) * slot_bytes;
-    g.nstage = int(std::max<size_t>(2, std::min<size_t>(8, 196608 / stage)));
-    g.threads = 32 + (g.gh * g.nsub * lph + 31) / 32 * 32;
-    g.smem = size_t(g.nstage) * stage + 16 * size_t(g.nstage) + 16 * kDecodeItemRing + 64;
+    g.chunk = g.qpt == 1 ? kDecodeChunk : kDecodeChunkGrp;
+    const int pairs_per_cta = kDecodeThreads / (D / 8);
+    g.nzg = (Hkv * g.nsub + pairs_per_cta - 1) / pairs_per_cta;
     return g;
 }
 
 size_t attn_decode_gqa_workspace_bytes(int B, int cap, int H, int Hkv, int D) {
     if (B < 1 || cap < 1 || H < 1 || (D != 64 && D != 128) || !valid_kv_heads(H, Hkv)) return 0;
     const DecGeom g = decode_geom(H, Hkv, D);
-    const size_t nsm = size_t((cap + kDecodeChunk - 1) / kDecodeChunk);
-    return align256(size_t(B) * g.ngroups * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
+    const size_t nsm = size_t((cap + g.chunk - 1) / g.chunk);
+    return align256(size_t(B) * g.nzg * 4) + align256(size_t(B) * nsm * H * 2 * 4) +
            align256(size_t(B) * nsm * H * D * 4);
 }
 
@@ -605,13 +595,12 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
     if (!valid_common(B, cap, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535) return ATTN_ERR_UNSUPPORTED;
     if (ws_bytes < attn_decode_gqa_workspace_bytes(B, cap, H, Hkv, D)) return ATTN_ERR_WORKSPACE;
     const DecGeom g = decode_geom(H, Hkv, D);
-    const int nsm = (cap + kDecodeChunk - 1) / kDecodeChunk;
+    if (g.nzg > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int nsm = (cap + g.chunk - 1) / g.chunk;
     const int span = W < cap ? W : cap;
-    const int nsplit = (span + kDecodeChunk - 1) / kDecodeChunk;
-    const long long n_items = (long long)nsplit * B * g.ngroups;
-    if (n_items > 0x7fff0000LL) return ATTN_ERR_UNSUPPORTED;
     DecParams p;
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
     p.kc = reinterpret_cast<const __nv_bfloat16*>(k_cache);
@@ -620,25 +609,20 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     p.o = reinterpret_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     char* ws = static_cast<char*>(workspace);
-    const size_t cnt_bytes = align256(size_t(B) * g.ngroups * 4);
-    p.tickets = reinterpret_cast<int*>(ws);
+    const size_t cnt_bytes = align256(size_t(B) * g.nzg * 4);
+    p.counters = reinterpret_cast<int*>(ws);
     p.part_ml = reinterpret_cast<float*>(ws + cnt_bytes);
     p.part_o = reinterpret_cast<float*>(ws + cnt_bytes + align256(size_t(B) * nsm * H * 2 * 4));
     p.B = B;
     p.cap = cap;
     p.H = H;
-    p.Hk = Hkv;
     p.kv_group = H / Hkv;
     p.nsub = g.nsub;
-    p.gh = g.gh;
-    p.ngroups = g.ngroups;
-    p.ss = g.ss;
-    p.nstage = g.nstage;
+    p.chunk = g.chunk;
     p.W = W;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.nsplit = nsplit;
+    p.nsplit = (span + g.chunk - 1) / g.chunk;
     p.nsplit_max = nsm;
-    p.n_items = int(n_items);
     p.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
     p.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
     p.kc_out = const_cast<__nv_bfloat16*>(p.kc);   // written only with the prologue (attn_decode_rope)
@@ -647,41 +631,33 @@ static int decode_impl(const attn_bf16* q, const attn_bf16* k_cache, const attn_
     p.rope_sin = rope.sn;
     p.max_pos = rope.max_pos;
     p.eps = rope.eps;
-    p.wait_limit = kDefaultWaitLimit;
+    const int pairs_per_cta = kDecodeThreads / (D / 8);
+    const int threads = ((std::min(Hkv * g.nsub, pairs_per_cta) * (D / 8)) + 31) / 32 * 32;
+    dim3 grid(p.nsplit, B, g.nzg);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     p.stream_slot = stream_slot(s);
-    const long long grid = std::min<long long>(n_items, sm_count());   // persistent: one CTA per SM
-    // the prefix of the sequences' chunk counts, after the fixed scalars (kDecodePrefixMax sequences)
-    const size_t smem = g.smem + (B <= kDecodePrefixMax ? size_t(B + 1) * 4 : 0);
-    if (smem > 232448) return ATTN_ERR_UNSUPPORTED;   // not reached: stages are sized to fit
-#define SWA_DECODE_LAUNCH(DD, QQ, RR)                                                                  \
-    do {                                                                                               \
-        if (!ensure_smem((const void*)swa_decode_kernel<DD, QQ, RR>, 232448)) return ATTN_ERR_LAUNCH;       \
-        swa_decode_kernel<DD, QQ, RR><<<unsigned(grid), g.threads, smem, s>>>(p);                        \
-    } while (0)
-#define SWA_DECODE_QPT(DD, QQ)                    \
-    do {                                          \
-        if (rope.cs)                              \
-            SWA_DECODE_LAUNCH(DD, QQ, true);      \
-        else                                      \
-            SWA_DECODE_LAUNCH(DD, QQ, false);     \
+#define SWA_DECODE_LAUNCH(DD, QQ)                                      \
+    do {                                                               \
+        if (rope.cs)                                                   \
+            swa_decode_kernel<DD, QQ, true><<<grid, threads, 0, s>>>(p);  \
+        else                                                           \
+            swa_decode_kernel<DD, QQ, false><<<grid, threads, 0, s>>>(p); \
     } while (0)
     if (D == 128) {
         switch (g.qpt) {
-            case 1: SWA_DECODE_QPT(128, 1); break;
-            case 2: SWA_DECODE_QPT(128, 2); break;
-            case 3: SWA_DECODE_QPT(128, 3); break;
-            default: SWA_DECODE_QPT(128, 4); break;
+            case 1: SWA_DECODE_LAUNCH(128, 1); break;
+            case 2: SWA_DECODE_LAUNCH(128, 2); break;
+            case 3: SWA_DECODE_LAUNCH(128, 3); break;
+            default: SWA_DECODE_LAUNCH(128, 4); break;
         }
     } else {
         switch (g.qpt) {
-            case 1: SWA_DECODE_QPT(64, 1); break;
-            case 2: SWA_DECODE_QPT(64, 2); break;
-            case 3: SWA_DECODE_QPT(64, 3); break;
-            default: SWA_DECODE_QPT(64, 4); break;
+            case 1: SWA_DECODE_LAUNCH(64, 1); break;
+            case 2: SWA_DECODE_LAUNCH(64, 2); break;
+            case 3: SWA_DECODE_LAUNCH(64, 3); break;
+            default: SWA_DECODE_LAUNCH(64, 4); break;
         }
     }
-#undef SWA_DECODE_QPT
 #undef SWA_DECODE_LAUNCH
     return launch_status();
 }
@@ -720,6 +696,76 @@ int attn_decode(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v
                 float scale, void* stream) {
     return attn_decode_gqa(q, k_cache, v_cache, cache_len, o, lse, workspace, ws_bytes, B, cap, H, H, D, W, scale,
                            stream);
+}
+
+size_t attn_fwd_fp8_workspace_bytes(int B, int T, int Hkv, int D) {
+    if (B < 1 || T < 1 || Hkv < 1 || D != 128) return 0;
+    const size_t Tp = (size_t(T) + 15) / 16 * 16;
+    return align256(size_t(B) * Hkv * 128 * Tp);
+}
+
+int attn_fwd_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v, const float* q_descale,
+                 const float* k_descale, const float* v_descale, attn_bf16* o, float* lse, void* workspace,
+                 size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, void* stream) {
+    if (!q || !k || !v || !q_descale || !k_descale || !v_descale || !o || !lse || !workspace)
+        return ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, o, lse};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+    const void* dsc[] = {q_descale, k_descale, v_descale};
+    for (const void* ptr : dsc)
+        if ((reinterpret_cast<uintptr_t>(ptr) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!valid_common(B, T, H, D, W, scale) || !valid_kv_heads(H, Hkv)) return ATTN_ERR_INVALID_ARG;
+    if (D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (ws_bytes < attn_fwd_fp8_workspace_bytes(B, T, Hkv, D)) return ATTN_ERR_WORKSPACE;
+    const int n_qblk = (T + 255) / 256;
+    const long long n_items = (long long)n_qblk * B * H;
+    if (n_items > 0x7fffffffLL || B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+    const int Tp = (T + 15) / 16 * 16;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* vt = static_cast<uint8_t*>(workspace);
+    // 1. V^T [B, Hkv, 128, Tp]: the P V product reads V as a K-major operand
+    swa_fp8_transpose_v_kernel<<<dim3(unsigned((T + 63) / 64), unsigned(Hkv), unsigned(B)), 256, 0, s>>>(v, vt, T, Hkv,
+                                                                                                          Tp);
+    if (launch_status() != ATTN_OK) return ATTN_ERR_LAUNCH;
+    // 2. the forward: 8-bit [B, T, H(kv), 128] maps, one 128 x 128-byte box per tile
+    auto enc = encode_fn();
+    if (!enc) return ATTN_ERR_LAUNCH;
+    auto map8 = [&](CUtensorMap* m, const void* base, cuuint64_t d0, cuuint64_t d1, cuuint64_t d2, cuuint64_t d3,
+                    cuuint32_t b0, cuuint32_t b1, cuuint32_t b2) {
+        cuuint64_t dims[4] = {d0, d1, d2, d3};
+        cuuint64_t strides[3] = {d0, d0 * d1, d0 * d1 * d2};
+        cuuint32_t box[4] = {b0, b1, b2, 1};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    CUtensorMap mq, mk, mvt;
+    if (!map8(&mq, q, 128, H, T, B, 128, 1, 128) || !map8(&mk, k, 128, Hkv, T, B, 128, 1, 128) ||
+        !map8(&mvt, vt, Tp, 128, Hkv, B, 128, 128, 1))
+        return ATTN_ERR_LAUNCH;
+    Fp8Params p;
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.dq = q_descale;
+    p.dk = k_descale;
+    p.dv = v_descale;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.G = H / Hkv;
+    p.W = W;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.n_qblk = n_qblk;
+    p.n_items = int(n_items);
+    p.stream_slot = stream_slot(s);
+    p.wait_limit = kDefaultWaitLimit;
+    const long long grid = n_items < sm_count() ? n_items : sm_count();
+    if (!ensure_smem((const void*)swa_fwd_fp8_kernel, Fp8Cfg::SMEM)) return ATTN_ERR_LAUNCH;
+    swa_fwd_fp8_kernel<<<unsigned(grid), Fp8Cfg::THREADS, Fp8Cfg::SMEM, s>>>(mq, mk, mvt, p);
+    return launch_status();
 }
 
 int attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_cache, const attn_bf16* v_cache,

@@ -58,6 +58,10 @@ _lib.attn_decode_gqa.argtypes = [_p] * 7 + [_sz, _i, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode_gqa.restype = _i
 _lib.attn_prefill.argtypes = [_p] * 8 + [_i, _i, _i, _i, _i, _i, _i, _f, _p]
 _lib.attn_prefill.restype = _i
+_lib.attn_fwd_fp8_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.attn_fwd_fp8_workspace_bytes.restype = _sz
+_lib.attn_fwd_fp8.argtypes = [_p] * 9 + [_sz] + [_i] * 6 + [_f, _p]
+_lib.attn_fwd_fp8.restype = _i
 _lib.attn_decode_noalloc.argtypes = [_p] * 6 + [_i, _i, _i, _i, _i, _f, _p]
 _lib.attn_decode_noalloc.restype = _i
 _d = ctypes.c_double
@@ -93,7 +97,7 @@ EXPORTED = ["attn_fwd", "attn_fwd_gqa", "attn_bwd_workspace_bytes", "attn_bwd", 
             "attn_selftest_wait_timeout",
             "attn_status_string", "attn_rope_tables", "attn_rope_qknorm", "attn_rope_qknorm_bwd",
             "attn_prefill_rope_workspace_bytes", "attn_prefill_rope", "attn_decode_rope", "attn_fwd_rope",
-            "attn_bwd_rope"]
+            "attn_bwd_rope", "attn_fwd_fp8_workspace_bytes", "attn_fwd_fp8"]
 
 
 class AttnError(RuntimeError):
@@ -245,6 +249,34 @@ def attn_bwd_set_profile_events(after_pre=None, after_main=None):
 
 def attn_device_status(clear: bool = True) -> int:
     return int(_lib.attn_device_status(1 if clear else 0))
+
+
+def attn_fwd_fp8_workspace_bytes(B: int, T: int, Hkv: int, D: int) -> int:
+    return int(_lib.attn_fwd_fp8_workspace_bytes(B, T, Hkv, D))
+
+
+def attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, workspace, W: int, scale=None, stream=None):
+    """FP8 forward: q [B, T, H, 128], k / v [B, T, Hkv, 128] torch.float8_e4m3fn (or uint8 holding e4m3
+    bytes); descales float32 [B, H] / [B, Hkv] / [B, Hkv] (real value = e4m3 value * descale);
+    o bf16 [B, T, H, 128] and lse float32 [B, H, T] written; workspace of attn_fwd_fp8_workspace_bytes."""
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    for t in (q, k, v):
+        if t.element_size() != 1 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("q, k, v must be contiguous 1-byte (e4m3) CUDA tensors")
+    if tuple(k.shape) != (B, T, Hkv, D) or tuple(v.shape) != (B, T, Hkv, D) or H % Hkv != 0:
+        raise ValueError("k and v must be [B, T, Hkv, D] with Hkv dividing H")
+    for t, shp in ((q_descale, (B, H)), (k_descale, (B, Hkv)), (v_descale, (B, Hkv))):
+        if t.dtype != torch.float32 or tuple(t.shape) != shp or not t.is_contiguous():
+            raise ValueError("descales must be contiguous float32 [B, H] (q) and [B, Hkv] (k, v)")
+    if o.dtype != torch.bfloat16 or tuple(o.shape) != (B, T, H, D):
+        raise ValueError("o must be bf16 [B, T, H, D]")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T):
+        raise ValueError("lse must be float32 [B, H, T]")
+    ws = workspace.numel() * workspace.element_size()
+    _check(_lib.attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), _ptr(o),
+                             _ptr(lse), _ptr(workspace), ws, B, T, H, Hkv, D, int(W), _scale(scale, D),
+                             _stream(stream)), "attn_fwd_fp8")
 
 
 def attn_poll_device_status(stream=None) -> int:

@@ -200,6 +200,26 @@ int attn_decode_rope(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16
                      int max_pos, float eps, attn_bf16* o, float* lse, void* workspace, size_t ws_bytes, int B,
                      int cap, int H, int Hkv, int D, int W, float scale, void* stream);
 
+/* Bytes of workspace attn_fwd_fp8 needs (V transposed to [B, Hkv, 128, T rounded up to 16]
+ * bytes); 0 for sizes it rejects (D other than 128). */
+size_t attn_fwd_fp8_workspace_bytes(int B, int T, int Hkv, int D);
+
+/*
+ * FP8 forward.  The pages name FP8 only for linear layers (apidog guide, section 3, mixed
+ * precision: --fp8 on H100 and Blackwell); the reading for attention: q [B, T, H, 128] and
+ * k, v [B, T, Hkv, 128] hold OCP E4M3 bytes (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits), each with one fp32 descale per (sequence, head): q_descale [B, H], k_descale and
+ * v_descale [B, Hkv], the real operand being the e4m3 value times its descale.  o [B, T, H, 128]
+ * bf16 and lse [B, H, T] fp32 are the windowed attention of attn_fwd_gqa on those real operands,
+ * up to the kernel's rounding of the softmax weights to e4m3 before the P V product (each weight
+ * off by at most 2^-4 of itself; lse uses the unrounded weights).  workspace: at least
+ * attn_fwd_fp8_workspace_bytes(B, T, Hkv, 128) bytes, 256-byte aligned (V is transposed into it);
+ * descale pointers 4-byte aligned.  D other than 128 returns ATTN_ERR_UNSUPPORTED.
+ */
+int attn_fwd_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v, const float* q_descale,
+                 const float* k_descale, const float* v_descale, attn_bf16* o, float* lse, void* workspace,
+                 size_t ws_bytes, int B, int T, int H, int Hkv, int D, int W, float scale, void* stream);
+
 /* Bytes of workspace attn_bwd needs: fp32 rows of lse*log2(e) and Delta, [B*H, T rounded up
  * to 128] each (256-byte padded). */
 size_t attn_bwd_workspace_bytes(int B, int T, int H, int D);

@@ -76,16 +76,13 @@ def test_workspace_sizes():
     assert ops.attn_bwd_workspace_bytes(1, 130, 1, 64) == 2 * 256 * 4   # Tp = 256
     assert ops.attn_bwd_workspace_bytes(1, 1, 1, 128) == 2 * 512   # 128 floats per row, no 256-byte padding needed
     assert ops.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
-    # ticket counters [B, head groups] + partial (m, l) and o for ceil(cap / 64) chunks of 64
-    # window slots; one head group holds every K/V head up to 384 consumer threads (D / 8 per head)
+    # ticket counters [B, head groups of 4 heads (D = 128) / 8 heads (D = 64)] + partial (m, l) and o
+    # for ceil(cap / 128) chunks of 128 cache slots
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert ops.attn_decode_workspace_bytes(32, 2048, 12, 128) == a256(32 * 1 * 4) + a256(32 * 32 * 12 * 2 * 4) + a256(
-        32 * 32 * 12 * 128 * 4)
-    assert ops.attn_decode_workspace_bytes(2, 100, 9, 64) == a256(2 * 1 * 4) + a256(2 * 2 * 9 * 2 * 4) + a256(
-        2 * 2 * 9 * 64 * 4)
-    # 40 heads at D = 128: 24 heads per group (384 threads) -> 2 groups
-    assert ops.attn_decode_workspace_bytes(1, 64, 40, 128) == a256(1 * 2 * 4) + a256(1 * 1 * 40 * 2 * 4) + a256(
-        1 * 1 * 40 * 128 * 4)
+    assert ops.attn_decode_workspace_bytes(32, 2048, 12, 128) == a256(32 * 3 * 4) + a256(32 * 16 * 12 * 2 * 4) + a256(
+        32 * 16 * 12 * 128 * 4)
+    assert ops.attn_decode_workspace_bytes(2, 100, 9, 64) == a256(2 * 2 * 4) + a256(2 * 1 * 9 * 2 * 4) + a256(
+        2 * 1 * 9 * 64 * 4)
     assert ops.attn_decode_workspace_bytes(1, 0, 1, 64) == 0
     for bad_d in (0, 4, 7, 96):
         assert ops.attn_decode_workspace_bytes(1, 16, 1, bad_d) == 0
@@ -93,23 +90,18 @@ def test_workspace_sizes():
 
 def test_grouped_decode_workspace_size():
     """With grouped K/V heads a thread serves up to 4 query heads of one K/V head (a divisor of the
-    group where there is one); a head group holds up to 256 consumer threads (D / 8 per (K/V head,
-    query subgroup) pair); counters per (sequence, head group), partials per query head and chunk
-    of 64 window slots."""
+    group where there is one) over runs of 64 cache slots; counters per group of 4 (D = 128) or 8
+    (D = 64) (K/V head, query subgroup) pairs, partials per query head and 64-slot run."""
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    # 12 query heads over 4 K/V heads: 3 per thread, 4 pairs -> 1 group, 32 chunks
+    # 12 query heads over 4 K/V heads: 3 per thread, 4 pairs -> 1 counter per sequence, 32 runs
     assert ops.attn_decode_gqa_workspace_bytes(32, 2048, 12, 4, 128) == a256(32 * 1 * 4) + a256(
         32 * 32 * 12 * 2 * 4) + a256(32 * 32 * 12 * 128 * 4)
-    # MQA, 8 query heads: 4 per thread, 2 subgroups -> 1 group
+    # MQA, 8 query heads: 4 per thread, 2 subgroups, 8 pairs per CTA at D = 64
     assert ops.attn_decode_gqa_workspace_bytes(2, 100, 8, 1, 64) == a256(2 * 1 * 4) + a256(2 * 2 * 8 * 2 * 4) + a256(
         2 * 2 * 8 * 64 * 4)
-    # 40 query heads over 8 K/V heads: groups of 5 -> 4 + 1 (ragged), 2 subgroups, 16 pairs -> 1 group
-    assert ops.attn_decode_gqa_workspace_bytes(1, 64, 40, 8, 128) == a256(1 * 1 * 4) + a256(1 * 1 * 40 * 2 * 4) + a256(
+    # 40 query heads over 8 K/V heads: groups of 5 -> 4 + 1 (ragged), 16 pairs -> 4 counters
+    assert ops.attn_decode_gqa_workspace_bytes(1, 64, 40, 8, 128) == a256(1 * 4 * 4) + a256(1 * 1 * 40 * 2 * 4) + a256(
         1 * 1 * 40 * 128 * 4)
-    # 64 query heads over 16 K/V heads at D = 128: 4 per thread, 16 pairs of 16 threads -> 1 group;
-    # over 32 K/V heads (2 per thread): 32 pairs -> 2 groups
-    assert ops.attn_decode_gqa_workspace_bytes(1, 64, 64, 32, 128) == a256(1 * 2 * 4) + a256(1 * 1 * 64 * 2 * 4) + a256(
-        1 * 1 * 64 * 128 * 4)
     for B, cap, H, D in ((32, 2048, 12, 128), (2, 100, 9, 64), (3, 1, 1, 128)):
         assert ops.attn_decode_gqa_workspace_bytes(B, cap, H, H, D) == ops.attn_decode_workspace_bytes(B, cap, H, D)
     assert ops.attn_decode_gqa_workspace_bytes(2, 64, 6, 4, 128) == 0      # 4 does not divide 6
@@ -247,3 +239,16 @@ def test_header_is_plain_c(tmp_path):
     src.write_text('#include "swa_attn.h"\n' + "".join(f"void* p_{n} = (void*)&{n};\n" for n in names))
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-c", "-I", os.path.dirname(HEADER),
                            str(src), "-o", str(tmp_path / "use_header.o")])
+
+
+def test_fp8_forward_argument_checks():
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert ops.attn_fwd_fp8_workspace_bytes(2, 100, 3, 128) == a256(2 * 3 * 128 * 112)   # T rounded up to 16
+    assert ops.attn_fwd_fp8_workspace_bytes(2, 100, 3, 64) == 0
+    f = ops._lib.attn_fwd_fp8
+    ws = ops.attn_fwd_fp8_workspace_bytes(1, 16, 1, 128)
+    assert f(None, A, A, A, A, A, A, A, A, ws, 1, 16, 1, 1, 128, 8, 0.1, None) == ERR_INVALID
+    assert f(A, A, A, A, A, A, A, A, A, ws, 1, 16, 1, 1, 64, 8, 0.1, None) == ERR_UNSUPPORTED
+    assert f(A, A, A, A, A, A, A, A, A, ws - 16, 1, 16, 1, 1, 128, 8, 0.1, None) == ERR_WORKSPACE
+    assert f(A, A, A, A + 2, A, A, A, A, A, ws, 1, 16, 1, 1, 128, 8, 0.1, None) == ERR_INVALID   # descale misaligned
+    assert f(A, A, A, A, A, A, A, A, A, ws, 1, 16, 4, 3, 128, 8, 0.1, None) == ERR_INVALID        # 3 does not divide 4
