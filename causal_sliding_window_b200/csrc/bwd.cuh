@@ -22,12 +22,11 @@
 //
 // Both main kernels are persistent (one CTA per SM) and draw head-major items from a
 // launch-wide counter (sm100.cuh), so CTAs that run at the same time share a head's
-// tiles through L2.  Roles:
-//   dK/dV (576 threads): warps 0..15 four warpgroups on the same 128 TMEM lanes (one key row per
-//                lane), warpgroup g taking query columns 32g .. 32g+31 of each step's score tile;
-//                warp 16 TMA producer; warp 17 MMA issuer (one thread)
-//   dQ (320 threads): warps 0..7 two warpgroups on the same 128 TMEM lanes, warps 0..3 taking key
-//                columns 0..63, warps 4..7 columns 64..127; warp 8 TMA producer; warp 9 MMA issuer
+// tiles through L2.  Roles (320 threads):
+//   warp 8       TMA producer
+//   warp 9       MMA issuer (one thread)
+//   warps 0..7   two warpgroups on the same 128 TMEM lanes (one row per lane): warps 0..3
+//                take columns 0..63 of the 128-column score tiles, warps 4..7 columns 64..127.
 #pragma once
 
 #include "rope.cuh"
@@ -154,11 +153,7 @@ struct BwdKVCfg {
     // Up to 1 KB of slack to align the tile region to 1024 bytes, within the per-block limit;
     // the kernel checks at run time that the aligned layout fits what it was given.
     static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
-    // Roles: warps 0..15 key-row warps (four warpgroups on the same 128 TMEM lanes, each taking
-    // 32 of a step's 128 query columns), warp 16 TMA producer, warp 17 MMA issuer.
-    static constexpr int NROW = 16;
-    static constexpr int THREADS = 32 * (NROW + 2);
-    static constexpr int PRODUCER = NROW, MMA = NROW + 1;
+    static constexpr int THREADS = 320;
     static constexpr uint32_t TMEM_COLS = 512;     // S^T | dP^T (then packed P^T, dS^T) | dV | dK
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BM, 0, 0);       // K-major A, K-major B
     static constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);      // K-major A, MN-major B
@@ -261,23 +256,23 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(do_empty(s), 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_free, 32 * C::NROW);
+        mbar_init(s_free, 256);
         mbar_init(dp_full, 1);
-        mbar_init(p_full, 32 * C::NROW);
-        mbar_init(ds_full, 32 * C::NROW);
+        mbar_init(p_full, 256);
+        mbar_init(ds_full, 256);
         mbar_init(mma_done, 1);
         mbar_init(acc_full, 1);
-        mbar_init(acc_free, 32 * C::NROW);
+        mbar_init(acc_free, 256);
         for (int e = 0; e < kItemRing; ++e) {
             mbar_init(item_full0 + 8u * e, 1);
-            mbar_init(item_empty0 + 8u * e, 1 + C::NROW);   // the MMA thread and the key-row warps
+            mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and warps 0..7
         }
         abort_flag[0] = 0;
         abort_flag[1] = p.stream_slot;   // read by a wait that gives up
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == C::MMA) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -287,7 +282,7 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tDP = tmem + 128u, tDV = tmem + 256u, tDK = tmem + 256u + uint32_t(D);
 
-    if (warp == C::PRODUCER) {
+    if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
         // Per item: K, Q_first, V, dO_first, then Q and dO per step, so that S of the item's
         // first step waits for K and one Q tile only.
@@ -360,7 +355,7 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (nk > 0) mbar_drain(k_full, uint32_t((nk - 1) & 1), p.wait_limit, p.stream_slot);
             if (nv > 0) mbar_drain(v_full, uint32_t((nv - 1) & 1), p.wait_limit, p.stream_slot);
         }
-    } else if (warp == C::MMA) {
+    } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             bool ok = true;
@@ -411,16 +406,16 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc_fence_after();
                     const SDesc od = sdesc_sw128_w(sDO(n), C::BOX, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < C::BM / 16; ++kk)   // queries 16kk.. : packed P^T of warpgroup kk/2
-                        mma_ts_w(tDV, tDP + (kk >> 1) * 32 + (kk & 1) * 8, od.lo + kk * (2048 >> 4), od.hi, C::IDESC_ACC,
+                    for (int kk = 0; kk < C::BM / 16; ++kk)   // query rows 16kk.. : P^T column pairs of warpgroup kk/4
+                        mma_ts_w(tDV, tDP + (kk >> 2) * 64 + (kk & 3) * 8, od.lo + kk * (2048 >> 4), od.hi, C::IDESC_ACC,
                                  (l > 0 || kk > 0) ? 1u : 0u);
                     // dK += dS^T Q
                     if (!(ok = wait(ds_full, n))) break;
                     tc_fence_after();
                     const SDesc qd = sdesc_sw128_w(sQ(n), C::BOX, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < C::BM / 16; ++kk)   // packed dS^T of warpgroup kk/2
-                        mma_ts_w(tDK, tDP + (kk >> 1) * 32 + 16 + (kk & 1) * 8, qd.lo + kk * (2048 >> 4), qd.hi,
+                    for (int kk = 0; kk < C::BM / 16; ++kk)
+                        mma_ts_w(tDK, tDP + (kk >> 2) * 64 + 32 + (kk & 3) * 8, qd.lo + kk * (2048 >> 4), qd.hi,
                                  C::IDESC_ACC, (l > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(q_empty(n));    // Q_n is read
                     tc_commit(do_empty(n));   // dO_n, lse and Delta of step n are read
@@ -434,14 +429,14 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else {
         // ------------------------------ key-row warps: P^T, dS^T, epilogue ------------------------------
-        // Thread = key row (TMEM lane); warpgroup qd = warp / 4 takes query columns 32qd .. 32qd+31.
-        const int qd = warp >> 2;
+        // Thread = key row (TMEM lane); warps 0..3 take query columns 0..63, warps 4..7 columns 64..127.
+        const int rh = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const float sl2 = p.scale_log2;
-        // Epilogue of the pki-th item (index pitem): warpgroups 0, 1 write the two halves of this row's
-        // dV, warpgroups 2, 3 those of scale * dK.  It runs at the start of the next item's first step,
-        // while that step's S^T and dP^T MMAs (issued earlier) execute.
+        // Epilogue of the pki-th item (index pitem): warps 0..3 write this row's dV,
+        // warps 4..7 scale * dK.  It runs at the start of the next item's first step, while
+        // that step's S^T and dP^T MMAs (issued earlier) execute.
         auto epilogue = [&](int pki, int pitem) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(acc_full, uint32_t(pki & 1), abort_flag, p.wait_limit,
                                                    kStatusTimeoutEpilogue)))
@@ -449,23 +444,27 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_after();
             const BwdKVItem pg = bwd_kv_item(p, pitem);
             const long long pkv = pg.k0 + row;
-            const bool isk = qd >= 2;
-            const int cb = (qd & 1) * (D / 2);   // this thread's half of the row
             __nv_bfloat16* dst =
-                pkv < T ? (isk ? p.dk : p.dv) + ((size_t(pg.b) * T + size_t(pkv)) * (p.H / p.G) + pg.h) * D + cb
+                pkv < T ? (rh == 0 ? p.dv : p.dk) + ((size_t(pg.b) * T + size_t(pkv)) * (p.H / p.G) + pg.h) * D
                         : nullptr;
-            const uint32_t src = (isk ? tDK : tDV) + lane_off + cb;
-            const float mul = isk ? p.scale : 1.f;
+            const uint32_t src = (rh == 0 ? tDV : tDK) + lane_off;
+            const float mul = rh == 0 ? 1.f : p.scale;
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {   // 32 columns at a time (register budget of 18 warps)
-                uint32_t a[32];
-                tmem_ld32(src + c * 32, a);
-                tmem_ld_wait(a);
-                if (c + 1 == D / 64) {
+#pragma unroll
+            for (int c = 0; c < D / 32; c += 2) {   // 64 columns per wait
+                uint32_t a0[32], a1[32];
+                tmem_ld32(src + c * 32, a0);
+                tmem_ld32(src + c * 32 + 32, a1);
+                tmem_ld_wait(a0);
+                tmem_ld_wait(a1);
+                if (c + 2 == D / 32) {
                     tc_fence_before();
                     mbar_arrive(acc_free);
                 }
-                if (dst) store_row32_bf16(dst + c * 32, a, mul);
+                if (dst) {
+                    store_row32_bf16(dst + c * 32, a0, mul);
+                    store_row32_bf16(dst + c * 32 + 32, a1, mul);
+                }
             }
             return true;
         };
@@ -484,7 +483,7 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 int qh, qt;
                 bwd_kv_step(p, g, l, qh, qt);
                 const long long q0 = (long long)qt * C::BM;
-                const uint32_t sL = sLSE(n) + qd * 128;   // this warpgroup's 32 lse2 values (Delta 512 B on)
+                const uint32_t sL = sLSE(n) + rh * 256;   // this half's 64 lse2 values
                 // The previous item's dV / dK leave TMEM before this item's first dV.
                 if (l == 0 && prev_ki >= 0) {
                     if (!(ok = epilogue(prev_ki, prev_item))) break;
@@ -497,81 +496,87 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                               kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                float pr[32];
+                float pr[64];
                 {
-                    uint32_t r0[32];
-                    tmem_ld32(tS + lane_off + qd * 32, r0);
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tS + lane_off + rh * 64, r0);
+                    tmem_ld32(tS + lane_off + rh * 64 + 32, r1);
                     tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
                     tc_fence_before();
                     mbar_arrive(s_free);   // S^T(n+1) may be written
 #pragma unroll
                     for (int gq = 0; gq < 8; ++gq) {
                         const float4 a = lds_f32x4(sL + gq * 16);
+                        const float4 b = lds_f32x4(sL + 128 + gq * 16);
                         pr[4 * gq + 0] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 0]), sl2, -a.x));
                         pr[4 * gq + 1] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 1]), sl2, -a.y));
                         pr[4 * gq + 2] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 2]), sl2, -a.z));
                         pr[4 * gq + 3] = ex2_approx(fmaf(__uint_as_float(r0[4 * gq + 3]), sl2, -a.w));
+                        pr[32 + 4 * gq + 0] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 0]), sl2, -b.x));
+                        pr[32 + 4 * gq + 1] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 1]), sl2, -b.y));
+                        pr[32 + 4 * gq + 2] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 2]), sl2, -b.z));
+                        pr[32 + 4 * gq + 3] = ex2_approx(fmaf(__uint_as_float(r1[4 * gq + 3]), sl2, -b.w));
                     }
                 }
                 // Tiles that cut the diagonal, the window's far edge or T: keep query columns clo..chi
                 // of this key row (queries kv .. kv+W-1, below T).  The test is uniform across the CTA.
                 const bool full = (k0 + C::BN - 1 <= q0) && (q0 + C::BM - 1 - k0 < W) && (q0 + C::BM <= T);
                 if (!full) {
-                    const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1)) - qd * 32;
+                    const int clo = int(imin_ll(imax_ll(kv - q0, 0), C::BM + 1)) - rh * 64;
                     const int chi =
                         (kv < T ? int(imin_ll(imax_ll(imin_ll(kv + W - 1, (long long)T - 1) - q0, -1), C::BM)) : -1) -
-                        qd * 32;
+                        rh * 64;
 #pragma unroll
-                    for (int col = 0; col < 32; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
+                    for (int col = 0; col < 64; ++col) pr[col] = (col >= clo && col <= chi) ? pr[col] : 0.f;
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                // This warpgroup's 32 dP^T columns: the first 16 take packed P^T, the last 16 packed
-                // dS^T, once the dP^T values are in registers.
-                const uint32_t tOwn = tDP + lane_off + qd * 32;
+                // This warpgroup's dP^T columns: the first 32 take packed P^T, the last 32 packed dS^T,
+                // each once its dP^T values are in registers.
+                const uint32_t tOwn = tDP + lane_off + rh * 64;
+                uint32_t w0[16];
                 {
-                    // dS^T = P^T (dP^T - Delta), in two halves of 16 columns (register budget of
-                    // 18 warps): columns 0..15 first, so their dP^T columns may take packed P^T.
-                    uint32_t w[16];
-                    {
-                        uint32_t r[16];
-                        tmem_ld16(tOwn, r);
-                        tmem_ld_wait(r);
+                    uint32_t r[32];
+                    tmem_ld32(tOwn, r);
+                    tmem_ld_wait(r);
 #pragma unroll
-                        for (int gq = 0; gq < 4; ++gq) {
-                            const float4 a = lds_f32x4(sL + 512 + gq * 16);
-                            const int c = 4 * gq;
-                            w[2 * gq] = pack_bf16x2(pr[c] * (__uint_as_float(r[c]) - a.x),
-                                                    pr[c + 1] * (__uint_as_float(r[c + 1]) - a.y));
-                            w[2 * gq + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(r[c + 2]) - a.z),
-                                                        pr[c + 3] * (__uint_as_float(r[c + 3]) - a.w));
-                        }
-                    }
-                    {
+                    for (int hh = 0; hh < 2; ++hh) {
                         uint32_t pk[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pr[2 * i], pr[2 * i + 1]);
-                        tmem_st16(tOwn, pk);
+                        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pr[hh * 32 + 2 * i], pr[hh * 32 + 2 * i + 1]);
+                        tmem_st16(tOwn + hh * 16, pk);
                     }
                     tmem_st_wait();
                     tc_fence_before();
                     mbar_arrive(p_full);
-                    {
-                        uint32_t r[16];
-                        tmem_ld16(tOwn + 16, r);
-                        tmem_ld_wait(r);
+                    // dS^T = P^T (dP^T - Delta), query columns 0..31 of this half
 #pragma unroll
-                        for (int gq = 0; gq < 4; ++gq) {
-                            const float4 a = lds_f32x4(sL + 512 + 64 + gq * 16);
-                            const int c = 4 * gq;
-                            w[8 + 2 * gq] = pack_bf16x2(pr[16 + c] * (__uint_as_float(r[c]) - a.x),
-                                                        pr[17 + c] * (__uint_as_float(r[c + 1]) - a.y));
-                            w[9 + 2 * gq] = pack_bf16x2(pr[18 + c] * (__uint_as_float(r[c + 2]) - a.z),
-                                                        pr[19 + c] * (__uint_as_float(r[c + 3]) - a.w));
-                        }
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 a = lds_f32x4(sL + 512 + gq * 16);
+                        const int c = 4 * gq;
+                        w0[2 * gq] = pack_bf16x2(pr[c] * (__uint_as_float(r[c]) - a.x),
+                                                 pr[c + 1] * (__uint_as_float(r[c + 1]) - a.y));
+                        w0[2 * gq + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(r[c + 2]) - a.z),
+                                                     pr[c + 3] * (__uint_as_float(r[c + 3]) - a.w));
                     }
-                    tmem_st16(tOwn + 16, w);
+                }
+                {
+                    uint32_t r[32], w1[16];   // query columns 32..63 of this half
+                    tmem_ld32(tOwn + 32, r);
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int gq = 0; gq < 8; ++gq) {
+                        const float4 a = lds_f32x4(sL + 512 + 128 + gq * 16);
+                        const int c = 4 * gq;
+                        w1[2 * gq] = pack_bf16x2(pr[32 + c] * (__uint_as_float(r[c]) - a.x),
+                                                 pr[33 + c] * (__uint_as_float(r[c + 1]) - a.y));
+                        w1[2 * gq + 1] = pack_bf16x2(pr[34 + c] * (__uint_as_float(r[c + 2]) - a.z),
+                                                     pr[35 + c] * (__uint_as_float(r[c + 3]) - a.w));
+                    }
+                    tmem_st16(tOwn + 32, w0);
+                    tmem_st16(tOwn + 48, w1);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -587,7 +592,7 @@ swa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == C::MMA) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ===========================================================================
@@ -616,11 +621,7 @@ struct BwdQCfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
-    // Roles: warps 0..15 query-row warps (four warpgroups on the same 128 TMEM lanes, each taking
-    // 32 of a step's 128 key columns), warp 16 TMA producer, warp 17 MMA issuer.
-    static constexpr int NROW = 16;
-    static constexpr int THREADS = 32 * (NROW + 2);
-    static constexpr int PRODUCER = NROW, MMA = NROW + 1;
+    static constexpr int THREADS = 320;
     static constexpr uint32_t TMEM_COLS = 512;      // S buffer 0 | S buffer 1 | dP | dQ
     static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);    // K-major A, K-major B
     static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, 0, 1);    // A from TMEM, MN-major B
@@ -709,24 +710,24 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(do_empty, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full(b), 1);
-            mbar_init(s_read(b), 32 * C::NROW);
+            mbar_init(s_read(b), 128);
         }
         mbar_init(dp_full, 1);
-        mbar_init(dp_free, 32 * C::NROW);
-        mbar_init(ds_full, 32 * C::NROW);
+        mbar_init(dp_free, 256);
+        mbar_init(ds_full, 256);
         mbar_init(dq_full, 1);
-        mbar_init(dq_free, 32 * C::NROW);
+        mbar_init(dq_free, 256);
         mbar_init(mma_done, 1);
         for (int e = 0; e < kItemRing; ++e) {
             mbar_init(item_full0 + 8u * e, 1);
-            mbar_init(item_empty0 + 8u * e, 1 + C::NROW);   // the MMA thread and the query-row warps
+            mbar_init(item_empty0 + 8u * e, 1 + 8);   // the MMA thread and warps 0..7
         }
         abort_flag[0] = 0;
         abort_flag[1] = p.stream_slot;   // read by a wait that gives up
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == C::MMA) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -737,7 +738,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto tSb = [&](int buf) { return tmem + uint32_t(buf) * 128u; };
     const uint32_t tDP = tmem + 256u, tDQ = tmem + 384u;
 
-    if (warp == C::PRODUCER) {
+    if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
         // Order per item: Q, K_jlo, dO, V_jlo, then K_j, V_j per step (Q and dO have their own buffers).
         if (lane == 0) {
@@ -792,7 +793,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (nq > 0) mbar_drain(q_full, uint32_t((nq - 1) & 1), p.wait_limit, p.stream_slot);
             if (ndo > 0) mbar_drain(do_full, uint32_t((ndo - 1) & 1), p.wait_limit, p.stream_slot);
         }
-    } else if (warp == C::MMA) {
+    } else if (warp == 9) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             bool ok = true;
@@ -857,55 +858,40 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
     } else {
         // ------------------------------ query-row warps: dS, epilogue ------------------------------
-        // Thread = query row (TMEM lane); warpgroup qd = warp / 4 takes key columns 32qd .. 32qd+31.
-        const int qd = warp >> 2;
+        // Thread = query row (TMEM lane); warps 0..3 take key columns 0..63, warps 4..7 columns 64..127.
+        const int rh = warp >> 2;
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const float sl2 = p.scale_log2;
-        // Epilogue of item pqi (this row's quarter of dQ at dst, null past T): dQ = scale * acc.  It
+        // Epilogue of item pqi (this row's half of dQ at dst, null past T): dQ = scale * acc.  It
         // runs after P of the next item's first step, so that P overlaps the last dQ MMA.
         auto epilogue = [&](int pqi, __nv_bfloat16* dst) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(dq_full, uint32_t(pqi & 1), abort_flag, p.wait_limit,
                                                    kStatusTimeoutEpilogue)))
                 return false;
             tc_fence_after();
-            if constexpr (D == 128) {
-                uint32_t acc[32];
-                tmem_ld32(tDQ + lane_off + qd * 32, acc);
-                tmem_ld_wait(acc);
-                tc_fence_before();
-                mbar_arrive(dq_free);
-                if (dst) store_row32_bf16(dst, acc, p.scale);
-            } else {
-                uint32_t acc[16];
-                tmem_ld16(tDQ + lane_off + qd * 16, acc);
-                tmem_ld_wait(acc);
-                tc_fence_before();
-                mbar_arrive(dq_free);
-                if (dst) {
+            uint32_t acc[D / 64][32];
 #pragma unroll
-                    for (int v4 = 0; v4 < 2; ++v4) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(acc[v4 * 8 + 0]) * p.scale, __uint_as_float(acc[v4 * 8 + 1]) * p.scale);
-                        w.y = pack_bf16x2(__uint_as_float(acc[v4 * 8 + 2]) * p.scale, __uint_as_float(acc[v4 * 8 + 3]) * p.scale);
-                        w.z = pack_bf16x2(__uint_as_float(acc[v4 * 8 + 4]) * p.scale, __uint_as_float(acc[v4 * 8 + 5]) * p.scale);
-                        w.w = pack_bf16x2(__uint_as_float(acc[v4 * 8 + 6]) * p.scale, __uint_as_float(acc[v4 * 8 + 7]) * p.scale);
-                        *reinterpret_cast<uint4*>(dst + v4 * 8) = w;
-                    }
-                }
+            for (int c = 0; c < D / 64; ++c) tmem_ld32(tDQ + lane_off + rh * (D / 2) + c * 32, acc[c]);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) tmem_ld_wait(acc[c]);
+            tc_fence_before();
+            mbar_arrive(dq_free);
+            if (dst) {
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) store_row32_bf16(dst + c * 32, acc[c], p.scale);
             }
             return true;
         };
-        // kRope epilogue of item pqi, query row pq of head (pb, ph): warpgroups 1..3 only release the
-        // accumulator; warpgroup 0 reads whole rows (pairs (i, i + D/2) together) in two passes, the
-        // first for the row's two sums, the second for the output, 16 columns (and their partners)
-        // at a time.
+        // kRope epilogue of item pqi, query row pq of head (pb, ph): warps 4..7 only release the
+        // accumulator; warps 0..3 read whole rows (pairs (i, i + D/2) together) in two passes, the
+        // first for the row's two sums, the second for the output.
         auto epilogue_rope = [&](int pqi, long long pq, int pb, int ph) -> bool {
             if (!__all_sync(0xffffffffu, mbar_wait(dq_full, uint32_t(pqi & 1), abort_flag, p.wait_limit,
                                                    kStatusTimeoutEpilogue)))
                 return false;
             tc_fence_after();
-            if (qd == 0) {
+            if (rh == 0) {
                 const uint32_t src = tDQ + lane_off;
                 const bool in = pq < T, posok = pq < p.max_pos;
                 const size_t roff = ((size_t(pb) * T + size_t(in ? pq : 0)) * p.H + ph) * D;
@@ -918,29 +904,23 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll 1
                 for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll 1
-                    for (int c = 0; c < D / 2; c += 16) {
-                        uint32_t a1[16], a2[16];   // dQ columns c.. and their partners c + D/2..
+                    for (int c = 0; c < D / 2; c += 32) {
+                        uint32_t a1[32], a2[32];   // dQ columns c.. and their partners c + D/2..
                         __syncwarp();              // the TMEM loads are warp-collective
-                        tmem_ld16(src + c, a1);
-                        tmem_ld16(src + D / 2 + c, a2);
+                        tmem_ld32(src + c, a1);
+                        tmem_ld32(src + D / 2 + c, a2);
                         tmem_ld_wait(a1);
                         tmem_ld_wait(a2);
                         if (!in) continue;
-#pragma unroll
-                        for (int v = 0; v < 16; v += 8) {
-                            if (!posok) {   // no table row: the gradient at the rotated query, as is
-                                if (pass == 1) {
-                                    float o1[8], o2[8];
-#pragma unroll
-                                    for (int i = 0; i < 8; ++i) {
-                                        o1[i] = __uint_as_float(a1[v + i]) * p.scale;
-                                        o2[i] = __uint_as_float(a2[v + i]) * p.scale;
-                                    }
-                                    *reinterpret_cast<uint4*>(dst + c + v) = bf16x8_pack(o1);
-                                    *reinterpret_cast<uint4*>(dst + D / 2 + c + v) = bf16x8_pack(o2);
-                                }
-                                continue;
+                        if (!posok) {   // no table row: the gradient at the rotated query, as is
+                            if (pass == 1) {
+                                store_row32_bf16(dst + c, a1, p.scale);
+                                store_row32_bf16(dst + D / 2 + c, a2, p.scale);
                             }
+                            continue;
+                        }
+#pragma unroll
+                        for (int v = 0; v < 32; v += 8) {
                             float x1[8], x2[8];
                             bf16x8_unpack(*reinterpret_cast<const uint4*>(xr + c + v), x1);
                             bf16x8_unpack(*reinterpret_cast<const uint4*>(xr + D / 2 + c + v), x2);
@@ -1009,27 +989,34 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 mbar_wait(s_full(buf), ph, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                float pr[32];
+                float pr[64];
                 {
-                    uint32_t r0[32];
-                    tmem_ld32(tSb(buf) + lane_off + qd * 32, r0);
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tSb(buf) + lane_off + rh * 64, r0);
+                    tmem_ld32(tSb(buf) + lane_off + rh * 64 + 32, r1);
                     tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pr[i] = ex2_approx(fmaf(__uint_as_float(r0[i]), sl2, -lse2_q));
+                    for (int i = 0; i < 32; ++i) {
+                        pr[i] = ex2_approx(fmaf(__uint_as_float(r0[i]), sl2, -lse2_q));
+                        pr[32 + i] = ex2_approx(fmaf(__uint_as_float(r1[i]), sl2, -lse2_q));
+                    }
                 }
-                // Packed dS of key columns 32qd.. goes to TMEM columns 16qd.. of the buffer, which hold
-                // S of key columns that warpgroup qd / 2 reads: every warpgroup says when it has read its S.
-                tc_fence_before();
-                mbar_arrive(s_read(buf));
+                // Packed dS of key columns 64..127 goes to TMEM columns 32..63 of the buffer, which hold
+                // S of key columns 32..63 that warps 0..3 read: those warps say when they have.
+                if (rh == 0) {
+                    tc_fence_before();
+                    mbar_arrive(s_read(buf));
+                }
                 // Tiles that cut the diagonal or the window's far edge: keep key columns clo..chi of this
                 // query row (keys q-W+1 .. q).  The test is uniform across the CTA.
                 const long long k0 = (long long)j * C::BN;
                 const bool full = (k0 + C::BN - 1 <= g.q0) && (k0 > g.q0 + C::BM - 1 - W);
                 if (!full) {
-                    const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN)) - qd * 32;
-                    const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1)) - qd * 32;
+                    const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN)) - rh * 64;
+                    const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1)) - rh * 64;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) pr[c] = (c >= clo && c <= chi) ? pr[c] : 0.f;
+                    for (int c = 0; c < 64; ++c) pr[c] = (c >= clo && c <= chi) ? pr[c] : 0.f;
                 }
                 if (!kRope && j == g.jlo && prev_qi >= 0) {
                     if (!(ok = epilogue(prev_qi, prev_dst))) break;
@@ -1039,32 +1026,37 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 mbar_wait(dp_full, uint32_t(n & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t pk[16];
+                uint32_t pk[32];
                 {
-                    uint32_t r0[32];
-                    tmem_ld32(tDP + lane_off + qd * 32, r0);
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tDP + lane_off + rh * 64, r0);
+                    tmem_ld32(tDP + lane_off + rh * 64 + 32, r1);
                     tmem_ld_wait(r0);
+                    tmem_ld_wait(r1);
                     tc_fence_before();
                     mbar_arrive(dp_free);   // dP(n+1) may be written
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
+                    for (int i = 0; i < 16; ++i) {
                         pk[i] = pack_bf16x2(pr[2 * i] * (__uint_as_float(r0[2 * i]) - delta_q),
                                             pr[2 * i + 1] * (__uint_as_float(r0[2 * i + 1]) - delta_q));
+                        pk[16 + i] = pack_bf16x2(pr[32 + 2 * i] * (__uint_as_float(r1[2 * i]) - delta_q),
+                                                 pr[33 + 2 * i] * (__uint_as_float(r1[2 * i + 1]) - delta_q));
+                    }
                 }
-                if (qd > 0) {   // the columns written here hold S that another warpgroup reads
+                if (rh == 1) {
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait(s_read(buf), ph, abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
                     if (!ok) break;
                     tc_fence_after();
                 }
-                tmem_st16(tSb(buf) + lane_off + qd * 16, pk);
+                tmem_st32(tSb(buf) + lane_off + rh * 32, pk);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(ds_full);
             }
             if (!ok) break;
             prev_qi = qi;
-            prev_dst = q < T ? p.dq + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D + qd * (D / 4) : nullptr;
+            prev_dst = q < T ? p.dq + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D + rh * (D / 2) : nullptr;
             prev_q = q;
             prev_b = g.b;
             prev_h = g.h;
@@ -1080,7 +1072,7 @@ swa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == C::MMA) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace swa
