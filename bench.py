@@ -266,6 +266,15 @@ def run_case(args):
         cl = torch.from_numpy(x["cache_len"]).to(dev)
         ws = ops.decode_workspace(dc["B"], dc["cap"], dc["H"], dc["D"], dev)
         call = lambda: ops.decode(q, kc, vc, cl, W, workspace=ws)  # noqa: E731
+    elif args.case == "fp8":
+        x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"], with_do=False)
+        # e4m3 inputs by torch's conversion of the bf16 values (unit descales: |x| stays far below 448)
+        q8, k8, v8 = (to_bf16(x[n], dev).float().to(torch.float8_e4m3fn) for n in ("q", "k", "v"))
+        ds = torch.ones((B, H), dtype=torch.float32, device=dev)
+        o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+        ws = torch.empty(ops.attn_fwd_fp8_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+        call = lambda: ops.attn_fwd_fp8(q8, k8, v8, ds, ds, ds, o, lse, ws, W)  # noqa: E731
     else:
         x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"])
         q, k, v, do = (to_bf16(x[n], dev) for n in ("q", "k", "v", "do"))
@@ -330,8 +339,11 @@ def run_configs(args):
 
     def tensor_row(row, W, kind, flops, ms):
         tf = flops / ms / 1e9
+        # FP8 rows against the FP8 peaks: twice the bf16 ones (the nominal dense ratio, 4.5 / 2.25 PF)
+        mult = 2.0 if kind == "fwd-fp8" else 1.0
         emit(row=row, W=W, kind=kind, ms=round(ms, 4), tflops=round(tf, 1),
-             frac_spec=round(tf / SPEC_BF16_TFLOPS, 4), frac_burst=round(tf / pt, 4), frac_sustained=round(tf / pts, 4))
+             frac_spec=round(tf / (mult * SPEC_BF16_TFLOPS), 4), frac_burst=round(tf / (mult * pt), 4),
+             frac_sustained=round(tf / (mult * pts), 4))
 
     def attention_rows(name, Hkv=None, label=None):
         cfg = inputs.WORKLOADS[name]
@@ -366,6 +378,22 @@ def run_configs(args):
     for name in ("d12", "d24", "d26"):
         attention_rows(name)
     attention_rows("d24", Hkv=4, label="d24 shape with 4 K/V heads (grouped)")
+
+    # FP8 forward on the depth-24 shape: e4m3 by torch's conversion of the seeded bf16 values
+    cfg = inputs.WORKLOADS["d24"]
+    B, T, H, D = cfg["B"], cfg["T"], cfg["H"], cfg["D"]
+    x = inputs.attention_inputs(B, T, H, D, seed=cfg["seed"], with_do=False)
+    q8, k8, v8 = (to_bf16(x[n], dev).float().to(torch.float8_e4m3fn) for n in ("q", "k", "v"))
+    del x
+    ds = torch.ones((B, H), dtype=torch.float32, device=dev)
+    o = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    ws8 = torch.empty(ops.attn_fwd_fp8_workspace_bytes(B, T, H, D), dtype=torch.uint8, device=dev)
+    for W in (2048, 512):
+        tensor_row(f"d24 B={B} T={T} H={H} D={D}, FP8 (e4m3) forward", W, "fwd-fp8", fwd_flops(B, T, H, D, W),
+                   timed_median(lambda: ops.attn_fwd_fp8(q8, k8, v8, ds, ds, ds, o, lse, ws8, W), reps))
+    del q8, k8, v8, o, lse, ws8
+    torch.cuda.empty_cache()
 
     cfg = inputs.WORKLOADS["d24"]
     B, T, H, D = cfg["B"], cfg["T"], cfg["H"], cfg["D"]
@@ -450,8 +478,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-log", default=None)
-    ap.add_argument("--case", default="step", choices=["step", "fwd", "bwd", "decode", "configs"],
-                    help="fwd / bwd / decode: run only that call repeatedly on a reduced batch, for profiling "
+    ap.add_argument("--case", default="step", choices=["step", "fwd", "bwd", "decode", "fp8", "configs"],
+                    help="fwd / bwd / decode / fp8: run only that call repeatedly on a reduced batch, for profiling "
                          "(no metric line); configs: standalone timing of every configuration row")
     ap.add_argument("--reps", type=int, default=20, help="timed calls per row for --case configs (>= 20)")
     ap.add_argument("--batch", type=int, default=8, help="batch for --case (d24 shape otherwise)")
