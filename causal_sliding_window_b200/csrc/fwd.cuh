@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
                                                          const int* __restrict__ cache_len, int B, int Tn, int cap,
                                                          int Hkv, int len_off, int tail, const float* __restrict__ cs,
                                                          const float* __restrict__ sn, int max_pos, float eps,
-                                                         int slot) {
+                                                         int stream_slot) {
     constexpr int CPR = D / 8;   // 16-byte chunks per head row
     const int span = Tn + tail;  // chunk rows plus the largest zeroed tail
     const long long total = (long long)B * span * Hkv * CPR;
@@ -669,7 +669,7 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
         // every branch below is uniform over the row's threads (it depends on b, t, hk only)
         if (t >= Tn && slot >= tile_end) continue;
         if (slot >= cap) {
-            if (t < Tn) report_status(slot, kStatusCacheOverflow);
+            if (t < Tn) report_status(stream_slot, kStatusCacheOverflow);
             continue;
         }
         const size_t dst = ((size_t(b) * cap + size_t(slot)) * Hkv + hk) * D + c * 8;
@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(256) swa_append_kernel(const __nv_bfloat16* __
             vw = *reinterpret_cast<const uint4*>(v_new + src);
             if (kRope) {
                 if (slot >= max_pos) {
-                    report_status(slot, kStatusPositionRange);
+                    report_status(stream_slot, kStatusPositionRange);
                     continue;
                 }
                 float f[8];

@@ -406,9 +406,16 @@ def test_prefill_overflow_is_reported_and_stays_in_bounds(ops):
     kc.t.zero_()
     vc.t.zero_()
     L = torch.tensor([0, 50], dtype=torch.int32, device="cuda")   # 50 + 64 > 100 for sequence 1
-    o, lse = ops.prefill(dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"]), kc.t, vc.t, L, W)
+    q, k, v = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    assert ops.attn_device_status(clear=True) == 0
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        o, lse = ops.prefill(q, k, v, kc.t, vc.t, L, W, stream=side)
+    assert ops.attn_poll_device_status(torch.cuda.current_stream()) == 0   # not this stream's error
+    assert ops.attn_poll_device_status(side) == -6      # ATTN_ERR_CACHE_OVERFLOW, on the launching stream
     torch.cuda.synchronize()
-    assert ops.attn_device_status(clear=True) == -6   # ATTN_ERR_CACHE_OVERFLOW
+    assert ops.attn_device_status(clear=True) == -6   # the device-wide word saw it too
     assert kc.guards_intact() and vc.guards_intact()
     ro, rl, _, _ = oracle_prefill(x["q"][:1], x["k"][:1], x["v"][:1], np.zeros((1, cap, H, D), np.uint16),
                                   np.zeros((1, cap, H, D), np.uint16), np.array([0]), W)
