@@ -113,15 +113,7 @@ __global__ void __launch_bounds__(256) swa_bwd_pre_kernel(const __nv_bfloat16* _
 
 // Store 32 fp32 values (bit patterns) of one row as bf16, times `mul`, 16 bytes at a time.
 __device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint32_t (&r)[32], float mul) {
-#pragma unroll
-    for (int v4 = 0; v4 < 4; ++v4) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * mul, __uint_as_float(r[v4 * 8 + 1]) * mul);
-        w.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * mul, __uint_as_float(r[v4 * 8 + 3]) * mul);
-        w.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * mul, __uint_as_float(r[v4 * 8 + 5]) * mul);
-        w.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * mul, __uint_as_float(r[v4 * 8 + 7]) * mul);
-        *reinterpret_cast<uint4*>(dst + v4 * 8) = w;
-    }
+    store_row_bf16<32>(dst, reinterpret_cast<const float*>(r), mul);
 }
 
 // ===========================================================================

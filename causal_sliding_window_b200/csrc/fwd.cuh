@@ -612,15 +612,7 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (qrow < T) {
                 const float inv_l = 1.f / l_run;
                 __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(qrow)) * p.H + g.h) * D;
-#pragma unroll
-                for (int v8 = 0; v8 < D / 8; ++v8) {
-                    uint4 w;
-                    w.x = pack_bf16x2(ov[v8 * 8 + 0] * inv_l, ov[v8 * 8 + 1] * inv_l);
-                    w.y = pack_bf16x2(ov[v8 * 8 + 2] * inv_l, ov[v8 * 8 + 3] * inv_l);
-                    w.z = pack_bf16x2(ov[v8 * 8 + 4] * inv_l, ov[v8 * 8 + 5] * inv_l);
-                    w.w = pack_bf16x2(ov[v8 * 8 + 6] * inv_l, ov[v8 * 8 + 7] * inv_l);
-                    *reinterpret_cast<uint4*>(orow + v8 * 8) = w;
-                }
+                store_row_bf16<D>(orow, ov, inv_l);
                 p.lse[(size_t(g.b) * p.H + g.h) * T + qrow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
             }
         }

@@ -440,15 +440,7 @@ swa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (q < T) {
                 const float mul = p.dv[size_t(g.b) * (p.H / p.G) + g.hk] / l_run;
                 __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(q)) * p.H + g.h) * D;
-#pragma unroll
-                for (int v8 = 0; v8 < D / 8; ++v8) {
-                    uint4 w;
-                    w.x = pack_bf16x2(ov[v8 * 8 + 0] * mul, ov[v8 * 8 + 1] * mul);
-                    w.y = pack_bf16x2(ov[v8 * 8 + 2] * mul, ov[v8 * 8 + 3] * mul);
-                    w.z = pack_bf16x2(ov[v8 * 8 + 4] * mul, ov[v8 * 8 + 5] * mul);
-                    w.w = pack_bf16x2(ov[v8 * 8 + 6] * mul, ov[v8 * 8 + 7] * mul);
-                    *reinterpret_cast<uint4*>(orow + v8 * 8) = w;
-                }
+                store_row_bf16<D>(orow, ov, mul);
                 p.lse[(size_t(g.b) * p.H + g.h) * T + q] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
             }
         }

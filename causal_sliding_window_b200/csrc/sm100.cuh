@@ -416,6 +416,39 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
+
+// One 32-byte global store (a whole sector); ptr must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
+// N fp32 values v[0..N) times mul, as bf16 at dst (N a multiple of 16): 32-byte stores when dst is
+// 32-byte aligned, else 16-byte ones (dst is always 16-byte aligned).  A thread writing its own
+// row this way issues half the store instructions of 16-byte stores.
+template <int N>
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float* v, float mul) {
+    if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+#pragma unroll
+        for (int k = 0; k < N / 16; ++k) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[16 * k + 2 * i] * mul, v[16 * k + 2 * i + 1] * mul);
+            st_global_v8(dst + 16 * k, w);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < N / 8; ++k) {
+            uint4 w;
+            w.x = pack_bf16x2(v[8 * k + 0] * mul, v[8 * k + 1] * mul);
+            w.y = pack_bf16x2(v[8 * k + 2] * mul, v[8 * k + 3] * mul);
+            w.z = pack_bf16x2(v[8 * k + 4] * mul, v[8 * k + 5] * mul);
+            w.w = pack_bf16x2(v[8 * k + 6] * mul, v[8 * k + 7] * mul);
+            *reinterpret_cast<uint4*>(dst + 8 * k) = w;
+        }
+    }
+}
 // Same packing on the integer pipe, for finite inputs: add half a bf16 ulp to the magnitude
 // bits and keep the high halves (round to nearest, ties away from zero; differs from
 // pack_bf16x2 only on exact ties).  Two adds and one byte permute, so the conversions of

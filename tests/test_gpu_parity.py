@@ -219,6 +219,33 @@ def test_forward_is_deterministic(ops):
     assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"])
 
 
+def test_outputs_16_byte_aligned_only(ops):
+    """O, dQ, dK, dV at addresses that are 16-byte but not 32-byte aligned: the epilogues fall back
+    from 32-byte to 16-byte stores and the results match the oracle as usual."""
+    B, T, H, D, W = 1, 300, 2, 128, 100
+    x = inputs.attention_inputs(B, T, H, D, seed=12)
+    q, k, v, do = (dev_bf16(x[n]) for n in ("q", "k", "v", "do"))
+    n = B * T * H * D
+
+    def offset_view():   # 8 bf16 = 16 bytes past a 256-byte aligned allocation
+        buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+        t = buf[8:].view(B, T, H, D)
+        assert t.data_ptr() % 32 == 16
+        return t
+
+    o, dq, dk, dv = offset_view(), offset_view(), offset_view(), offset_view()
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    ops.attn_fwd(q, k, v, o, lse, W)
+    ws = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, D), dtype=torch.uint8, device="cuda")
+    ops.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, W)
+    torch.cuda.synchronize()
+    ro, rl = oracle_fwd(x["q"], x["k"], x["v"], W)
+    assert rel_l2(host_f64(o), ro) <= O_REL
+    rdq, rdk, rdv = oracle_bwd(x["q"], x["k"], x["v"], x["do"], W)
+    for got, ref in ((dq, rdq), (dk, rdk), (dv, rdv)):
+        assert rel_l2(host_f64(got), ref) <= G_REL
+
+
 def test_bounded_wait_reports_timeout_without_hanging(ops):
     assert ops.attn_device_status(clear=True) == 0
     assert ops.attn_selftest_wait_timeout(200_000) == 0
