@@ -246,6 +246,46 @@ def test_outputs_16_byte_aligned_only(ops):
         assert rel_l2(host_f64(got), ref) <= G_REL
 
 
+def test_concurrent_streams_keep_their_own_work_counters(ops):
+    """Forward and backward launches on two streams, interleaved with no synchronisation between
+    them: each stream's persistent kernels draw work items from its own counter, so both
+    results equal (bit for bit) those of the same calls run one after another."""
+    def setup(B, T, H, seed):
+        x = inputs.attention_inputs(B, T, H, 128, seed=seed)
+        t = {n: dev_bf16(x[n]) for n in ("q", "k", "v", "do")}
+        t["o"], t["dq"], t["dk"], t["dv"] = (torch.empty_like(t["q"]) for _ in range(4))
+        t["lse"] = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+        t["ws"] = torch.empty(ops.attn_bwd_workspace_bytes(B, T, H, 128), dtype=torch.uint8, device="cuda")
+        return t
+
+    def run(t, W, stream=None):
+        ops.attn_fwd(t["q"], t["k"], t["v"], t["o"], t["lse"], W, stream=stream)
+        ops.attn_bwd(t["q"], t["k"], t["v"], t["o"], t["lse"], t["do"], t["dq"], t["dk"], t["dv"], t["ws"], W,
+                     stream=stream)
+
+    ta, tb = setup(2, 1024, 40, 31), setup(1, 700, 24, 32)   # several items per CTA in each launch
+    run(ta, 256)
+    run(tb, 1000)
+    torch.cuda.synchronize()
+    ref = {k: {n: t[n].clone() for n in ("o", "lse", "dq", "dk", "dv")} for k, t in (("a", ta), ("b", tb))}
+    for t in (ta, tb):
+        for n in ("o", "lse", "dq", "dk", "dv"):
+            t[n].zero_()
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    sa.wait_stream(torch.cuda.current_stream())
+    sb.wait_stream(torch.cuda.current_stream())
+    for _ in range(3):
+        with torch.cuda.stream(sa):
+            run(ta, 256, stream=sa)
+        with torch.cuda.stream(sb):
+            run(tb, 1000, stream=sb)
+    torch.cuda.synchronize()
+    assert ops.attn_poll_device_status(sa) == 0 and ops.attn_poll_device_status(sb) == 0
+    for k, t in (("a", ta), ("b", tb)):
+        for n in ("o", "lse", "dq", "dk", "dv"):
+            assert torch.equal(t[n], ref[k][n]), (k, n)
+
+
 def test_bounded_wait_reports_timeout_without_hanging(ops):
     assert ops.attn_device_status(clear=True) == 0
     assert ops.attn_selftest_wait_timeout(200_000) == 0
