@@ -117,6 +117,159 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int item) {
     return it;
 }
 
+// Softmax warpgroup of query tile t = warp / 4 (warps 0..7 of a forward kernel), for every item
+// of the CTA: thread = row; online softmax of S_t in the exp2 domain, P_t written back to TMEM as
+// bf16 over the first half of S_t's columns, O_t rescaled in TMEM only when a warp's running max
+// grows by more than 2^8, then the epilogue O / l and lse.  kDown: the item's key tiles arrive
+// from the band's last to its first (the order the kernel's MMAs use).  The barriers are those of
+// tile t.
+template <int D, bool kOffset, bool kDown>
+__device__ __forceinline__ void fwd_softmax_warpgroup(const FwdParams& p, uint32_t tS_t, uint32_t tO_t,
+                                                      uint32_t s_full, uint32_t p_full, uint32_t o_full,
+                                                      uint32_t o_free, volatile int* ring, uint32_t item_full0,
+                                                      uint32_t item_empty0, volatile int* abort_flag) {
+using C = FwdCfg<D>;
+const int T = p.T;
+const long long W = p.W;
+const int warp = warp_id(), lane = lane_id();
+const int t = warp >> 2;            // query tile of this warpgroup
+const int quarter = warp & 3;       // TMEM lane quarter this warp may access
+const int row = quarter * 32 + lane;
+const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+const uint32_t tS = tS_t + lane_off, tO = tO_t + lane_off;
+    const float sl2 = p.scale_log2;
+    int ns = 0;      // S tiles consumed so far (all items): parity of s_full / o_full
+    bool ok = true;
+    for (int k = 0;; ++k) {
+        const int item = item_consume_warp(k, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                           kStatusTimeoutSoftmax, ok);
+        if (!ok || item >= p.n_items) break;
+        const FwdItem g = fwd_item<kOffset>(p, item);
+        if (t == 1 && !g.valid1) continue;
+        const long long qt0 = g.q0 + t * 128;    // first row of this tile
+        const long long q = qt0 + row;           // query row of this thread (position g.L + q)
+        const int jlo = t ? g.jlo1 : g.jlo0, jhi = t ? g.jhi1 : g.jhi0;
+        float m_run = -INFINITY, l_run = 0.f;
+        int nloc = 0;
+        for (int j = kDown ? jhi : jlo; (kDown ? j >= jlo : j <= jhi) && ok; j += kDown ? -1 : 1, ++ns, ++nloc) {
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(s_full, uint32_t(ns & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
+            if (!ok) break;
+            tc_fence_after();
+            // All 128 columns are requested before the single wait, so the TMEM load
+            // latency is paid once per tile.
+            float s[C::BN];
+            {
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(tS, r0);
+                tmem_ld32(tS + 32, r1);
+                tmem_ld32(tS + 64, r2);
+                tmem_ld32(tS + 96, r3);
+                tmem_ld_wait(r0);
+                tmem_ld_wait(r1);
+                tmem_ld_wait(r2);
+                tmem_ld_wait(r3);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    s[i] = __uint_as_float(r0[i]);
+                    s[32 + i] = __uint_as_float(r1[i]);
+                    s[64 + i] = __uint_as_float(r2[i]);
+                    s[96 + i] = __uint_as_float(r3[i]);
+                }
+            }
+            // Tiles that cut the diagonal or the window's left edge: keep columns clo..chi of this
+            // row (keys k0+c with q-W < k0+c <= q).  The test is uniform across the CTA.
+            // k0: the key tile's first position, counted like the query rows (absolute - g.L)
+            const long long k0 = (long long)j * C::BN - g.L;
+            const bool full = (k0 + C::BN - 1 <= qt0) && (k0 > qt0 + C::BM - 1 - W);
+            if (!full) {
+                const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN));
+                const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1));
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) s[c] = (c >= clo && c <= chi) ? s[c] : -INFINITY;
+            }
+            // Row max and row sum over 8 independent partials (short dependency chains).
+            float mp[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mp[u] = s[u];
+#pragma unroll
+            for (int c = 8; c < C::BN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+            const float m_tile = mx * sl2;
+            const float m_new = fmaxf(m_run, m_tile);
+            const bool need = m_new > m_run + 8.0f;
+            const bool warp_need = __any_sync(0xffffffffu, need);
+            const float m_use = warp_need ? m_new : m_run;
+            const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+            const float alpha = (m_use == -INFINITY) ? 1.f : ex2_approx(m_run - m_use);
+            float sp[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sp[u] = 0.f;
+#pragma unroll
+            for (int c = 0; c < C::BN / 64; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_sub));
+                    const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
+                    sp[(2 * i) & 7] += p0;
+                    sp[(2 * i + 1) & 7] += p1;
+                    pk[i] = pack_bf16x2_alu(p0, p1);   // integer pipe: exp2 keeps the SFU
+                }
+                tmem_st32(tS + c * 32, pk);
+            }
+            const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            l_run = l_run * alpha + rowsum;
+            tmem_st_wait();
+            if (warp_need && nloc > 0) {
+                // O_t holds the sum over the key tiles walked before j: wait for their PV_t, then rescale.
+                ok = __all_sync(0xffffffffu, mbar_wait(o_full, uint32_t((ns - 1) & 1), abort_flag,
+                                                       p.wait_limit, kStatusTimeoutSoftmax));
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tO + c * 32, r);
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(tO + c * 32, r);
+                }
+                tmem_st_wait();
+            }
+            m_run = m_use;
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (!ok || nloc == 0) break;
+        // ---- epilogue: O = O / l, lse = ln(sum exp S) ----
+        ok = __all_sync(0xffffffffu, mbar_wait(o_full, uint32_t((ns - 1) & 1), abort_flag, p.wait_limit,
+                                               kStatusTimeoutEpilogue));
+        if (!ok) break;
+        tc_fence_after();
+        float ov[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[c * 32 + i] = __uint_as_float(r[i]);
+        }
+        tc_fence_before();
+        mbar_arrive(o_free);   // the next item's first PV may overwrite O_t now
+        const long long qrow = q;
+        if (qrow < T) {
+            const float inv_l = 1.f / l_run;
+            __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(qrow)) * p.H + g.h) * D;
+            store_row_bf16<D>(orow, ov, inv_l);
+            p.lse[(size_t(g.b) * p.H + g.h) * T + qrow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+        }
+    }
+}
+
 // kOffset: chunked prefill (query rows start at q_offset[b]); false for training, where the
 // offset is zero and costs nothing.  kRope: the rotary + QK-norm prologue of the queries runs
 // inside the kernel (warps 10 and 11), on each Q tile in shared memory between its load and the
@@ -155,8 +308,6 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
     volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
 
-    const int T = p.T;
-    const long long W = p.W;
     const int warp = warp_id(), lane = lane_id();
 
     if (threadIdx.x == 0) {
@@ -480,142 +631,261 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (pt == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // stores complete before exit
     } else {
         // ------------------------------ softmax warpgroups ------------------------------
-        const int t = warp >> 2;            // query tile of this warpgroup
-        const int quarter = warp & 3;       // TMEM lane quarter this warp may access
-        const int row = quarter * 32 + lane;
-        const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-        const uint32_t tS = (t ? tS1 : tS0) + lane_off, tO = (t ? tO1 : tO0) + lane_off;
-        const float sl2 = p.scale_log2;
-        int ns = 0;      // S tiles consumed so far (all items): parity of s_full / o_full
-        bool ok = true;
-        for (int k = 0;; ++k) {
-            const int item = item_consume_warp(k, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
-                                               kStatusTimeoutSoftmax, ok);
-            if (!ok || item >= p.n_items) break;
-            const FwdItem g = fwd_item<kOffset>(p, item);
-            if (t == 1 && !g.valid1) continue;
-            const long long qt0 = g.q0 + t * 128;    // first row of this tile
-            const long long q = qt0 + row;           // query row of this thread (position g.L + q)
-            const int jlo = t ? g.jlo1 : g.jlo0, jhi = t ? g.jhi1 : g.jhi0;
-            float m_run = -INFINITY, l_run = 0.f;
-            int nloc = 0;
-            for (int j = jlo; j <= jhi && ok; ++j, ++ns, ++nloc) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(s_full(t), uint32_t(ns & 1), abort_flag, p.wait_limit, kStatusTimeoutSoftmax));
-                if (!ok) break;
-                tc_fence_after();
-                // All 128 columns are requested before the single wait, so the TMEM load
-                // latency is paid once per tile.
-                float s[C::BN];
-                {
-                    uint32_t r0[32], r1[32], r2[32], r3[32];
-                    tmem_ld32(tS, r0);
-                    tmem_ld32(tS + 32, r1);
-                    tmem_ld32(tS + 64, r2);
-                    tmem_ld32(tS + 96, r3);
-                    tmem_ld_wait(r0);
-                    tmem_ld_wait(r1);
-                    tmem_ld_wait(r2);
-                    tmem_ld_wait(r3);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        s[i] = __uint_as_float(r0[i]);
-                        s[32 + i] = __uint_as_float(r1[i]);
-                        s[64 + i] = __uint_as_float(r2[i]);
-                        s[96 + i] = __uint_as_float(r3[i]);
-                    }
-                }
-                // Tiles that cut the diagonal or the window's left edge: keep columns clo..chi of this
-                // row (keys k0+c with q-W < k0+c <= q).  The test is uniform across the CTA.
-                // k0: the key tile's first position, counted like the query rows (absolute - g.L)
-                const long long k0 = (long long)j * C::BN - g.L;
-                const bool full = (k0 + C::BN - 1 <= qt0) && (k0 > qt0 + C::BM - 1 - W);
-                if (!full) {
-                    const int chi = int(imin_ll(imax_ll(q - k0, -1), C::BN));
-                    const int clo = int(imin_ll(imax_ll(q - W + 1 - k0, 0), C::BN + 1));
-#pragma unroll
-                    for (int c = 0; c < C::BN; ++c) s[c] = (c >= clo && c <= chi) ? s[c] : -INFINITY;
-                }
-                // Row max and row sum over 8 independent partials (short dependency chains).
-                float mp[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) mp[u] = s[u];
-#pragma unroll
-                for (int c = 8; c < C::BN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-                const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-                const float m_tile = mx * sl2;
-                const float m_new = fmaxf(m_run, m_tile);
-                const bool need = m_new > m_run + 8.0f;
-                const bool warp_need = __any_sync(0xffffffffu, need);
-                const float m_use = warp_need ? m_new : m_run;
-                const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-                const float alpha = (m_use == -INFINITY) ? 1.f : ex2_approx(m_run - m_use);
-                float sp[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) sp[u] = 0.f;
-#pragma unroll
-                for (int c = 0; c < C::BN / 64; ++c) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_sub));
-                        const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
-                        sp[(2 * i) & 7] += p0;
-                        sp[(2 * i + 1) & 7] += p1;
-                        pk[i] = pack_bf16x2_alu(p0, p1);   // integer pipe: exp2 keeps the SFU
-                    }
-                    tmem_st32(tS + c * 32, pk);
-                }
-                const float rowsum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-                l_run = l_run * alpha + rowsum;
-                tmem_st_wait();
-                if (warp_need && nloc > 0) {
-                    // O_t holds the sum up to key tile j-1: wait for PV_t(j-1), then rescale.
-                    ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((ns - 1) & 1), abort_flag,
-                                                           p.wait_limit, kStatusTimeoutSoftmax));
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(tO + c * 32, r);
-                        tmem_ld_wait(r);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(tO + c * 32, r);
-                    }
-                    tmem_st_wait();
-                }
-                m_run = m_use;
-                tc_fence_before();
-                mbar_arrive(p_full(t));
-            }
-            if (!ok || nloc == 0) break;
-            // ---- epilogue: O = O / l, lse = ln(sum exp S) ----
-            ok = __all_sync(0xffffffffu, mbar_wait(o_full(t), uint32_t((ns - 1) & 1), abort_flag, p.wait_limit,
-                                                   kStatusTimeoutEpilogue));
-            if (!ok) break;
-            tc_fence_after();
-            float ov[D];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tO + c * 32, r);
-                tmem_ld_wait(r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) ov[c * 32 + i] = __uint_as_float(r[i]);
-            }
-            tc_fence_before();
-            mbar_arrive(o_free(t));   // the next item's first PV may overwrite O_t now
-            const long long qrow = q;
-            if (qrow < T) {
-                const float inv_l = 1.f / l_run;
-                __nv_bfloat16* orow = p.o + ((size_t(g.b) * T + size_t(qrow)) * p.H + g.h) * D;
-                store_row_bf16<D>(orow, ov, inv_l);
-                p.lse[(size_t(g.b) * p.H + g.h) * T + qrow] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
-            }
+        const int t = warp >> 2;
+        fwd_softmax_warpgroup<D, kOffset, false>(p, t ? tS1 : tS0, t ? tO1 : tO0, s_full(t), p_full(t), o_full(t),
+                                                 o_free(t), ring, item_full0, item_empty0, abort_flag);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Forward for windows shorter than the sequence (W < T; training, no offset, no prologue).
+// Same tiles, K/V ring and TMEM plan as swa_fwd_kernel, with one MMA issuer thread per query
+// tile (warps 9 and 10) and the key tiles of an item walked from the last to the first: tile 1
+// alone at the item's last key tile (the diagonal of its rows), both tiles on the same key tile
+// through the middle, tile 0 alone at the first (the window's edge of its rows).  The issuer of
+// a tile that has finished its item goes on to the next one, so tile 1 starts the next item
+// while tile 0 finishes this one, instead of idling for that key step.  Each issuer walks the
+// ring on its own and releases every entry once (after its MMAs that read it, or at once for a
+// key tile outside its band); each query tile has its own Q buffer.  With W >= T both tiles
+// start at key tile 0 and tile 0 would lead tile 1 through the item, holding twice the ring
+// entries; swa_fwd_kernel (one issuer, lockstep order) serves that case.
+// ---------------------------------------------------------------------------
+template <int D>
+struct FwdShortCfg : FwdCfg<D> {
+    // kv_full, kv_empty per stage; q_full, q_empty, q_ready, s_full, p_full, o_full, o_free, mma_done
+    // per tile; item_full, item_empty per entry of the item ring
+    static constexpr int NUM_BAR = 2 * FwdCfg<D>::NSTAGE + 8 * FwdCfg<D>::NQ + 2 * kItemRing;
+    static constexpr int OFF_MISC = FwdCfg<D>::OFF_BAR + NUM_BAR * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 64;
+    static constexpr int SMEM = SMEM_USED + 1024 <= 232448 ? SMEM_USED + 1024 : 232448;
+    static constexpr int THREADS = 352;   // softmax 0..7, producer 8, MMA issuers 9 and 10
+    static_assert(SMEM_USED <= 232448, "shared memory");
+};
+
+template <int D>
+__global__ void __launch_bounds__(FwdShortCfg<D>::THREADS, 1)
+swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using C = FwdShortCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    if (int(base - raw) + C::SMEM_USED > C::SMEM) {   // uniform across the CTA: nothing started yet
+        if (threadIdx.x == 0) report_status(p.stream_slot, kStatusSmemLayout);
+        return;
+    }
+    const uint32_t sQ = base + C::OFF_Q;
+    const uint32_t sKV = base + C::OFF_KV;
+    const uint32_t bar0 = base + C::OFF_BAR;
+    auto kv_full = [&](int s) { return bar0 + 8u * s; };
+    auto kv_empty = [&](int s) { return bar0 + 8u * (C::NSTAGE + s); };
+    const uint32_t bt = bar0 + 8u * (2 * C::NSTAGE);   // per-tile barriers start here
+    auto q_full = [&](int t) { return bt + 8u * t; };
+    auto q_empty = [&](int t) { return bt + 8u * (C::NQ + t); };
+    auto s_full = [&](int t) { return bt + 8u * (3 * C::NQ + t); };
+    auto p_full = [&](int t) { return bt + 8u * (4 * C::NQ + t); };
+    auto o_full = [&](int t) { return bt + 8u * (5 * C::NQ + t); };
+    auto o_free = [&](int t) { return bt + 8u * (6 * C::NQ + t); };
+    auto mma_done = [&](int t) { return bt + 8u * (7 * C::NQ + t); };
+    const uint32_t item_full0 = bt + 8u * (8 * C::NQ), item_empty0 = item_full0 + 8u * kItemRing;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
+    volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
+    const int warp = warp_id(), lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(kv_full(s), 1);
+            mbar_init(kv_empty(s), 2);   // both MMA issuers
         }
+        for (int t = 0; t < C::NQ; ++t) {
+            mbar_init(q_full(t), 1);
+            mbar_init(q_empty(t), 1);
+            mbar_init(s_full(t), 1);
+            mbar_init(p_full(t), 128);
+            mbar_init(o_full(t), 1);
+            mbar_init(o_free(t), 128);
+            mbar_init(mma_done(t), 1);
+        }
+        for (int e = 0; e < kItemRing; ++e) {
+            mbar_init(item_full0 + 8u * e, 1);
+            mbar_init(item_empty0 + 8u * e, 2 + 8);   // the MMA threads and the softmax warps
+        }
+        abort_flag[0] = 0;
+        abort_flag[1] = p.stream_slot;   // read by a wait that gives up
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS0 = tmem, tS1 = tmem + 128u;
+    const uint32_t tO0 = tmem + 256u, tO1 = tmem + 256u + uint32_t(D);
+
+    if (warp == 8) {
+        // ------------------------------ TMA producer ------------------------------
+        // Key tiles are walked from the last (jend) down to the first (jbeg).  Per item: Q_1 (tile 1
+        // is the one active at jend), K and V of the first key tile walked, Q_0, then the remaining
+        // K / V tiles.
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            int it = 0;
+            int nq[2] = {0, 0};   // Q tiles loaded per query tile
+            bool ok = true;
+            auto load_q = [&](const FwdItem& g, int t) -> bool {
+                if (nq[t] > 0 && !(ok = mbar_wait(q_empty(t), uint32_t((nq[t] - 1) & 1), abort_flag, p.wait_limit,
+                                                  kStatusTimeoutProducer)))
+                    return false;
+                mbar_arrive_expect_tx(q_full(t), C::TILE);
+                for (int x = 0; x < C::NBOX; ++x)
+                    tma_load_4d(sQ + t * C::TILE + x * C::BOX, &tm_q, q_full(t), x * 64, g.h, int(g.q0) + t * 128, g.b);
+                ++nq[t];
+                return true;
+            };
+            for (int qi = 0;; ++qi) {
+                const int item =
+                    item_produce(p.stream_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
+                if (!ok || item >= p.n_items) break;
+                const FwdItem g = fwd_item<false>(p, item);
+                const int tf = g.valid1 ? 1 : 0;   // the tile active at jend
+                if (!load_q(g, tf)) break;
+                bool q0 = tf == 0;   // tile 0's Q is issued
+                for (int j = g.jend; j >= g.jbeg && ok; --j) {
+                    for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
+                        const int s = it % C::NSTAGE;
+                        const uint32_t ph = (it / C::NSTAGE) & 1;
+                        ok = mbar_wait(kv_empty(s), ph ^ 1u, abort_flag, p.wait_limit, kStatusTimeoutProducer);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(kv_full(s), C::TILE);
+                        const CUtensorMap* m = kv ? &tm_v : &tm_k;
+                        for (int x = 0; x < C::NBOX; ++x)
+                            tma_load_4d(sKV + s * C::TILE + x * C::BOX, m, kv_full(s), x * 64, g.hk, j * C::BN, g.b);
+                    }
+                    if (ok && !q0 && !(q0 = load_q(g, 0))) break;
+                }
+            }
+            work_slot_finish(p.stream_slot);
+            // Drain: make sure no copy is still landing when the CTA exits.
+            for (int s = 0; s < C::NSTAGE && s < it; ++s) {
+                const int fills = (it - s + C::NSTAGE - 1) / C::NSTAGE;
+                mbar_drain(kv_full(s), uint32_t((fills - 1) & 1), p.wait_limit, p.stream_slot);
+            }
+            for (int t = 0; t < C::NQ; ++t)
+                if (nq[t] > 0) mbar_drain(q_full(t), uint32_t((nq[t] - 1) & 1), p.wait_limit, p.stream_slot);
+        }
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------ MMA issuers, one per query tile ------------------------------
+        if (lane == 0) {
+            const int t = warp - 9;
+            const uint32_t tS = t ? tS1 : tS0, tO = t ? tO1 : tO0;
+            bool ok = true;
+            int it = 0;    // ring entries passed (used or not)
+            int npv = 0;   // PV MMAs issued (all items)
+            int nep = 0;   // items of this tile (= epilogues owed)
+            int nq = 0;    // Q tiles waited for
+            auto issue_s = [&](int stage) {
+                const SDesc qd = sdesc_sw128_w(sQ + t * C::TILE, 16, 1024);
+                const SDesc kd = sdesc_sw128_w(sKV + stage * C::TILE, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * C::BOX + (kk & 3) * 32) >> 4;
+                    mma_ss_w(tS, qd.lo + off, qd.hi, kd.lo + off, kd.hi, C::IDESC_S, kk > 0);
+                }
+                tc_commit(s_full(t));
+            };
+            auto issue_pv = [&](int stage, bool first) {
+                const SDesc vd = sdesc_sw128_w(sKV + stage * C::TILE, C::BOX, 1024);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    mma_ts_w(tO, tS + kk * 8, vd.lo + kk * (2048 >> 4), vd.hi, C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+                tc_commit(o_full(t));
+            };
+            auto take = [&](int& stage) -> bool {   // the next ring entry has landed
+                stage = it % C::NSTAGE;
+                ok = mbar_wait(kv_full(stage), uint32_t((it / C::NSTAGE) & 1), abort_flag, p.wait_limit,
+                               kStatusTimeoutMma);
+                ++it;
+                return ok;
+            };
+            auto pass = [&](int n) -> bool {   // n ring entries this tile does not read: release them
+                for (int i = 0; i < n; ++i) {
+                    int s;
+                    if (!take(s)) return false;
+                    mbar_arrive(kv_empty(s));
+                }
+                return true;
+            };
+            // S_t overwrites the columns the last PV_t read P from; both are issued by this thread,
+            // and the MMAs of one thread execute in issue order, so S_t needs no wait for PV_t.
+            for (int qi = 0;; ++qi) {
+                const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
+                                                     kStatusTimeoutMma, ok);
+                if (!ok || item >= p.n_items) break;
+                const FwdItem g = fwd_item<false>(p, item);
+                if (t == 1 && !g.valid1) {
+                    if (!pass(2 * (g.jend - g.jbeg + 1))) break;
+                    continue;
+                }
+                const int jlo = t ? g.jlo1 : g.jlo0, jhi = t ? g.jhi1 : g.jhi0;
+                if (!pass(2 * (g.jend - jhi))) break;   // key tiles above this tile's band
+                if (!(ok = mbar_wait(q_full(t), uint32_t(nq & 1), abort_flag, p.wait_limit,
+                                     kStatusTimeoutMma)))
+                    break;
+                ++nq;
+                int sk;
+                if (!take(sk)) break;
+                tc_fence_after();
+                issue_s(sk);
+                if (jlo == jhi) tc_commit(q_empty(t));
+                for (int j = jhi; j >= jlo && ok; --j) {
+                    int sv, sk_next = 0;
+                    const bool more = j > jlo;
+                    if (!take(sv) || (more && !take(sk_next))) break;
+                    if (!(ok = mbar_wait(p_full(t), uint32_t(npv & 1), abort_flag, p.wait_limit, kStatusTimeoutMma)))
+                        break;
+                    // O_t is overwritten by the item's first PV: the previous epilogue must have read it.
+                    if (j == jhi && nep > 0 &&
+                        !(ok = mbar_wait(o_free(t), uint32_t((nep - 1) & 1), abort_flag, p.wait_limit,
+                                         kStatusTimeoutMma)))
+                        break;
+                    tc_fence_after();
+                    issue_pv(sv, j == jhi);
+                    ++npv;
+                    if (more) {
+                        issue_s(sk_next);
+                        if (j - 1 == jlo) tc_commit(q_empty(t));   // the item's last S of this tile
+                    }
+                    // K_j (read by the S MMA issued one step earlier) and V_j are free once this
+                    // thread's MMAs issued so far complete.
+                    tc_commit(kv_empty(sk));
+                    tc_commit(kv_empty(sv));
+                    sk = sk_next;
+                }
+                if (!ok) break;
+                if (!pass(2 * (jlo - g.jbeg))) break;   // key tiles below this tile's band
+                ++nep;
+            }
+            tc_commit(mma_done(t));
+            mbar_wait(mma_done(t), 0, abort_flag, p.wait_limit, kStatusTimeoutMma);
+        }
+    } else if (warp < 8) {
+        // ------------------------------ softmax warpgroups ------------------------------
+        const int t = warp >> 2;
+        fwd_softmax_warpgroup<D, false, true>(p, t ? tS1 : tS0, t ? tO1 : tO0, s_full(t), p_full(t), o_full(t),
+                                              o_free(t), ring, item_full0, item_empty0, abort_flag);
     }
 
     tc_fence_before();

@@ -226,7 +226,18 @@ static int launch_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v
         swa_fwd_kernel<DD, OO, RR><<<unsigned(grid), FwdCfg<DD>::threads(RR), FwdCfg<DD>::SMEM, s>>>(mq, mk, mv, \
                                                                                                        mqr, p);  \
     } while (0)
-    if (D == 128) {
+    // Windows shorter than the sequence (training, no prologue): one MMA issuer per query tile and
+    // the key tiles walked downwards, so consecutive items overlap at their solo key steps.
+#define SWA_FWD_SHORT(DD)                                                                                         \
+    do {                                                                                                          \
+        if (!ensure_smem((const void*)swa_fwd_short_kernel<DD>, FwdShortCfg<DD>::SMEM)) return ATTN_ERR_LAUNCH;  \
+        swa_fwd_short_kernel<DD><<<unsigned(grid), FwdShortCfg<DD>::THREADS, FwdShortCfg<DD>::SMEM, s>>>(mq, mk, \
+                                                                                                         mv, p);  \
+    } while (0)
+    const bool short_window = !off && !r && (long long)W < T;
+    if (short_window) {
+        if (D == 128) SWA_FWD_SHORT(128); else SWA_FWD_SHORT(64);
+    } else if (D == 128) {
         if (off) {
             if (r) SWA_FWD(128, true, true); else SWA_FWD(128, true, false);
         } else {
@@ -240,6 +251,7 @@ static int launch_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v
         }
     }
 #undef SWA_FWD
+#undef SWA_FWD_SHORT
     return launch_status();
 }
 
