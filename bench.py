@@ -88,7 +88,9 @@ def load_peaks():
 PROFILE_FOR_KERNEL = {
     "swa_bwd_dkdv_kernel<128>": "swa_bwd_dkdv_kernel_d24shape_b8.md",
     "swa_bwd_dq_kernel<128>": "swa_bwd_dq_kernel_d24shape_b8.md",
-    "swa_fwd_kernel<128>": "swa_fwd_kernel_d24shape_b8.md",
+    # the forward runs swa_fwd_short_kernel for W < T and swa_fwd_kernel otherwise; one summary
+    # covers both, per window
+    "swa_fwd_short_kernel<128> (W < T) / swa_fwd_kernel<128>": "swa_fwd_kernel_d24shape_b8.md",
     "swa_decode_kernel<128>": "swa_decode_kernel_decode_workload.md",
 }
 
@@ -658,7 +660,8 @@ def main():
         peak_t = peaks.get(peak_kind, FALLBACK_PEAKS[peak_kind])
         peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         if dominant == "fwd_ms":
-            roof = {"kernel": "swa_fwd_kernel<128>", "bound": "tensor", "achieved": fwd_tf, "peak": peak_t,
+            roof = {"kernel": "swa_fwd_short_kernel<128> (W < T) / swa_fwd_kernel<128>", "bound": "tensor",
+                    "achieved": fwd_tf, "peak": peak_t,
                     "unit": "TFLOP/s"}
         elif dominant == "decode_ms":
             roof = {"kernel": "swa_decode_kernel<128>", "bound": "hbm", "achieved": dec_gbs, "peak": peak_h,
