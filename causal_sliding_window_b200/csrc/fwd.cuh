@@ -215,7 +215,9 @@ const uint32_t tS = tS_t + lane_off, tO = tO_t + lane_off;
                     const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_sub));
                     sp[(2 * i) & 7] += p0;
                     sp[(2 * i + 1) & 7] += p1;
-                    pk[i] = pack_bf16x2_alu(p0, p1);   // integer pipe: exp2 keeps the SFU
+                    // bf16 rounding of P: one cvt per pair in the short-window kernel, three integer
+                    // instructions (round half up) in the lockstep one; each measured the faster there.
+                    pk[i] = kDown ? pack_bf16x2(p0, p1) : pack_bf16x2_alu(p0, p1);
                 }
                 tmem_st32(tS + c * 32, pk);
             }
