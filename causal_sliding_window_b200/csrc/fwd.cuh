@@ -657,6 +657,14 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // start at key tile 0 and tile 0 would lead tile 1 through the item, holding twice the ring
 // entries; swa_fwd_kernel (one issuer, lockstep order) serves that case.
 // ---------------------------------------------------------------------------
+// The other MMA issuer held the issue token through 2^27 attempts (about a second): record the
+// timeout and stop (see swa_fwd_short_kernel).
+__device__ __noinline__ bool token_gave_up(volatile int* abort_flag) {
+    abort_flag[0] = 1;
+    report_status(abort_flag[1], kStatusTimeoutMma);
+    return false;
+}
+
 template <int D>
 struct FwdShortCfg : FwdCfg<D> {
     // kv_full, kv_empty per stage; q_full, q_empty, q_ready, s_full, p_full, o_full, o_free, mma_done
@@ -699,6 +707,10 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 16);
     volatile int* ring = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 32);
+    // Issue token of the two MMA issuers (0 free, 1 held): each holds it while it issues one
+    // P*V + S group, so that the groups reach the tensor pipe one after the other instead of
+    // interleaved, which would delay both tiles' S.
+    int* mma_token = reinterpret_cast<int*>(gbase + C::OFF_MISC + 48);
     const int warp = warp_id(), lane = lane_id();
 
     if (threadIdx.x == 0) {
@@ -721,6 +733,7 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         abort_flag[0] = 0;
         abort_flag[1] = p.stream_slot;   // read by a wait that gives up
+        *mma_token = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
@@ -830,6 +843,13 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 return true;
             };
+            auto acquire = [&]() -> bool {   // the issue token, within a bounded number of attempts
+                if (atomicCAS(mma_token, 0, 1) == 0) return true;
+                for (uint32_t n = 0; atomicCAS(mma_token, 0, 1) != 0;)
+                    if (++n > (1u << 27)) return ok = token_gave_up(abort_flag);
+                return true;
+            };
+            auto release = [&]() { atomicExch(mma_token, 0); };
             // S_t overwrites the columns the last PV_t read P from; both are issued by this thread,
             // and the MMAs of one thread execute in issue order, so S_t needs no wait for PV_t.
             for (int qi = 0;; ++qi) {
@@ -848,9 +868,10 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     break;
                 ++nq;
                 int sk;
-                if (!take(sk)) break;
+                if (!take(sk) || !acquire()) break;
                 tc_fence_after();
                 issue_s(sk);
+                release();
                 if (jlo == jhi) tc_commit(q_empty(t));
                 for (int j = jhi; j >= jlo && ok; --j) {
                     int sv, sk_next = 0;
@@ -863,6 +884,7 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         !(ok = mbar_wait(o_free(t), uint32_t((nep - 1) & 1), abort_flag, p.wait_limit,
                                          kStatusTimeoutMma)))
                         break;
+                    if (!acquire()) break;
                     tc_fence_after();
                     issue_pv(sv, j == jhi);
                     ++npv;
@@ -870,6 +892,7 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         issue_s(sk_next);
                         if (j - 1 == jlo) tc_commit(q_empty(t));   // the item's last S of this tile
                     }
+                    release();
                     // K_j (read by the S MMA issued one step earlier) and V_j are free once this
                     // thread's MMAs issued so far complete.
                     tc_commit(kv_empty(sk));
