@@ -645,7 +645,8 @@ swa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 // ---------------------------------------------------------------------------
-// Forward for windows shorter than the sequence (W < T; training, no offset, no prologue).
+// Forward for windows shorter than the sequence (W < T in training, W shorter than the cache in
+// chunked prefill, kOffset; no prologue).
 // Same tiles, K/V ring and TMEM plan as swa_fwd_kernel, with one MMA issuer thread per query
 // tile (warps 9 and 10) and the key tiles of an item walked from the last to the first: tile 1
 // alone at the item's last key tile (the diagonal of its rows), both tiles on the same key tile
@@ -677,7 +678,7 @@ struct FwdShortCfg : FwdCfg<D> {
     static_assert(SMEM_USED <= 232448, "shared memory");
 };
 
-template <int D>
+template <int D, bool kOffset = false>
 __global__ void __launch_bounds__(FwdShortCfg<D>::THREADS, 1)
 swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -774,7 +775,7 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int item =
                     item_produce(p.stream_slot, qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit, ok);
                 if (!ok || item >= p.n_items) break;
-                const FwdItem g = fwd_item<false>(p, item);
+                const FwdItem g = fwd_item<kOffset>(p, item);
                 const int tf = g.valid1 ? 1 : 0;   // the tile active at jend
                 if (!load_q(g, tf)) break;
                 bool q0 = tf == 0;   // tile 0's Q is issued
@@ -856,7 +857,7 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int item = item_consume_thread(qi, ring, item_full0, item_empty0, abort_flag, p.wait_limit,
                                                      kStatusTimeoutMma, ok);
                 if (!ok || item >= p.n_items) break;
-                const FwdItem g = fwd_item<false>(p, item);
+                const FwdItem g = fwd_item<kOffset>(p, item);
                 if (t == 1 && !g.valid1) {
                     if (!pass(2 * (g.jend - g.jbeg + 1))) break;
                     continue;
@@ -909,7 +910,7 @@ swa_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     } else if (warp < 8) {
         // ------------------------------ softmax warpgroups ------------------------------
         const int t = warp >> 2;
-        fwd_softmax_warpgroup<D, false, true>(p, t ? tS1 : tS0, t ? tO1 : tO0, s_full(t), p_full(t), o_full(t),
+        fwd_softmax_warpgroup<D, kOffset, true>(p, t ? tS1 : tS0, t ? tO1 : tO0, s_full(t), p_full(t), o_full(t),
                                               o_free(t), ring, item_full0, item_empty0, abort_flag);
     }
 

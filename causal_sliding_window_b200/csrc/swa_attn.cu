@@ -226,17 +226,22 @@ static int launch_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v
         swa_fwd_kernel<DD, OO, RR><<<unsigned(grid), FwdCfg<DD>::threads(RR), FwdCfg<DD>::SMEM, s>>>(mq, mk, mv, \
                                                                                                        mqr, p);  \
     } while (0)
-    // Windows shorter than the sequence (training, no prologue): one MMA issuer per query tile and
-    // the key tiles walked downwards, so consecutive items overlap at their solo key steps.
-#define SWA_FWD_SHORT(DD)                                                                                         \
+    // Windows shorter than the sequence (training) or than the cache (chunked prefill), no prologue:
+    // one MMA issuer per query tile and the key tiles walked downwards, so consecutive items overlap
+    // at their solo key steps.
+#define SWA_FWD_SHORT(DD, OO)                                                                                     \
     do {                                                                                                          \
-        if (!ensure_smem((const void*)swa_fwd_short_kernel<DD>, FwdShortCfg<DD>::SMEM)) return ATTN_ERR_LAUNCH;  \
-        swa_fwd_short_kernel<DD><<<unsigned(grid), FwdShortCfg<DD>::THREADS, FwdShortCfg<DD>::SMEM, s>>>(mq, mk, \
-                                                                                                         mv, p);  \
+        if (!ensure_smem((const void*)swa_fwd_short_kernel<DD, OO>, FwdShortCfg<DD>::SMEM)) return ATTN_ERR_LAUNCH; \
+        swa_fwd_short_kernel<DD, OO><<<unsigned(grid), FwdShortCfg<DD>::THREADS, FwdShortCfg<DD>::SMEM, s>>>(    \
+            mq, mk, mv, p);                                                                                       \
     } while (0)
-    const bool short_window = !off && !r && (long long)W < T;
+    const bool short_window = !r && (long long)W < (off ? Tk : T);
     if (short_window) {
-        if (D == 128) SWA_FWD_SHORT(128); else SWA_FWD_SHORT(64);
+        if (D == 128) {
+            if (off) SWA_FWD_SHORT(128, true); else SWA_FWD_SHORT(128, false);
+        } else {
+            if (off) SWA_FWD_SHORT(64, true); else SWA_FWD_SHORT(64, false);
+        }
     } else if (D == 128) {
         if (off) {
             if (r) SWA_FWD(128, true, true); else SWA_FWD(128, true, false);
