@@ -1,4 +1,4 @@
-// fwd.cuh -- forward kernel: O and logsumexp of causal sliding-window attention.
+// fwd.cuh -- forward kernels: O and logsumexp of causal sliding-window attention.
 //
 // The operation is the one nanochat's GPT calls once per layer,
 // flash_attn_func(q, k, v, causal=True, window_size=W) (apidog guide "Train
@@ -22,6 +22,10 @@
 // The next item's Q load and first S MMAs overlap the current item's last PV
 // MMAs and epilogue.  Key tiles entirely outside the band are never loaded;
 // only tiles that cut the diagonal or the window's left edge are masked.
+// That is swa_fwd_kernel, the one MMA issuer moving both tiles in lockstep.
+// swa_fwd_short_kernel (further down) serves windows shorter than the sequence:
+// one issuer per tile and a downward walk, so consecutive items overlap.  Both
+// use the same softmax warpgroup (fwd_softmax_warpgroup).
 #pragma once
 
 #include "rope.cuh"
